@@ -1,0 +1,975 @@
+/*
+ * llvq_oracle.c -- plain CPU oracle for LLVQ (Leech lattice vector quantization).
+ *
+ * TEST INFRASTRUCTURE ONLY: used by the tests, the package smoke check and the bench's
+ * CPU-baseline leg, never by the product path.  It shares nothing with the CUDA library.
+ *
+ * Everything here is written for clarity, not speed: exact unsigned 128-bit integer
+ * arithmetic for indices, fp64 for the matrix-vector product, linear scans where a scan
+ * is the plainest statement of a step.
+ *
+ * Page references ("Leech Lattice Vector Quantization for Efficient LLM Compression"):
+ *   [notes-K1]  papernotes.org, 方法详解 / 关键设计 1: shells of norm^2 2m, union m = 2..M,
+ *               shape-gain split with unit directions x/|x|.
+ *   [notes-K2]  papernotes.org, 方法详解 / 关键设计 2: G24 with 4096 codewords; shell by
+ *               cumulative offsets; classes = magnitude multiset + even/odd coset, contiguous
+ *               ranges; r = I_class mod A, I' = floor(I_class/A), s = I' mod 2^B,
+ *               I'' = floor(I'/2^B); r = Golay refinement, s = sign pattern meeting the
+ *               congruence check, I'' = lexicographic permutation rank.
+ *   [notes-K4]  papernotes.org, 方法详解 / 关键设计 4: fused dequantize-and-multiply.
+ *   [gist-M1]   gist.science, Methodik 1: Leech lattice built from G24, integer vectors in
+ *               even and odd cosets, shells of equal squared norm.
+ *   [gist-M3]   gist.science, Methodik 3: index hierarchy shell -> class -> local symmetries.
+ * Textbook facts the pages point to but do not print (Conway & Sloane, "Sphere Packings,
+ * Lattices and Groups", ch. 4 sec. 11): the sqrt(8)-scaled Leech lattice is the set of
+ * integer vectors x with all x_i of one parity, {i : x_i = 2 (mod 4)} (even case) or
+ * {i : x_i = 1 (mod 4)} (odd case) a Golay codeword, and sum x_i = 0 (even) or 4 (odd) mod 8.
+ */
+#include "llvq_oracle.h"
+
+#include <math.h>
+#include <pthread.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+typedef unsigned __int128 u128;
+
+#define MAXM 256              /* largest shell any supported budget reaches (96 bits: 214) */
+
+static u128 mk128(uint64_t lo, uint64_t hi) { return ((u128)hi << 64) | lo; }
+static void split128(u128 v, uint64_t *lo, uint64_t *hi) {
+    *lo = (uint64_t)v;
+    *hi = (uint64_t)(v >> 64);
+}
+
+/* ===================================================================================== */
+/* Extended binary Golay code.  Reading: the cyclic [23,12] Golay code with generator      */
+/* polynomial g(x) = 1 + x^2 + x^4 + x^5 + x^6 + x^10 + x^11 (coefficient of x^i on        */
+/* coordinate i), extended by an overall parity bit on coordinate 23.  The pages only say  */
+/* "extended binary Golay code, 4096 codewords" [notes-K2]; any equivalent code gives an    */
+/* isometric lattice, so fixing one is part of the index format.                           */
+/* ===================================================================================== */
+static int popcount24(uint32_t w) { return __builtin_popcount(w & 0xFFFFFFu); }
+
+static void golay_generate(uint32_t words[4096]) {
+    const uint32_t g = (1u << 0) | (1u << 2) | (1u << 4) | (1u << 5) | (1u << 6) | (1u << 10) | (1u << 11);
+    uint32_t rows[12];
+    for (int i = 0; i < 12; i++) {
+        uint32_t w = g << i;                       /* x^i g(x), coordinates 0..22 */
+        uint32_t parity = (uint32_t)(popcount24(w) & 1);
+        rows[i] = w | (parity << 23);              /* overall parity on coordinate 23 */
+    }
+    for (uint32_t msg = 0; msg < 4096; msg++) {    /* every combination of the 12 rows */
+        uint32_t w = 0;
+        for (int i = 0; i < 12; i++)
+            if (msg >> i & 1u) w ^= rows[i];
+        words[msg] = w;
+    }
+}
+
+static int cmp_u32(const void *a, const void *b) {
+    uint32_t x = *(const uint32_t *)a, y = *(const uint32_t *)b;
+    return (x > y) - (x < y);
+}
+static int cmp_weight_mask(const void *a, const void *b) {
+    uint32_t x = *(const uint32_t *)a, y = *(const uint32_t *)b;
+    int wx = popcount24(x), wy = popcount24(y);
+    if (wx != wy) return wx - wy;
+    return (x > y) - (x < y);
+}
+
+int ora_golay_by_mask(uint32_t out[4096]) {
+    golay_generate(out);
+    qsort(out, 4096, sizeof(uint32_t), cmp_u32);
+    return 0;
+}
+
+int ora_golay_by_weight(uint32_t out[4096], int32_t base[26]) {
+    golay_generate(out);
+    qsort(out, 4096, sizeof(uint32_t), cmp_weight_mask);
+    for (int w = 0; w <= 25; w++) base[w] = 4096;
+    for (int i = 4095; i >= 0; i--) base[popcount24(out[i])] = i;
+    for (int w = 24; w >= 0; w--)            /* weights with no word point at the next one */
+        if (base[w] == 4096 || base[w] > base[w + 1]) base[w] = base[w + 1];
+    return 0;
+}
+
+static int golay_contains(const uint32_t sorted_by_mask[4096], uint32_t w, int *pos) {
+    int lo = 0, hi = 4095;
+    while (lo <= hi) {
+        int mid = (lo + hi) / 2;
+        if (sorted_by_mask[mid] == w) { if (pos) *pos = mid; return 1; }
+        if (sorted_by_mask[mid] < w) lo = mid + 1; else hi = mid - 1;
+    }
+    return 0;
+}
+
+/* ===================================================================================== */
+/* Lattice membership by the congruences (textbook; [gist-M1] "even and odd cosets").       */
+/* ===================================================================================== */
+static int mod_pos(int a, int m) { int r = a % m; return r < 0 ? r + m : r; }
+
+static uint32_t g_golay_mask[4096];
+static int g_golay_ready = 0;
+static void ensure_golay(void) {
+    if (!g_golay_ready) { ora_golay_by_mask(g_golay_mask); g_golay_ready = 1; }
+}
+
+int ora_in_leech(const int32_t x[ORA_DIM]) {
+    ensure_golay();
+    int par = mod_pos(x[0], 2);
+    int sum = 0;
+    uint32_t pattern = 0;
+    for (int i = 0; i < ORA_DIM; i++) {
+        if (mod_pos(x[i], 2) != par) return 0;                 /* mod 2: one parity */
+        sum += x[i];
+        int r4 = mod_pos(x[i], 4);
+        if (par == 0 && r4 == 2) pattern |= 1u << i;            /* even: the 2 (mod 4) set */
+        if (par == 1 && r4 == 1) pattern |= 1u << i;            /* odd:  the 1 (mod 4) set */
+    }
+    if (!golay_contains(g_golay_mask, pattern, NULL)) return 0;  /* mod 4: a codeword */
+    return mod_pos(sum, 8) == (par == 0 ? 0 : 4);                /* mod 8 */
+}
+
+/* ===================================================================================== */
+/* Shell enumeration by direct search (no class formula): for each coset and each          */
+/* codeword, assign coordinates with the prescribed residue mod 4 and check the norm and    */
+/* the mod-8 sum.                                                                          */
+/* ===================================================================================== */
+typedef struct {
+    int32_t *out;
+    uint64_t cap, n;
+    int target_sum8;
+    int res[ORA_DIM];        /* required residue mod 4 per coordinate */
+    int minrest[ORA_DIM + 1];/* least squared norm the coordinates i.. can take */
+    int x[ORA_DIM];
+} enum_ctx;
+
+static void enum_rec(enum_ctx *e, int i, int rem, int sum) {
+    if (i == ORA_DIM) {
+        if (rem == 0 && mod_pos(sum, 8) == e->target_sum8) {
+            if (e->out && e->n < e->cap)
+                for (int j = 0; j < ORA_DIM; j++) e->out[e->n * ORA_DIM + j] = e->x[j];
+            e->n++;
+        }
+        return;
+    }
+    int vmax = (int)floor(sqrt((double)rem)) + 1;
+    for (int v = -vmax; v <= vmax; v++) {
+        if (mod_pos(v, 4) != e->res[i]) continue;
+        int r2 = rem - v * v;
+        if (r2 < e->minrest[i + 1]) continue;
+        e->x[i] = v;
+        enum_rec(e, i + 1, r2, sum + v);
+    }
+}
+
+uint64_t ora_shell_enumerate(int32_t m, int32_t *out, uint64_t cap) {
+    ensure_golay();
+    enum_ctx e;
+    memset(&e, 0, sizeof e);
+    e.out = out;
+    e.cap = cap;
+    for (int odd = 0; odd <= 1; odd++) {
+        e.target_sum8 = odd ? 4 : 0;
+        for (int w = 0; w < 4096; w++) {
+            uint32_t cw = g_golay_mask[w];
+            for (int i = 0; i < ORA_DIM; i++) {
+                int in = (int)(cw >> i & 1u);
+                e.res[i] = odd ? (in ? 1 : 3) : (in ? 2 : 0);
+            }
+            e.minrest[ORA_DIM] = 0;
+            for (int i = ORA_DIM - 1; i >= 0; i--) {
+                int least = (e.res[i] == 0) ? 0 : (e.res[i] == 2 ? 4 : 1);
+                e.minrest[i] = e.minrest[i + 1] + least;
+            }
+            enum_rec(&e, 0, 16 * m, 0);
+        }
+    }
+    return e.n;
+}
+
+/* Shell sizes by a coordinate-wise dynamic programme.  For a codeword of weight k the     */
+/* number of admissible vectors depends only on k, so the count is                        */
+/* sum_k (#codewords of weight k) * (DP over k coordinates of one residue class and 24-k   */
+/* of the other), tracking the squared norm and the sum mod 8.                             */
+int ora_shell_counts_dp(int32_t mmax, uint64_t *lo, uint64_t *hi) {
+    if (mmax < 0 || mmax > MAXM) return -1;
+    uint32_t words[4096];
+    golay_generate(words);
+    u128 nk[ORA_DIM + 1];
+    memset(nk, 0, sizeof nk);
+    for (int i = 0; i < 4096; i++) nk[popcount24(words[i])] += 1;
+
+    const int NMAX = 16 * mmax;
+    const int S = (NMAX + 1) * 8;
+    u128 *cur = calloc((size_t)S, sizeof(u128));
+    u128 *nxt = calloc((size_t)S, sizeof(u128));
+    u128 *total = calloc((size_t)(mmax + 1), sizeof(u128));
+    if (!cur || !nxt || !total) { free(cur); free(nxt); free(total); return -2; }
+
+    for (int odd = 0; odd <= 1; odd++) {
+        for (int k = 0; k <= ORA_DIM; k++) {
+            if (nk[k] == 0) continue;
+            memset(cur, 0, (size_t)S * sizeof(u128));
+            cur[0] = 1;                                      /* norm 0, sum 0 */
+            for (int i = 0; i < ORA_DIM; i++) {
+                int in = i < k;                              /* first k coordinates: in word */
+                int res = odd ? (in ? 1 : 3) : (in ? 2 : 0);
+                memset(nxt, 0, (size_t)S * sizeof(u128));
+                int vmax = (int)floor(sqrt((double)NMAX)) + 1, nv = 0;
+                int vlist[4 * 64];
+                for (int v = -vmax; v <= vmax; v++)           /* values with residue res mod 4 */
+                    if (mod_pos(v, 4) == res && v * v <= NMAX) vlist[nv++] = v;
+                for (int n = 0; n <= NMAX; n++)
+                    for (int s = 0; s < 8; s++) {
+                        u128 c = cur[n * 8 + s];
+                        if (!c) continue;
+                        for (int t = 0; t < nv; t++) {
+                            int v = vlist[t], n2 = n + v * v;
+                            if (n2 > NMAX) continue;
+                            nxt[n2 * 8 + mod_pos(s + v, 8)] += c;
+                        }
+                    }
+                u128 *t = cur; cur = nxt; nxt = t;
+            }
+            for (int m = 0; m <= mmax; m++) total[m] += nk[k] * cur[(16 * m) * 8 + (odd ? 4 : 0)];
+        }
+    }
+    for (int m = 0; m <= mmax; m++) split128(total[m], &lo[m], &hi[m]);
+    free(cur); free(nxt); free(total);
+    return 0;
+}
+
+/* ===================================================================================== */
+/* Lexicographic ranking of arrangements of a multiset ([notes-K2]: "I'' indexes the       */
+/* permutation in lexicographic order").  Each group of equal magnitudes has a side and   */
+/* each position a side; a group may only occupy positions of its own side.  The number   */
+/* of completions is the product of the multinomials of the two sides.                     */
+/* ===================================================================================== */
+static u128 fact128(int n) {
+    u128 f = 1;
+    for (int i = 2; i <= n; i++) f *= (u128)i;
+    return f;
+}
+
+/* binomial coefficients C(n, k), n <= 24, by Pascal's rule */
+static u128 g_binom[ORA_DIM + 1][ORA_DIM + 1];
+static int g_binom_ready = 0;
+static void ensure_binom(void) {
+    if (g_binom_ready) return;
+    for (int n = 0; n <= ORA_DIM; n++) {
+        g_binom[n][0] = 1;
+        for (int k = 1; k <= n; k++) g_binom[n][k] = g_binom[n - 1][k - 1] + (k < n ? g_binom[n - 1][k] : 0);
+    }
+    g_binom_ready = 1;
+}
+
+/* number of distinct arrangements of the remaining groups of one side:
+ * n! / prod(c_g!) = C(n, c_0) * C(n - c_0, c_1) * ... */
+static u128 multinomial_side(int ng, const int *rem, const int *gside, int side) {
+    int n = 0;
+    for (int g = 0; g < ng; g++) if (gside[g] == side) n += rem[g];
+    u128 r = 1;
+    for (int g = 0; g < ng; g++)
+        if (gside[g] == side) { r *= g_binom[n][rem[g]]; n -= rem[g]; }
+    return r;
+}
+
+static u128 completions(int ng, const int *rem, const int *gside) {
+    return multinomial_side(ng, rem, gside, 0) * multinomial_side(ng, rem, gside, 1);
+}
+
+/* unrank: position i (0..n) of side pside[i]; writes group indices to seq */
+static int arr_unrank(int ng, const int *cnt, const int *gside, int n, const int *pside, u128 p,
+                      int *seq) {
+    int rem[ORA_DIM];
+    for (int g = 0; g < ng; g++) rem[g] = cnt[g];
+    if (p >= completions(ng, rem, gside)) return -1;
+    for (int i = 0; i < n; i++) {
+        int chosen = -1;
+        for (int g = 0; g < ng; g++) {                    /* groups in ascending magnitude */
+            if (gside[g] != pside[i] || rem[g] == 0) continue;
+            rem[g]--;
+            u128 c = completions(ng, rem, gside);
+            rem[g]++;
+            if (p < c) { chosen = g; break; }
+            p -= c;
+        }
+        if (chosen < 0) return -1;
+        seq[i] = chosen;
+        rem[chosen]--;
+    }
+    return 0;
+}
+
+static int arr_rank(int ng, const int *cnt, const int *gside, int n, const int *pside,
+                    const int *seq, u128 *out) {
+    int rem[ORA_DIM];
+    for (int g = 0; g < ng; g++) rem[g] = cnt[g];
+    u128 p = 0;
+    for (int i = 0; i < n; i++) {
+        int gi = seq[i];
+        if (gi < 0 || gi >= ng || rem[gi] == 0 || gside[gi] != pside[i]) return -1;
+        for (int g = 0; g < gi; g++) {                    /* smaller magnitudes at position i */
+            if (gside[g] != pside[i] || rem[g] == 0) continue;
+            rem[g]--;
+            p += completions(ng, rem, gside);
+            rem[g]++;
+        }
+        rem[gi]--;
+    }
+    *out = p;
+    return 0;
+}
+
+int ora_unrank_arrangement(int32_t nv, const int32_t *cnt, uint64_t lo, uint64_t hi, int32_t *seq) {
+    ensure_binom();
+    int c[ORA_DIM], gs[ORA_DIM], ps[ORA_DIM] = {0}, s[ORA_DIM];
+    int n = 0;
+    if (nv < 1 || nv > ORA_DIM) return -1;
+    for (int g = 0; g < nv; g++) { c[g] = cnt[g]; gs[g] = 0; n += cnt[g]; }
+    if (n > ORA_DIM) return -1;
+    for (int i = 0; i < n; i++) ps[i] = 0;
+    if (arr_unrank(nv, c, gs, n, ps, mk128(lo, hi), s)) return -1;
+    for (int i = 0; i < n; i++) seq[i] = s[i];
+    return 0;
+}
+
+int ora_rank_arrangement(int32_t nv, const int32_t *cnt, int32_t n, const int32_t *seq,
+                         uint64_t *lo, uint64_t *hi) {
+    ensure_binom();
+    int c[ORA_DIM], gs[ORA_DIM], ps[ORA_DIM], s[ORA_DIM];
+    if (nv < 1 || nv > ORA_DIM || n > ORA_DIM) return -1;
+    for (int g = 0; g < nv; g++) { c[g] = cnt[g]; gs[g] = 0; }
+    for (int i = 0; i < n; i++) { ps[i] = 0; s[i] = seq[i]; }
+    u128 p;
+    if (arr_rank(nv, c, gs, n, ps, s, &p)) return -1;
+    split128(p, lo, hi);
+    return 0;
+}
+
+/* ===================================================================================== */
+/* Classes ([notes-K2] "leader = multiset of absolute coordinates plus even/odd coset",     */
+/* contiguous index ranges).  Readings: within a shell, even-coset classes come first,    */
+/* then odd; inside a coset, classes are ordered by their magnitudes sorted descending,   */
+/* compared lexicographically ascending.                                                  */
+/*   even: k = #{|x_i| = 2 mod 4} must be a Golay weight (0, 8, 12, 16, 24); when k = 0   */
+/*         sum|x_i|/4 must be even.  A = #codewords of weight k, B = #nonzero - [k > 0],  */
+/*         P = k!/prod(c_v!, v = 2 mod 4) * (24-k)!/prod(c_v!, v = 0 mod 4).              */
+/*   odd:  sum_i (a_i if a_i = 3 mod 4 else -a_i) = 4 mod 8 (the value with T empty; the   */
+/*         mod-8 sum does not depend on T).  A = 4096, B = 0, P = 24!/prod(c_v!).          */
+/* ===================================================================================== */
+typedef struct {
+    int16_t m;
+    int8_t odd, k, nvals;
+    uint8_t vals[ORA_DIM], cnts[ORA_DIM];
+    uint16_t A;
+    int8_t B;
+    u128 P, size, offset;       /* offset: global first index */
+} ocls;
+
+typedef void (*class_cb)(void *ctx, const ocls *c);
+
+typedef struct {
+    int m, odd, target;
+    int a[ORA_DIM];
+    const int *nk;          /* codewords per weight */
+    class_cb cb;
+    void *ctx;
+} cenum_ctx;
+
+static void make_class(cenum_ctx *e, ocls *c) {
+    /* a[] holds the magnitudes sorted descending */
+    memset(c, 0, sizeof *c);
+    c->m = (int16_t)e->m;
+    c->odd = (int8_t)e->odd;
+    int nv = 0;
+    for (int i = ORA_DIM - 1; i >= 0; i--) {      /* ascending distinct values */
+        if (nv > 0 && c->vals[nv - 1] == e->a[i]) c->cnts[nv - 1]++;
+        else { c->vals[nv] = (uint8_t)e->a[i]; c->cnts[nv] = 1; nv++; }
+    }
+    c->nvals = (int8_t)nv;
+}
+
+static int class_valid_and_size(ocls *c, const int *nk) {
+    int sumabs = 0, nnz = 0, k = 0;
+    for (int g = 0; g < c->nvals; g++) {
+        sumabs += c->vals[g] * c->cnts[g];
+        if (c->vals[g] != 0) nnz += c->cnts[g];
+        if (c->vals[g] % 4 == 2) k += c->cnts[g];
+    }
+    if (!c->odd) {
+        if (nk[k] == 0) return 0;
+        if (k == 0 && (sumabs / 4) % 2 != 0) return 0;
+        c->k = (int8_t)k;
+        c->A = (uint16_t)nk[k];
+        c->B = (int8_t)(k > 0 ? nnz - 1 : nnz);
+        u128 ps = fact128(k), pc = fact128(ORA_DIM - k);
+        for (int g = 0; g < c->nvals; g++) {
+            if (c->vals[g] % 4 == 2) ps /= fact128(c->cnts[g]);
+            else pc /= fact128(c->cnts[g]);
+        }
+        c->P = ps * pc;
+    } else {
+        int s = 0;
+        for (int g = 0; g < c->nvals; g++)
+            s += (c->vals[g] % 4 == 3 ? 1 : -1) * c->vals[g] * c->cnts[g];
+        if (mod_pos(s, 8) != 4) return 0;
+        c->k = 0;
+        c->A = 4096;
+        c->B = 0;
+        u128 p = fact128(ORA_DIM);
+        for (int g = 0; g < c->nvals; g++) p /= fact128(c->cnts[g]);
+        c->P = p;
+    }
+    c->size = (u128)c->A * ((u128)1 << c->B) * c->P;
+    return 1;
+}
+
+/* choose a[d] ascending (so descending tuples come out in ascending lexicographic order) */
+static void cenum_rec(cenum_ctx *e, int d, int rem, int prev) {
+    int low = e->odd ? 1 : 0;
+    if (d == ORA_DIM) {
+        if (rem != 0) return;
+        ocls c;
+        make_class(e, &c);
+        if (class_valid_and_size(&c, e->nk)) e->cb(e->ctx, &c);
+        return;
+    }
+    int left = ORA_DIM - d;               /* coordinates still to fill, this one included */
+    for (int v = low; v <= prev; v += 2) {
+        int r2 = rem - v * v;
+        if (r2 < (left - 1) * low * low) break;         /* the rest cannot be that small */
+        if ((long)left * v * v < rem) continue;          /* the rest cannot reach rem */
+        e->a[d] = v;
+        cenum_rec(e, d + 1, r2, v);
+    }
+}
+
+static void enumerate_classes(int m, const int *nk, class_cb cb, void *ctx) {
+    cenum_ctx e;
+    memset(&e, 0, sizeof e);
+    e.m = m;
+    e.nk = nk;
+    e.cb = cb;
+    e.ctx = ctx;
+    int top = (int)floor(sqrt((double)(16 * m))) + 1;
+    for (int odd = 0; odd <= 1; odd++) {               /* even coset first */
+        e.odd = odd;
+        int start = top;
+        if ((start & 1) != odd) start--;
+        cenum_rec(&e, 0, 16 * m, start);
+    }
+}
+
+/* ===================================================================================== */
+/* Codec                                                                                   */
+/* ===================================================================================== */
+struct ora_codec {
+    int bits, M;
+    int nk[ORA_DIM + 1];
+    uint32_t golay_mask[4096];       /* by mask */
+    uint32_t golay_weight[4096];     /* by (weight, mask) */
+    int32_t wbase[26];
+    u128 shell_off[MAXM + 2];        /* first global index of shell m; shell_off[M+1] = N_M */
+    int64_t ncls[MAXM + 1];          /* classes per shell (-1: not built) */
+    ocls *cls[MAXM + 1];
+    int store_all;                   /* 1: keep every shell's class list */
+};
+
+typedef struct { ocls *v; int64_t n, cap; u128 next; } clist;
+static void clist_push(void *ctx, const ocls *c) {
+    clist *l = ctx;
+    if (l->n == l->cap) {
+        l->cap = l->cap ? 2 * l->cap : 64;
+        l->v = realloc(l->v, (size_t)l->cap * sizeof(ocls));
+    }
+    l->v[l->n] = *c;
+    l->v[l->n].offset = l->next;
+    l->next += c->size;
+    l->n++;
+}
+
+static int build_shell(ora_codec *c, int m) {
+    if (c->ncls[m] >= 0) return 0;
+    clist l = {0};
+    l.next = c->shell_off[m];
+    enumerate_classes(m, c->nk, clist_push, &l);
+    if (l.next != c->shell_off[m + 1]) {           /* class sums must equal the DP count */
+        fprintf(stderr, "oracle: shell %d class sum disagrees with the shell count\n", m);
+        free(l.v);
+        return -1;
+    }
+    c->cls[m] = l.v;
+    c->ncls[m] = l.n;
+    return 0;
+}
+
+static void drop_shell(ora_codec *c, int m) {
+    if (!c->store_all && c->ncls[m] >= 0) {
+        free(c->cls[m]);
+        c->cls[m] = NULL;
+        c->ncls[m] = -1;
+    }
+}
+
+ora_codec *ora_codec_create(int32_t index_bits) {
+    if (index_bits != 48 && index_bits != 72 && index_bits != 96) return NULL;
+    ora_codec *c = calloc(1, sizeof *c);
+    if (!c) return NULL;
+    ensure_golay();
+    ensure_binom();
+    c->bits = index_bits;
+    ora_golay_by_mask(c->golay_mask);
+    ora_golay_by_weight(c->golay_weight, c->wbase);
+    for (int i = 0; i < 4096; i++) c->nk[popcount24(c->golay_mask[i])]++;
+    for (int m = 0; m <= MAXM; m++) c->ncls[m] = -1;
+
+    /* shell sizes far enough to pass 2^index_bits (M = 13, 53, 214 for 48, 72, 96 bits) */
+    int mbound = index_bits == 48 ? 20 : (index_bits == 72 ? 64 : 230);
+    uint64_t lo[MAXM + 1], hi[MAXM + 1];
+    if (ora_shell_counts_dp(mbound, lo, hi)) { free(c); return NULL; }
+    u128 limit = (u128)1 << index_bits, cum = 0;
+    int M = 1;
+    c->shell_off[2] = 0;
+    for (int m = 2; m <= mbound; m++) {
+        u128 n = mk128(lo[m], hi[m]);
+        if (cum + n > limit) break;
+        cum += n;
+        M = m;
+        c->shell_off[m + 1] = cum;
+    }
+    c->M = M;
+    c->store_all = index_bits <= 72;
+    if (c->store_all)
+        for (int m = 2; m <= M; m++)
+            if (build_shell(c, m)) { ora_codec_destroy(c); return NULL; }
+    return c;
+}
+
+void ora_codec_destroy(ora_codec *c) {
+    if (!c) return;
+    for (int m = 0; m <= MAXM; m++) free(c->cls[m]);
+    free(c);
+}
+
+int32_t ora_codec_max_shell(const ora_codec *c) { return c->M; }
+
+void ora_codec_npoints(const ora_codec *c, uint64_t *lo, uint64_t *hi) {
+    split128(c->shell_off[c->M + 1], lo, hi);
+}
+
+void ora_codec_shell_offset(const ora_codec *c, int32_t m, uint64_t *lo, uint64_t *hi) {
+    if (m < 2 || m > c->M + 1) { *lo = *hi = 0; return; }
+    split128(c->shell_off[m], lo, hi);
+}
+
+int64_t ora_codec_shell_nclasses(ora_codec *c, int32_t m) {
+    if (m < 2 || m > c->M) return -1;
+    if (build_shell(c, m)) return -1;
+    int64_t n = c->ncls[m];
+    drop_shell(c, m);
+    return n;
+}
+
+static void info_from(const ocls *o, ora_class_info *out) {
+    memset(out, 0, sizeof *out);
+    out->m = o->m;
+    out->odd = o->odd;
+    out->k = o->k;
+    out->nvals = o->nvals;
+    for (int g = 0; g < o->nvals; g++) { out->vals[g] = o->vals[g]; out->cnts[g] = o->cnts[g]; }
+    out->A = o->A;
+    out->B = o->B;
+    split128(o->P, &out->P_lo, &out->P_hi);
+    split128(o->size, &out->size_lo, &out->size_hi);
+    split128(o->offset, &out->offset_lo, &out->offset_hi);
+}
+
+int ora_codec_shell_class(ora_codec *c, int32_t m, int64_t j, ora_class_info *out) {
+    if (m < 2 || m > c->M) return -1;
+    if (build_shell(c, m)) return -1;
+    int rc = -1;
+    if (j >= 0 && j < c->ncls[m]) { info_from(&c->cls[m][j], out); rc = 0; }
+    drop_shell(c, m);
+    return rc;
+}
+
+/* the class holding global index I (shell by cumulative offsets, then class) */
+static int find_class(ora_codec *c, u128 I, ocls *out) {
+    if (I >= c->shell_off[c->M + 1]) return -1;
+    int m = 2;
+    while (!(I < c->shell_off[m + 1])) m++;            /* [notes-K2] shell by cumulative offsets */
+    if (build_shell(c, m)) return -1;
+    /* classes are contiguous ranges in order: the last class whose offset is <= I */
+    int64_t lo = 0, hi = c->ncls[m] - 1;
+    while (lo < hi) {
+        int64_t mid = (lo + hi + 1) / 2;
+        if (c->cls[m][mid].offset <= I) lo = mid; else hi = mid - 1;
+    }
+    *out = c->cls[m][lo];
+    drop_shell(c, m);
+    return 0;
+}
+
+/* position sides: even class -> 0 on the codeword S, 1 elsewhere; odd -> all 0 */
+static void class_sides(const ocls *o, uint32_t S, int *gside, int *pside) {
+    for (int g = 0; g < o->nvals; g++)
+        gside[g] = o->odd ? 0 : (o->vals[g] % 4 == 2 ? 0 : 1);
+    for (int i = 0; i < ORA_DIM; i++)
+        pside[i] = o->odd ? 0 : ((S >> i & 1u) ? 0 : 1);
+}
+
+/* decode ([notes-K2]): shell -> class -> r, s, I'' by division and remainder, then the
+ * codeword, the lexicographic arrangement of the magnitudes and the signs. */
+static int decode_one(ora_codec *c, u128 I, int32_t x[ORA_DIM], int *shell) {
+    ocls o;
+    if (find_class(c, I, &o)) return -1;
+    u128 Iclass = I - o.offset;
+    u128 r = Iclass % o.A;                       /* r  = I_class mod A           */
+    u128 I1 = Iclass / o.A;                      /* I' = floor(I_class / A)      */
+    u128 s = I1 % ((u128)1 << o.B);              /* s  = I' mod 2^B              */
+    u128 p = I1 / ((u128)1 << o.B);              /* I''= floor(I' / 2^B)         */
+
+    uint32_t word;
+    if (o.odd) word = c->golay_mask[(int)r];                 /* T: r-th codeword by mask */
+    else word = c->golay_weight[c->wbase[o.k] + (int)r];     /* S: r-th word of weight k */
+
+    int cnt[ORA_DIM], gside[ORA_DIM], pside[ORA_DIM], seq[ORA_DIM];
+    for (int g = 0; g < o.nvals; g++) cnt[g] = o.cnts[g];
+    class_sides(&o, word, gside, pside);
+    if (arr_unrank(o.nvals, cnt, gside, ORA_DIM, pside, p, seq)) return -1;
+    int a[ORA_DIM];
+    for (int i = 0; i < ORA_DIM; i++) a[i] = o.vals[seq[i]];
+
+    if (o.odd) {
+        /* x_i = 1 (mod 4) exactly on T */
+        for (int i = 0; i < ORA_DIM; i++) {
+            int inT = (int)(word >> i & 1u);
+            x[i] = (inT == (a[i] % 4 == 1)) ? a[i] : -a[i];
+        }
+    } else {
+        /* bit j of s -> j-th nonzero coordinate (ascending), skipping the highest coordinate
+         * of S, which takes the sign that makes #negatives on S = sum|x|/4 (mod 2) */
+        int top = -1;
+        if (o.k > 0) for (int i = 0; i < ORA_DIM; i++) if (word >> i & 1u) top = i;
+        int j = 0, negS = 0, sumabs = 0;
+        for (int i = 0; i < ORA_DIM; i++) {
+            sumabs += a[i];
+            x[i] = a[i];
+            if (a[i] == 0 || i == top) continue;
+            if ((s >> j) & 1) { x[i] = -a[i]; if (word >> i & 1u) negS++; }
+            j++;
+        }
+        if (top >= 0 && (negS & 1) != ((sumabs / 4) & 1)) x[top] = -a[top];
+    }
+    if (shell) *shell = o.m;
+    return 0;
+}
+
+int ora_decode(ora_codec *c, uint64_t lo, uint64_t hi, int32_t x[ORA_DIM]) {
+    return decode_one(c, mk128(lo, hi), x, NULL);
+}
+
+static int cmp_int_desc(const void *a, const void *b) {
+    int x = *(const int *)a, y = *(const int *)b;
+    return (x < y) - (x > y);
+}
+
+/* encode: the inverse of decode, step by step */
+int ora_encode(ora_codec *c, const int32_t x[ORA_DIM], uint64_t *lo, uint64_t *hi) {
+    if (!ora_in_leech(x)) return -1;
+    int nrm = 0, a[ORA_DIM], sorted[ORA_DIM];
+    for (int i = 0; i < ORA_DIM; i++) {
+        a[i] = x[i] < 0 ? -x[i] : x[i];
+        nrm += a[i] * a[i];
+        sorted[i] = a[i];
+    }
+    if (nrm % 16) return -1;
+    int m = nrm / 16;
+    if (m < 2 || m > c->M) return -1;
+    qsort(sorted, ORA_DIM, sizeof(int), cmp_int_desc);
+    if (build_shell(c, m)) return -1;
+    int odd = a[0] & 1;
+    /* locate the class by its magnitudes and coset */
+    int64_t found = -1;
+    for (int64_t j = 0; j < c->ncls[m] && found < 0; j++) {
+        const ocls *o = &c->cls[m][j];
+        if (o->odd != odd) continue;
+        int idx = 0, same = 1;
+        for (int g = o->nvals - 1; g >= 0 && same; g--)
+            for (int t = 0; t < o->cnts[g]; t++)
+                if (sorted[idx++] != o->vals[g]) { same = 0; break; }
+        if (same) found = j;
+    }
+    if (found < 0) { drop_shell(c, m); return -1; }
+    ocls o = c->cls[m][found];
+    drop_shell(c, m);
+
+    uint32_t word = 0;
+    for (int i = 0; i < ORA_DIM; i++) {
+        if (odd && mod_pos(x[i], 4) == 1) word |= 1u << i;
+        if (!odd && a[i] % 4 == 2) word |= 1u << i;
+    }
+    u128 r = 0;
+    if (odd) {
+        int pos;
+        if (!golay_contains(c->golay_mask, word, &pos)) return -1;
+        r = (u128)pos;
+    } else {
+        int found_r = -1;
+        for (int t = c->wbase[o.k]; t < c->wbase[o.k + 1]; t++)
+            if (c->golay_weight[t] == word) { found_r = t - c->wbase[o.k]; break; }
+        if (found_r < 0) return -1;
+        r = (u128)found_r;
+    }
+    u128 s = 0;
+    if (!odd) {
+        int top = -1;
+        if (o.k > 0) for (int i = 0; i < ORA_DIM; i++) if (word >> i & 1u) top = i;
+        int j = 0;
+        for (int i = 0; i < ORA_DIM; i++) {
+            if (a[i] == 0 || i == top) continue;
+            if (x[i] < 0) s |= (u128)1 << j;
+            j++;
+        }
+    }
+    int cnt[ORA_DIM], gside[ORA_DIM], pside[ORA_DIM], seq[ORA_DIM];
+    for (int g = 0; g < o.nvals; g++) cnt[g] = o.cnts[g];
+    class_sides(&o, word, gside, pside);
+    for (int i = 0; i < ORA_DIM; i++) {
+        seq[i] = -1;
+        for (int g = 0; g < o.nvals; g++) if (o.vals[g] == a[i]) seq[i] = g;
+    }
+    u128 p;
+    if (arr_rank(o.nvals, cnt, gside, ORA_DIM, pside, seq, &p)) return -1;
+    u128 I = o.offset + r + (u128)o.A * (s + ((u128)1 << o.B) * p);
+    split128(I, lo, hi);
+    return 0;
+}
+
+int64_t ora_decode_batch_shell(ora_codec *c, int64_t n, const uint64_t *lo, const uint64_t *hi,
+                               int8_t *out, int32_t *shell) {
+    int64_t bad = 0;
+    for (int64_t t = 0; t < n; t++) {
+        int32_t x[ORA_DIM];
+        int m = 0;
+        u128 I = mk128(lo[t], hi ? hi[t] : 0);
+        if (decode_one(c, I, x, &m)) {
+            memset(x, 0, sizeof x);
+            m = 0;
+            bad++;
+        }
+        for (int i = 0; i < ORA_DIM; i++) out[t * ORA_DIM + i] = (int8_t)x[i];
+        if (shell) shell[t] = m;
+    }
+    return bad;
+}
+
+int64_t ora_decode_batch(ora_codec *c, int64_t n, const uint64_t *lo, const uint64_t *hi,
+                         int8_t *out) {
+    return ora_decode_batch_shell(c, n, lo, hi, out, NULL);
+}
+
+/* ===================================================================================== */
+/* fp16 -> fp64 (IEEE binary16, exact)                                                   */
+/* ===================================================================================== */
+double ora_half_to_double(uint16_t h) {
+    int sign = h >> 15, e = (h >> 10) & 0x1F, f = h & 0x3FF;
+    double v;
+    if (e == 0) v = ldexp((double)f, -24);                        /* subnormal */
+    else if (e == 31) v = f ? NAN : INFINITY;
+    else v = ldexp((double)(f | 0x400), e - 25);
+    return sign ? -v : v;
+}
+
+/* ===================================================================================== */
+/* GEMV / small-batch GEMM in fp64 ([notes-K4]: each block's 24-dim integer vector is      */
+/* scaled by its gain and dotted with the activations; [notes-K1]: shape-gain, the        */
+/* direction is v/|v| and the gain a scalar).                                            */
+/* ===================================================================================== */
+static void unpack_word(const uint8_t *wp, int word_bytes, int bits, u128 *index, int *code) {
+    uint64_t lo, hi = 0;
+    memcpy(&lo, wp, 8);
+    if (word_bytes == 16) memcpy(&hi, wp + 8, 8);
+    u128 w = mk128(lo, hi);
+    *index = w & (((u128)1 << bits) - 1);
+    *code = (int)((w >> bits) & 0xFF);
+}
+
+typedef struct {
+    const ora_codec *c;
+    int32_t rows, nb, word_bytes, gain_mode, batch;
+    const void *words;
+    int64_t pitch;
+    const uint16_t *gains, *x;
+    double *y;
+    int32_t r0, r1;
+    int64_t bad;
+} gemm_job;
+
+static void gemm_rows(gemm_job *J) {
+    /* each worker keeps private class lists when shells are built on demand */
+    ora_codec *c = (ora_codec *)J->c;
+    const uint8_t *W = J->words;
+    int64_t K = (int64_t)J->nb * ORA_DIM;
+    for (int32_t r = J->r0; r < J->r1; r++) {
+        for (int32_t b = 0; b < J->batch; b++) J->y[(int64_t)b * J->rows + r] = 0.0;
+        for (int32_t j = 0; j < J->nb; j++) {
+            u128 I;
+            int code, m = 0;
+            unpack_word(W + ((int64_t)r * J->pitch + j) * J->word_bytes, J->word_bytes, c->bits, &I,
+                        &code);
+            int32_t v[ORA_DIM];
+            if (decode_one(c, I, v, &m)) { J->bad++; continue; }
+            double scale;
+            if (J->gain_mode == 0) scale = ora_half_to_double(J->gains[(int64_t)r * J->nb + j]);
+            else scale = ora_half_to_double(J->gains[(int64_t)r * 256 + code]) / (4.0 * sqrt((double)m));
+            for (int32_t b = 0; b < J->batch; b++) {
+                const uint16_t *xb = J->x + (int64_t)b * K + (int64_t)j * ORA_DIM;
+                double acc = 0.0;
+                for (int t = 0; t < ORA_DIM; t++) acc += (scale * (double)v[t]) * ora_half_to_double(xb[t]);
+                J->y[(int64_t)b * J->rows + r] += acc;
+            }
+        }
+    }
+}
+
+int64_t ora_gemm(ora_codec *c, int32_t rows, int32_t nb, const void *words, int32_t word_bytes,
+                 int64_t row_pitch_words, int32_t gain_mode, const uint16_t *gains,
+                 const uint16_t *x, int32_t batch, double *y) {
+    if ((c->bits == 48) != (word_bytes == 8)) return -1;
+    gemm_job J = {c, rows, nb, word_bytes, gain_mode, batch, words, row_pitch_words, gains, x, y,
+                  0, rows, 0};
+    gemm_rows(&J);
+    return J.bad;
+}
+
+static void *gemm_thread(void *arg) { gemm_rows((gemm_job *)arg); return NULL; }
+
+int64_t ora_gemm_mt(const ora_codec *c, int32_t rows, int32_t nb, const void *words,
+                    int32_t word_bytes, int64_t row_pitch_words, int32_t gain_mode,
+                    const uint16_t *gains, const uint16_t *x, int32_t batch, double *y,
+                    int32_t nthreads) {
+    if ((c->bits == 48) != (word_bytes == 8)) return -1;
+    if (!c->store_all) nthreads = 1;     /* on-demand shell lists are not shared safely */
+    if (nthreads < 1) nthreads = 1;
+    if (nthreads > rows) nthreads = rows > 0 ? rows : 1;
+    gemm_job *jobs = calloc((size_t)nthreads, sizeof(gemm_job));
+    pthread_t *th = calloc((size_t)nthreads, sizeof(pthread_t));
+    for (int t = 0; t < nthreads; t++) {
+        gemm_job J = {c, rows, nb, word_bytes, gain_mode, batch, words, row_pitch_words, gains, x, y,
+                      (int32_t)((int64_t)rows * t / nthreads), (int32_t)((int64_t)rows * (t + 1) / nthreads), 0};
+        jobs[t] = J;
+        pthread_create(&th[t], NULL, gemm_thread, &jobs[t]);
+    }
+    int64_t bad = 0;
+    for (int t = 0; t < nthreads; t++) { pthread_join(th[t], NULL); bad += jobs[t].bad; }
+    free(jobs);
+    free(th);
+    return bad;
+}
+
+/* ===================================================================================== */
+/* Exhaustive self-checks over whole shells (threads split the codewords).                */
+/* ===================================================================================== */
+typedef struct {
+    ora_codec *c;
+    int m_lo, m_hi, tid, nthreads;
+    uint64_t *bitmap;              /* one bit per index of shells m_lo..m_hi */
+    u128 base;                     /* first index of shell m_lo */
+    int64_t points, bad_encode, bad_range, dup, bad_roundtrip, bad_norm;
+} check_job;
+
+static void check_point(check_job *J, const int *x, int m) {
+    int32_t xx[ORA_DIM];
+    for (int i = 0; i < ORA_DIM; i++) xx[i] = x[i];
+    uint64_t lo, hi;
+    J->points++;
+    if (ora_encode(J->c, xx, &lo, &hi)) { J->bad_encode++; return; }
+    u128 I = mk128(lo, hi);
+    if (I < J->c->shell_off[m] || I >= J->c->shell_off[m + 1]) { J->bad_range++; return; }
+    u128 rel = I - J->base;
+    uint64_t bit = 1ull << (uint64_t)(rel % 64);
+    uint64_t old = __atomic_fetch_or(&J->bitmap[(size_t)(rel / 64)], bit, __ATOMIC_RELAXED);
+    if (old & bit) J->dup++;
+    int32_t y[ORA_DIM];
+    int shell = 0;
+    if (decode_one(J->c, I, y, &shell)) { J->bad_roundtrip++; return; }
+    int nrm = 0;
+    for (int i = 0; i < ORA_DIM; i++) { if (y[i] != xx[i]) { J->bad_roundtrip++; return; } nrm += y[i] * y[i]; }
+    if (nrm != 16 * m || shell != m || !ora_in_leech(y)) J->bad_norm++;
+}
+
+static void check_rec(check_job *J, enum_ctx *e, int i, int rem, int sum, int m) {
+    if (i == ORA_DIM) {
+        if (rem == 0 && mod_pos(sum, 8) == e->target_sum8) check_point(J, e->x, m);
+        return;
+    }
+    int vmax = (int)floor(sqrt((double)rem)) + 1;
+    for (int v = -vmax; v <= vmax; v++) {
+        if (mod_pos(v, 4) != e->res[i]) continue;
+        int r2 = rem - v * v;
+        if (r2 < e->minrest[i + 1]) continue;
+        e->x[i] = v;
+        check_rec(J, e, i + 1, r2, sum + v, m);
+    }
+}
+
+static void *check_thread(void *arg) {
+    check_job *J = arg;
+    enum_ctx e;
+    memset(&e, 0, sizeof e);
+    for (int m = J->m_lo; m <= J->m_hi; m++)
+        for (int odd = 0; odd <= 1; odd++) {
+            e.target_sum8 = odd ? 4 : 0;
+            for (int w = J->tid; w < 4096; w += J->nthreads) {
+                uint32_t cw = g_golay_mask[w];
+                for (int i = 0; i < ORA_DIM; i++) {
+                    int in = (int)(cw >> i & 1u);
+                    e.res[i] = odd ? (in ? 1 : 3) : (in ? 2 : 0);
+                }
+                e.minrest[ORA_DIM] = 0;
+                for (int i = ORA_DIM - 1; i >= 0; i--)
+                    e.minrest[i] = e.minrest[i + 1] + (e.res[i] == 0 ? 0 : (e.res[i] == 2 ? 4 : 1));
+                check_rec(J, &e, 0, 16 * m, 0, m);
+            }
+        }
+    return NULL;
+}
+
+/* Enumerate every point of shells m_lo..m_hi by direct search, encode it, require the
+ * index to fall in its shell's range and to be hit exactly once, and require decode to
+ * give the point back (with the right norm and lattice membership).  result[0..6] =
+ * points, bad encodes, out-of-range, duplicates, bad round trips, bad norms, indices of
+ * the range never hit.  Returns 0 when every count but result[0] is zero. */
+int ora_check_shells(ora_codec *c, int32_t m_lo, int32_t m_hi, int32_t nthreads, int64_t result[7]) {
+    if (!c->store_all || m_lo < 2 || m_hi > c->M || m_lo > m_hi) return -1;
+    if (nthreads < 1) nthreads = 1;
+    u128 base = c->shell_off[m_lo], span = c->shell_off[m_hi + 1] - base;
+    size_t words = (size_t)((span + 63) / 64);
+    uint64_t *bm = calloc(words, sizeof(uint64_t));
+    check_job *jobs = calloc((size_t)nthreads, sizeof(check_job));
+    pthread_t *th = calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!bm || !jobs || !th) { free(bm); free(jobs); free(th); return -2; }
+    for (int t = 0; t < nthreads; t++) {
+        jobs[t].c = c; jobs[t].m_lo = m_lo; jobs[t].m_hi = m_hi; jobs[t].tid = t;
+        jobs[t].nthreads = nthreads; jobs[t].bitmap = bm; jobs[t].base = base;
+        pthread_create(&th[t], NULL, check_thread, &jobs[t]);
+    }
+    for (int k = 0; k < 7; k++) result[k] = 0;
+    for (int t = 0; t < nthreads; t++) {
+        pthread_join(th[t], NULL);
+        result[0] += jobs[t].points; result[1] += jobs[t].bad_encode; result[2] += jobs[t].bad_range;
+        result[3] += jobs[t].dup; result[4] += jobs[t].bad_roundtrip; result[5] += jobs[t].bad_norm;
+    }
+    int64_t missing = 0;
+    for (u128 i = 0; i < span; i++)
+        if (!(bm[(size_t)(i / 64)] >> (uint64_t)(i % 64) & 1ull)) missing++;
+    result[6] = missing;
+    free(bm); free(jobs); free(th);
+    for (int k = 1; k < 7; k++) if (result[k]) return 1;
+    return 0;
+}
