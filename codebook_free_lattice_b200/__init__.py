@@ -1,0 +1,142 @@
+"""LLVQ (Leech lattice vector quantization) decode and fused decode-and-multiply on B200.
+
+A thin ctypes binding over libllvq.so (the C ABI in include/llvq.h).  Every step of the
+decode and of the products runs in the library's CUDA kernels; this module only marshals
+arguments (device pointers of torch tensors, the current CUDA stream).  There is no CPU
+fallback: importing the binding fails if libllvq.so is missing or cannot be loaded.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libllvq.so")
+
+LLVQ_OK = 0
+LLVQ_ERR_ARG = 1
+LLVQ_ERR_UNSUPPORTED = 2
+LLVQ_ERR_CUDA = 3
+LLVQ_ERR_DEVICE_FLAG = 4
+LLVQ_GAIN_FP16_DIRECT = 0
+LLVQ_GAIN_U8_TABLE = 1
+LLVQ_FLAG_INDEX_RANGE = 0x1
+
+
+class llvq_weight(C.Structure):
+    _fields_ = [("rows", C.c_int32), ("cols", C.c_int32), ("blocks_per_row", C.c_int32),
+                ("index_bits", C.c_int32), ("word_bytes", C.c_int32), ("gain_mode", C.c_int32),
+                ("row_pitch_words", C.c_int64), ("words", C.c_void_p), ("gains", C.c_void_p)]
+
+
+class LLVQError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what}: {llvq_status_string(status)} ({status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"libllvq.so not built at {LIB_PATH}; run codebook_free_lattice_b200/build.py")
+        L = C.CDLL(LIB_PATH)
+        L.llvq_status_string.argtypes = [C.c_int]
+        L.llvq_status_string.restype = C.c_char_p
+        L.llvq_codec_create.argtypes = [C.c_int32, C.POINTER(C.c_void_p)]
+        L.llvq_codec_destroy.argtypes = [C.c_void_p]
+        L.llvq_codec_destroy.restype = None
+        L.llvq_codec_info.argtypes = [C.c_void_p, C.POINTER(C.c_int32), C.POINTER(C.c_uint64),
+                                      C.POINTER(C.c_uint64), C.POINTER(C.c_int64)]
+        L.llvq_decode.argtypes = [C.c_void_p, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
+        L.llvq_gemv.argtypes = [C.c_void_p, C.POINTER(llvq_weight), C.c_void_p, C.c_void_p, C.c_void_p]
+        L.llvq_gemm_smallbatch.argtypes = [C.c_void_p, C.POINTER(llvq_weight), C.c_void_p, C.c_int32,
+                                           C.c_void_p, C.c_void_p]
+        L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
+        for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
+                  "llvq_gemm_smallbatch", "llvq_get_error"):
+            getattr(L, f).restype = C.c_int
+        _lib = L
+    return _lib
+
+
+EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
+            "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string")
+
+
+def llvq_status_string(status: int) -> str:
+    return lib().llvq_status_string(status).decode()
+
+
+def _check(status: int, what: str):
+    if status != LLVQ_OK:
+        raise LLVQError(status, what)
+
+
+def _stream(stream) -> C.c_void_p:
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return C.c_void_p(stream.cuda_stream)
+
+
+class Codec:
+    """Decode tables of one index budget (48 or 72 bits) on the current CUDA device."""
+
+    def __init__(self, index_bits: int = 48):
+        h = C.c_void_p()
+        _check(lib().llvq_codec_create(index_bits, C.byref(h)), f"llvq_codec_create({index_bits})")
+        self._h = h
+        self.index_bits = index_bits
+        M, lo, hi, nc = C.c_int32(), C.c_uint64(), C.c_uint64(), C.c_int64()
+        _check(lib().llvq_codec_info(h, C.byref(M), C.byref(lo), C.byref(hi), C.byref(nc)), "llvq_codec_info")
+        self.max_shell = M.value
+        self.n_points = (hi.value << 64) | lo.value
+        self.n_classes = nc.value
+        self.word_bytes = 8 if index_bits == 48 else 16
+
+    @property
+    def handle(self) -> C.c_void_p:
+        return self._h
+
+    def close(self):
+        if getattr(self, "_h", None) and self._h.value:
+            lib().llvq_codec_destroy(self._h)
+            self._h = C.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def weight(self, words, gains, rows: int, cols: int, gain_mode: int,
+               row_pitch_words: int | None = None) -> llvq_weight:
+        nb = -(-cols // 24)
+        pitch = nb if row_pitch_words is None else row_pitch_words
+        return llvq_weight(rows, cols, nb, self.index_bits, self.word_bytes, gain_mode, pitch,
+                           words.data_ptr(), gains.data_ptr())
+
+    def decode(self, words, out, n: int | None = None, stream=None):
+        """words: device tensor of packed words; out: device int8 [n, 24]."""
+        n = out.shape[0] if n is None else n
+        _check(lib().llvq_decode(self._h, C.c_void_p(words.data_ptr()), self.word_bytes, n,
+                                 C.c_void_p(out.data_ptr()), _stream(stream)), "llvq_decode")
+
+    def gemv(self, w: llvq_weight, x, y, stream=None):
+        _check(lib().llvq_gemv(self._h, C.byref(w), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()),
+                               _stream(stream)), "llvq_gemv")
+
+    def gemm(self, w: llvq_weight, X, Y, batch: int, stream=None):
+        _check(lib().llvq_gemm_smallbatch(self._h, C.byref(w), C.c_void_p(X.data_ptr()), batch,
+                                          C.c_void_p(Y.data_ptr()), _stream(stream)), "llvq_gemm_smallbatch")
+
+    def get_error(self, stream=None) -> int:
+        flags = C.c_uint32()
+        st = lib().llvq_get_error(self._h, _stream(stream), C.byref(flags))
+        if st not in (LLVQ_OK, LLVQ_ERR_DEVICE_FLAG):
+            raise LLVQError(st, "llvq_get_error")
+        return flags.value

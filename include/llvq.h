@@ -1,0 +1,120 @@
+/*
+ * llvq.h -- C ABI of libllvq: Leech lattice vector quantization (LLVQ) decode and fused
+ * decode-and-multiply on one NVIDIA B200 (sm_100a).
+ *
+ * What the calls compute ("Leech Lattice Vector Quantization for Efficient LLM Compression",
+ * arXiv 2603.11021):
+ *   - A packed word carries one block index I into the union of Leech lattice shells
+ *     m = 2..M (shell m: squared norm 2m; papernotes.org notes, 方法详解 / 关键设计 1).
+ *   - I decodes by the hierarchical bijection of 关键设计 2: the shell from cumulative shell
+ *     offsets, the class (magnitude multiset + even/odd coset) from class offsets, then
+ *     r = I_class mod A (Golay codeword), I' = floor(I_class / A), s = I' mod 2^B (signs),
+ *     I'' = floor(I' / 2^B) (lexicographic arrangement rank).  The result is a 24-dim integer
+ *     vector of the sqrt(8)-scaled Leech lattice (sum of squares 16 m).
+ *   - The fused calls scale each block vector by its shape-gain gain and accumulate its dot
+ *     product with fp16 activations, never writing dequantized weights to memory (关键设计 4;
+ *     gist.science summary, Methodik 4 "Dequantisierungskernel").
+ * The concrete index format (Golay generator, class order, sign order, arrangement order)
+ * is fixed by the readings documented with the repository.
+ *
+ * Conventions for every call:
+ *   - Pointers named d_* are DEVICE pointers on the device current when the codec was
+ *     created; they are owned by the caller and must stay valid until the stream has run
+ *     the call.  Host pointers are plain host memory.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *   - Calls validate their arguments on the host and return LLVQ_ERR_ARG without launching
+ *     anything when a check fails.  Launch failures return LLVQ_ERR_CUDA.  No call allocates
+ *     device memory or synchronises, except llvq_codec_create/destroy and llvq_get_error.
+ *   - Device-side faults in the data (an index >= N_M) do not trap: the block decodes to the
+ *     zero vector and a sticky flag is set, read back by llvq_get_error.
+ *   - Kernels are written for sm_100a only; there is no CPU fallback.
+ */
+#ifndef LLVQ_H
+#define LLVQ_H
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LLVQ_OK = 0,
+    LLVQ_ERR_ARG = 1,          /* invalid argument: null pointer, size, alignment, mismatch */
+    LLVQ_ERR_UNSUPPORTED = 2,  /* valid request the library does not implement */
+    LLVQ_ERR_CUDA = 3,         /* CUDA runtime error (no device, launch failure, ...) */
+    LLVQ_ERR_DEVICE_FLAG = 4   /* a kernel raised a sticky data flag (see llvq_get_error) */
+} llvq_status;
+
+typedef enum {
+    LLVQ_GAIN_FP16_DIRECT = 0, /* gains: fp16 [rows][blocks_per_row]; weight = g * v */
+    LLVQ_GAIN_U8_TABLE = 1     /* gains: fp16 [rows][256], code in the word's 8 bits above the
+                                  index; weight = table[code] * v / |v|, |v| = 4 sqrt(m)
+                                  (shape-gain: unit direction times a scalar gain) */
+} llvq_gain_mode;
+
+/* Sticky device flags returned by llvq_get_error. */
+#define LLVQ_FLAG_INDEX_RANGE 0x1u /* some index was >= N_M (its block decoded to zero) */
+
+/* Opaque codec: owns the decode tables of one index budget on one device. */
+typedef struct llvq_codec llvq_codec;
+
+/* A compressed weight matrix W [rows][cols], split into 24-weight blocks along cols.
+ * words: device, [rows][row_pitch_words] packed words of word_bytes bytes (row-major).
+ *   word_bytes 8  (index_bits 48): bits [0,48) index, [48,56) gain code, [56,64) zero.
+ *   word_bytes 16 (index_bits 72): little-endian; bits [0,72) index, [72,80) gain code.
+ * Block j of row r covers columns [24 j, 24 j + 24); cols beyond the logical width are
+ * padding, and the activations must be zero there.  Alignment: words 8-byte (16-byte for
+ * 16-byte words) aligned, gains 2-byte aligned. */
+typedef struct {
+    int32_t rows;              /* M */
+    int32_t cols;              /* K (logical); blocks_per_row = ceil(K / 24) */
+    int32_t blocks_per_row;    /* nb */
+    int32_t index_bits;        /* 48 or 72; must equal the codec's */
+    int32_t word_bytes;        /* 8 for 48-bit, 16 for 72-bit */
+    int32_t gain_mode;         /* llvq_gain_mode */
+    int64_t row_pitch_words;   /* >= blocks_per_row */
+    const void *words;         /* device */
+    const void *gains;         /* device fp16 (see llvq_gain_mode) */
+} llvq_weight;
+
+/* Build the tables for an index budget (48 -> shells 2..13, 72 -> shells 2..53; 96 bits is
+ * LLVQ_ERR_UNSUPPORTED) on the current device and upload them.  *out is owned by the caller
+ * and released with llvq_codec_destroy.  Thread-safe to use from several streams afterwards
+ * (the codec is read-only except for its sticky flag word). */
+llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out);
+void llvq_codec_destroy(llvq_codec *codec);
+
+/* Host query: largest shell M, number of coded points N_M (as lo/hi 64-bit halves) and the
+ * number of classes. Any output pointer may be NULL. */
+llvq_status llvq_codec_info(const llvq_codec *codec, int32_t *max_shell, uint64_t *n_points_lo,
+                            uint64_t *n_points_hi, int64_t *n_classes);
+
+/* Decode n packed words (their index bits; gain bits are ignored) into int8 d_out [n][24]
+ * (the lattice coordinates).  d_words: device, n words of word_bytes (8 or 16, matching the
+ * codec), aligned to word_bytes.  d_out: device, 24*n bytes, 8-byte aligned.  n >= 0. */
+llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t word_bytes, int64_t n,
+                        int8_t *d_out, void *stream);
+
+/* Fused decode-and-multiply, batch 1: d_y[r] = sum_j scale(r, j) * <v(r, j), x[24 j .. 24 j + 23]>
+ * with fp32 accumulation.  d_x: device fp16 [blocks_per_row * 24] (zero beyond cols), 4-byte
+ * aligned.  d_y: device fp32 [rows], overwritten. */
+llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void *d_x, float *d_y,
+                      void *stream);
+
+/* Fused decode-and-multiply for 1 <= batch <= 16: d_Y[b][r] for activations d_X [batch][nb*24]
+ * (fp16, row stride nb*24, zero beyond cols).  Each block is decoded once for the whole batch.
+ * d_Y: device fp32 [batch][rows], overwritten. */
+llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, const void *d_X,
+                                 int32_t batch, float *d_Y, void *stream);
+
+/* Synchronise `stream`, return the sticky device flags raised since the last call in *flags
+ * and clear them.  Returns LLVQ_ERR_DEVICE_FLAG when any flag was set, LLVQ_OK otherwise. */
+llvq_status llvq_get_error(const llvq_codec *codec, void *stream, uint32_t *flags);
+
+/* Static string for a status code. */
+const char *llvq_status_string(llvq_status status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LLVQ_H */

@@ -1,0 +1,216 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Decoded lattice vectors must match bit for bit; fused products must be within max relative
+error 2e-3 of the oracle's fp64 result (tests.common.max_rel_err).  Inputs come from the
+seeded generator, sized so the oracle finishes in seconds while spanning many CTAs and ragged
+tails; the full-size layers are checked on sampled rows.
+"""
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from codebook_free_lattice_b200 import synth
+from tests.common import GEMV_RTOL, Layer, max_rel_err
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from codebook_free_lattice_b200 import build
+    build.build()
+    return torch.device("cuda:0")
+
+
+@pytest.fixture(scope="module")
+def gcodec(dev):
+    import codebook_free_lattice_b200 as L
+    return L.Codec(48)
+
+
+@pytest.fixture(scope="module")
+def ocodec():
+    return oracle.Codec(48)
+
+
+def gpu_decode(gcodec, words_np):
+    w = torch.from_numpy(words_np.view(np.int64)).cuda()
+    out = torch.empty((words_np.shape[0], 24), dtype=torch.int8, device="cuda")
+    gcodec.decode(w, out)
+    torch.cuda.synchronize()
+    return out.cpu().numpy()
+
+
+def test_codec_info_matches_oracle(gcodec, ocodec):
+    assert gcodec.max_shell == ocodec.max_shell == 13
+    assert gcodec.n_points == ocodec.n_points == 280974212784720
+    assert gcodec.n_classes == 383
+
+
+def test_decode_shell2_all_and_shells_2_4_uniform(gcodec, ocodec):
+    """All 196560 shell-2 indices, then 65536 seeded uniform indices over shells 2..4."""
+    idx = np.arange(196560, dtype=np.uint64)
+    lo, _ = synth.uniform_indices(synth.rng(1, 0), 65536, 415003680, 48)
+    idx = np.concatenate([idx, lo])
+    got = gpu_decode(gcodec, idx)
+    ref = ocodec.decode_batch(idx)
+    assert np.array_equal(got, ref)
+    assert gcodec.get_error() == 0
+
+
+def test_decode_uniform_full_budget(gcodec, ocodec):
+    lo, _ = synth.uniform_indices(synth.rng(2, 0), 300_000, ocodec.n_points, 48)
+    codes = synth.gain_codes(synth.rng(2, 1), lo.shape[0])
+    words = synth.pack_words(lo, None, codes, 48)          # gain bits must be ignored
+    got = gpu_decode(gcodec, words)
+    assert np.array_equal(got, ocodec.decode_batch(lo))
+
+
+def test_decode_class_boundaries(gcodec, ocodec):
+    """First and last index of every class (and the last coded index)."""
+    idx = []
+    for c in ocodec.classes():
+        idx += [c.offset, c.offset + c.size - 1, c.offset + c.size // 2]
+    idx = np.array(idx, dtype=np.uint64)
+    assert np.array_equal(gpu_decode(gcodec, idx), ocodec.decode_batch(idx))
+
+
+@pytest.mark.parametrize("n", [0, 1, 31, 33, 513, 4097])
+def test_decode_ragged_sizes(gcodec, ocodec, n):
+    lo, _ = synth.uniform_indices(synth.rng(3, n), max(n, 1), ocodec.n_points, 48)
+    lo = lo[:n]
+    if n == 0:
+        out = torch.full((4, 24), 7, dtype=torch.int8, device="cuda")
+        gcodec.decode(torch.zeros(1, dtype=torch.int64, device="cuda"), out, n=0)
+        torch.cuda.synchronize()
+        assert (out.cpu() == 7).all()
+        return
+    assert np.array_equal(gpu_decode(gcodec, lo), ocodec.decode_batch(lo))
+
+
+def test_decode_out_of_range_sets_flag(gcodec, ocodec):
+    N = ocodec.n_points
+    idx = np.array([0, N - 1, N, N + 12345, 2**48 - 1, 5], dtype=np.uint64)
+    got = gpu_decode(gcodec, idx)
+    assert gcodec.get_error() == 1
+    ref = ocodec.decode_batch(idx)             # the oracle writes zero rows for bad indices
+    assert np.array_equal(got, ref)
+    assert (got[2:5] == 0).all()
+    assert gcodec.get_error() == 0             # cleared by the previous read
+
+
+# ------------------------------------------------------------------ fused products ---------
+def run_gemm(gcodec, layer, batch=None):
+    import codebook_free_lattice_b200 as L
+    batch = layer.batch if batch is None else batch
+    words = torch.from_numpy(np.ascontiguousarray(layer.words).view(np.int64)).cuda()
+    gains = torch.from_numpy(layer.gains.view(np.int16)).cuda()
+    X = torch.from_numpy(layer.x[:batch].view(np.int16)).cuda()
+    Y = torch.full((batch, layer.rows), float("nan"), dtype=torch.float32, device="cuda")
+    w = gcodec.weight(words, gains, layer.rows, layer.K, layer.gain_mode, layer.pitch)
+    if batch == 1:
+        gcodec.gemv(w, X, Y)
+    else:
+        gcodec.gemm(w, X, Y, batch)
+    torch.cuda.synchronize()
+    assert gcodec.get_error() == 0
+    return Y.cpu().numpy().astype(np.float64)
+
+
+def oracle_gemm(ocodec, layer, rows=None, batch=None, threads=None):
+    batch = layer.batch if batch is None else batch
+    words = layer.words if rows is None else layer.words[rows]
+    gains = layer.gains if rows is None else layer.gains[rows]
+    return ocodec.gemm(words, layer.nb, layer.gain_mode, gains, layer.x[:batch], batch,
+                       row_pitch_words=layer.pitch, threads=threads or (os.cpu_count() or 1))
+
+
+def norms_from_oracle(ocodec):
+    def fn(lo, hi):
+        v = ocodec.decode_batch(lo).astype(np.float64)
+        return np.sqrt((v ** 2).sum(1))
+    return fn
+
+
+def test_gemv_small_direct_gains(gcodec, ocodec):
+    """240 x 384 (16 blocks per row), indices uniform over shells 2..4, direct fp16 gains."""
+    layer = Layer(48, 240, 384, 1, 1, ocodec.n_points, 0, index_limit=415003680,
+                  norms_fn=norms_from_oracle(ocodec))
+    y = run_gemm(gcodec, layer)
+    ref = oracle_gemm(ocodec, layer)
+    assert max_rel_err(y, ref) < GEMV_RTOL
+
+
+def test_gemv_one_hot_exact(gcodec, ocodec):
+    """x = e_j with direct gains: y = g * v exactly (one product, exact in fp32)."""
+    layer = Layer(48, 300, 24 * 7, 1, 4, ocodec.n_points, 0, norms_fn=norms_from_oracle(ocodec))
+    for j in (0, 23, 24 * 7 - 1, 77):
+        layer.x[:] = 0
+        layer.x[0, j] = 1.0
+        y = run_gemm(gcodec, layer)
+        ref = oracle_gemm(ocodec, layer, threads=1)
+        assert np.array_equal(y, ref)
+
+
+@pytest.mark.parametrize("rows,K,batch,pitch", [(97, 1000, 1, None), (333, 24 * 37, 3, 40),
+                                                (64, 4096, 8, None), (50, 2000, 16, None)])
+def test_gemm_table_gains_ragged(gcodec, ocodec, rows, K, batch, pitch):
+    layer = Layer(48, rows, K, batch, 5 + batch, ocodec.n_points, 1, pitch=pitch)
+    y = run_gemm(gcodec, layer)
+    ref = oracle_gemm(ocodec, layer)
+    assert max_rel_err(y, ref) < GEMV_RTOL
+
+
+def test_gemm_batch_equals_gemv_columns(gcodec, ocodec):
+    layer = Layer(48, 200, 24 * 50, 5, 9, ocodec.n_points, 1)
+    Y = run_gemm(gcodec, layer)
+    for b in range(5):
+        sub = Layer(48, 200, 24 * 50, 5, 9, ocodec.n_points, 1)
+        sub.x = layer.x[b:b + 1].copy()
+        sub.batch = 1
+        yb = run_gemm(gcodec, sub)
+        assert max_rel_err(yb[0], Y[b]) < 1e-5
+
+
+@pytest.mark.parametrize("rows,K,batch", [(4096, 4096, 1), (11008, 4096, 4), (4096, 11008, 1)])
+def test_gemm_full_size_sampled_rows(gcodec, ocodec, rows, K, batch):
+    """Llama-2-7B layer shapes at the bench's launch configuration; the oracle checks a seeded
+    sample of 256 rows."""
+    layer = Layer(48, rows, K, batch, 20 + rows % 97, ocodec.n_points, 1)
+    y = run_gemm(gcodec, layer)
+    rs = np.sort(np.random.default_rng(rows + K).choice(rows, 256, replace=False))
+    ref = oracle_gemm(ocodec, layer, rows=rs)
+    assert max_rel_err(y[:, rs], ref) < GEMV_RTOL
+    assert np.isfinite(y).all()
+
+
+def test_argument_errors(gcodec):
+    import codebook_free_lattice_b200 as L
+    lib = L.lib()
+    words = torch.zeros(64, dtype=torch.int64, device="cuda")
+    out = torch.zeros(64 * 24 + 8, dtype=torch.int8, device="cuda")
+    import ctypes as C
+    s = C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    assert lib.llvq_decode(gcodec.handle, C.c_void_p(words.data_ptr()), 16, 4, C.c_void_p(out.data_ptr()), s) == L.LLVQ_ERR_ARG
+    assert lib.llvq_decode(gcodec.handle, C.c_void_p(words.data_ptr() + 4), 8, 4, C.c_void_p(out.data_ptr()), s) == L.LLVQ_ERR_ARG
+    assert lib.llvq_decode(gcodec.handle, C.c_void_p(words.data_ptr()), 8, -1, C.c_void_p(out.data_ptr()), s) == L.LLVQ_ERR_ARG
+    gains = torch.zeros(256 * 4, dtype=torch.int16, device="cuda")
+    x = torch.zeros(24 * 4, dtype=torch.int16, device="cuda")
+    y = torch.zeros(4 * 16, dtype=torch.float32, device="cuda")
+    w = gcodec.weight(words, gains, 4, 96, 1)
+    for batch in (0, 17):
+        assert lib.llvq_gemm_smallbatch(gcodec.handle, C.byref(w), C.c_void_p(x.data_ptr()), batch,
+                                        C.c_void_p(y.data_ptr()), s) == L.LLVQ_ERR_ARG
+    bad = gcodec.weight(words, gains, 4, 96, 1)
+    bad.blocks_per_row = 5
+    assert lib.llvq_gemv(gcodec.handle, C.byref(bad), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()), s) == L.LLVQ_ERR_ARG
+    bad = gcodec.weight(words, gains, 4, 96, 1)
+    bad.index_bits = 72
+    assert lib.llvq_gemv(gcodec.handle, C.byref(bad), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()), s) == L.LLVQ_ERR_ARG
+    assert L.Codec(48).get_error() == 0
