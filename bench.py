@@ -145,7 +145,7 @@ def cpu_baseline(steps_seconds=12.0):
     from codebook_free_lattice_b200 import synth
     oc = oracle.Codec(48)
     cores = os.cpu_count() or 1
-    rows = 64 * cores
+    rows = min(64 * cores, ROWS)
     n = rows * NB
     lo, _ = synth.uniform_indices(synth.rng(CONFIG_ID, 0), n, oc.n_points, 48)
     codes = synth.gain_codes(synth.rng(CONFIG_ID, 1), n)
