@@ -50,13 +50,15 @@ struct alignas(16) Rec48 {
     uint32_t cum;              // bytes: cumulative counts C_<=g, g = 0..3 (saturating at 24)
     uint32_t vals;             // bytes: magnitudes of groups 0..3
     uint32_t A;                // 1, 759, 2576 or 4096
+    uint32_t gflag;            // bytes: per-group sign flag, groups 0..3 (odd: |x| = 1 mod 4;
+                               //        even: |x| != 0)
     uint8_t val4;              // magnitude of group 4
+    uint8_t gflag4;            // sign flag of group 4
     uint8_t nS;                // places on the codeword side: k (even) or 24 (odd)
     uint8_t B;                 // free sign bits
     uint8_t flags;             // bit0 odd coset, bit1 parity target (sum|x|/4 odd)
-    uint16_t wbase;            // even: first by-weight Golay slot of weight k
     uint8_t m;                 // shell
-    uint8_t pad;
+    uint16_t wbase;            // even: first by-weight Golay slot of weight k
 };
 static_assert(sizeof(Rec48) == 48, "Rec48 layout");
 
@@ -102,6 +104,11 @@ __device__ __forceinline__ uint32_t bytes_to_nibble(uint32_t b) {
     return ((b & 0x01010101u) * 0x01020408u) >> 24 & 0xFu;
 }
 
+// exact double of a small non-negative integer (n < 2^31) without a conversion instruction
+__device__ __forceinline__ double small_to_double(uint32_t n) {
+    return __hiloint2double(0x43300000, (int)n) - 0x1p52;
+}
+
 // deposit the low bits of src on the set bits of mask (24-bit), lowest first
 __device__ __forceinline__ uint32_t pdep24(uint32_t src, uint32_t mask, const Smem48 &S) {
     uint32_t out = 0;
@@ -145,49 +152,54 @@ __device__ __forceinline__ bool decode48(unsigned long long idx, const Smem48 &S
     const bool odd = R.flags & 1u;
     const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min(R.wbase + r, 4095u)];
     const uint32_t side0 = odd ? 0xFFFFFFu : word;
-    // 4. arrangement, coordinate by coordinate
+    // 4. arrangement, coordinate by coordinate.  Byte b of cumB is 0x7F + C_<=b (remaining
+    //    items of groups 0..b, biased one below the guard bit so the byte-wise subtraction of
+    //    the slot is borrow-free).  The loop keeps to the FMA, ALU and fp64 pipes: floor() by
+    //    the 2^52 magic add, int -> double by building 2^52 + n, the group count by a byte dot
+    //    product.
     double f = __dmul_ru((double)p, R.invP);
-    uint32_t cum = R.cum;
-    int L0 = R.nS, L1 = 24 - R.nS, Lt = 24;
-    uint32_t sel[6] = {0, 0, 0, 0, 0, 0};
+    uint32_t cumB = R.cum + 0x7F7F7F7Fu;
+    int L0 = R.nS, L1 = 24 - R.nS;
+    uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
 #pragma unroll
     for (int i = 0; i < 24; i++) {
-        const bool on0 = (side0 >> i) & 1u;
+        const bool on0 = side0 & (1u << i);
         const int L = on0 ? L0 : L1;
         const int off = on0 ? 0 : L0;
-        const double g = __dmul_ru(f, (double)L);
-        const uint32_t slot = (uint32_t)(int)g + (uint32_t)off;
-        const uint32_t u = (cum | 0x80808080u) - (slot + 1u) * 0x01010101u;
-        const uint32_t grp = __popc(~u & 0x80808080u);
-        const uint32_t st = __byte_perm(0u, cum, 0x3333u + grp) ;           // C_<grp
-        const uint32_t en = __byte_perm(cum, (uint32_t)Lt, 0x5550u + grp);  // C_<=grp
-        const uint32_t cnt = min(en - st, 31u);                             // in 1..24
-        f = __dmul_ru(__dadd_ru(g, -(double)((int)st - off)), S.invc[cnt]);
-        cum -= (uint32_t)(0x0101010101010101ull << (8u * grp));
-        Lt -= 1;
+        const double g = __dmul_ru(f, small_to_double((uint32_t)L));
+        const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52)) + (uint32_t)off;
+        const uint32_t u = cumB - slot * 0x01010101u;            // bit 7 of byte b: C_<=b > slot
+        const uint32_t dm = (u >> 7) & 0x01010101u;              // one per group >= grp
+        const uint32_t ssel = (uint32_t)__dp4a((int)dm, -1, 7);          // grp + 3
+        const uint32_t esel = (uint32_t)__dp4a((int)dm, -1, 0x5554);     // 0x5550 + grp
+        const uint32_t stB = __byte_perm(0x7F7F7F7Fu, cumB, ssel);       // 0x7F7F7F7F + C_<grp
+        const uint32_t enB = __byte_perm(cumB, 0x7F7F7F7Fu + (uint32_t)(24 - i), esel);  // + C_<=grp
+        const uint32_t cnt = min(enB - stB, 31u);                        // in 1..24
+        const uint32_t stl = stB - 0x7F7F7F7Fu - (uint32_t)off;
+        f = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), S.invc[cnt]);
+        cumB -= dm;                                              // groups >= grp lose one item
         L0 -= on0 ? 1 : 0;
         L1 -= on0 ? 0 : 1;
-        sel[i >> 2] |= grp << (4 * (i & 3));
+        sel[i >> 2] += ssel << (4 * (i & 3));                    // nibble = grp (bias -0x3333)
     }
-    uint32_t mag[6];
+    // 5. magnitudes and per-coordinate sign flags by byte permutation of the group tables
+    uint32_t mag[6], F = 0;
 #pragma unroll
-    for (int qq = 0; qq < 6; qq++) mag[qq] = __byte_perm(R.vals, (uint32_t)R.val4, sel[qq]);
-    // 5. signs -> mask of negative coordinates
+    for (int qq = 0; qq < 6; qq++) {
+        mag[qq] = __byte_perm(R.vals, (uint32_t)R.val4, sel[qq]);
+        F |= bytes_to_nibble(__byte_perm(R.gflag, (uint32_t)R.gflag4, sel[qq])) << (4 * qq);
+    }
+    // 6. signs.  odd: x_i = 1 (mod 4) exactly on T, so |x_i| = 1 (mod 4) is negative off T
+    //    and |x_i| = 3 (mod 4) negative on T.  even: bit j of s negates the j-th nonzero
+    //    coordinate (ascending), skipping the highest coordinate of S, whose sign makes the
+    //    number of negatives on S = sum|x|/4 (mod 2).
     uint32_t neg;
     if (odd) {
-        uint32_t one_mod4 = 0;                 // coordinates with |x| = 1 (mod 4)
-#pragma unroll
-        for (int qq = 0; qq < 6; qq++) one_mod4 |= bytes_to_nibble(mag[qq] & ~(mag[qq] >> 1)) << (4 * qq);
-        neg = word ^ one_mod4;                 // x = 1 (mod 4) exactly on T
+        neg = word ^ F;
     } else {
-        uint32_t nz = 0;
-#pragma unroll
-        for (int qq = 0; qq < 6; qq++) nz |= bytes_to_nibble((mag[qq] + 0x7F7F7F7Fu) >> 7) << (4 * qq);
-        const int top = word ? 31 - __clz(word) : -1;           // parity coordinate
-        const uint32_t topbit = top >= 0 ? (1u << top) : 0u;
-        neg = pdep24(s, nz & ~topbit, S);
-        const uint32_t par = (__popc(neg & word) ^ (R.flags >> 1)) & 1u;
-        neg |= par ? topbit : 0u;
+        const uint32_t topbit = word ? (0x80000000u >> __clz(word)) : 0u;
+        neg = pdep24(s, F & ~topbit, S);
+        neg |= ((__popc(neg & word) ^ (R.flags >> 1)) & 1u) ? topbit : 0u;
     }
 #pragma unroll
     for (int qq = 0; qq < 6; qq++) {
@@ -200,7 +212,7 @@ __device__ __forceinline__ bool decode48(unsigned long long idx, const Smem48 &S
 // --------------------------------------------------------------------------------------
 // kernels
 // --------------------------------------------------------------------------------------
-__global__ void __launch_bounds__(512) k_decode48(const Smem48 *__restrict__ image, int nclasses,
+__global__ void __launch_bounds__(512, 3) k_decode48(const Smem48 *__restrict__ image, int nclasses,
                                                   unsigned long long npoints,
                                                   const unsigned long long *__restrict__ words,
                                                   long long n, int8_t *__restrict__ out,
@@ -225,31 +237,37 @@ __global__ void __launch_bounds__(512) k_decode48(const Smem48 *__restrict__ ima
 }
 
 // Fused decode and multiply, batch BATCH (1..16).  Each CTA owns a contiguous range of rows;
-// threads walk the CTA's blocks in row-major order (coalesced word loads), decode each block
-// once and accumulate scale * <v, x_b> into shared-memory row sums.
+// its threads walk the range's blocks in row-major order (each warp reads 32 consecutive
+// packed words), decode each block once and form scale * <v, x_b> for every batch row.
+// Contributions go to shared-memory accumulators acc[b][row][lane] by atomic add (the lanes of a
+// warp hit distinct words, so only warps of the same CTA can meet on a word); at the end one
+// warp per (b, row) sums the 32 lane slots and writes the output.
 template <int BATCH>
-__global__ void __launch_bounds__(512) k_gemm48(const Smem48 *__restrict__ image, int nclasses,
-                                                unsigned long long npoints,
-                                                const unsigned long long *__restrict__ words,
-                                                long long pitch, int rows, int nb, int gain_mode,
-                                                const __half_raw *__restrict__ gains,
-                                                const __half_raw *__restrict__ X, float *__restrict__ Y,
-                                                int rows_per_cta, unsigned *__restrict__ flags) {
+constexpr int gemm_ctas_per_sm() { return BATCH == 1 ? 3 : 2; }
+
+template <int BATCH>
+__global__ void __launch_bounds__(512, gemm_ctas_per_sm<BATCH>()) k_gemm48(
+    const Smem48 *__restrict__ image, int nclasses, unsigned long long npoints,
+    const unsigned long long *__restrict__ words, long long pitch, int rows, int nb, uint32_t nb_recip,
+    int gain_mode, const __half_raw *__restrict__ gains, const __half_raw *__restrict__ X,
+    float *__restrict__ Y, int rows_per_cta, unsigned *__restrict__ flags) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem48 &S = *reinterpret_cast<Smem48 *>(smem_raw);
-    float *acc = reinterpret_cast<float *>(smem_raw + sizeof(Smem48));   // [BATCH][rows_per_cta]
+    float *acc = reinterpret_cast<float *>(smem_raw + sizeof(Smem48));   // [BATCH][rows_per_cta][32]
     load_smem_image(&S, image, sizeof(Smem48));
-    for (int i = threadIdx.x; i < BATCH * rows_per_cta; i += blockDim.x) acc[i] = 0.f;
+    for (int i = threadIdx.x; i < BATCH * rows_per_cta * 32; i += blockDim.x) acc[i] = 0.f;
     __syncthreads();
     const int row0 = blockIdx.x * rows_per_cta;
     const int nrows = min(rows_per_cta, rows - row0);
     const long long K = (long long)nb * 24;
+    const int lane = threadIdx.x & 31;
     bool bad = false;
     if (nrows > 0) {
-        const long long total = (long long)nrows * nb;
-        for (long long t = threadIdx.x; t < total; t += blockDim.x) {
-            const int rl = (int)(t / nb);
-            const int j = (int)(t - (long long)rl * nb);
+        const int total = nrows * nb;
+        for (int t = threadIdx.x; t < total; t += blockDim.x) {
+            // row of block t: t / nb by a multiply-high with ceil(2^32 / nb) (exact for t < 2^32 / nb)
+            const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
+            const int j = t - rl * nb;
             const int r = row0 + rl;
             const unsigned long long w = __ldg(words + (long long)r * pitch + j);
             uint32_t v[6];
@@ -267,7 +285,7 @@ __global__ void __launch_bounds__(512) k_gemm48(const Smem48 *__restrict__ image
 #pragma unroll
             for (int qq = 0; qq < 6; qq++)
 #pragma unroll
-                for (int b = 0; b < 4; b++) wv[4 * qq + b] = (float)(int8_t)(v[qq] >> (8 * b));
+                for (int e = 0; e < 4; e++) wv[4 * qq + e] = (float)(int8_t)(v[qq] >> (8 * e));
 #pragma unroll
             for (int bb = 0; bb < BATCH; bb++) {
                 const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
@@ -283,16 +301,20 @@ __global__ void __launch_bounds__(512) k_gemm48(const Smem48 *__restrict__ image
                         dot = fmaf(wv[8 * c + 2 * e + 1], xf.y, dot);
                     }
                 }
-                atomicAdd(&acc[bb * rows_per_cta + rl], scale * dot);
+                atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * dot);   // lanes never collide
             }
         }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < BATCH * nrows; i += blockDim.x) {
+    const int warp = threadIdx.x >> 5;
+    for (int i = warp; i < BATCH * nrows; i += blockDim.x >> 5) {
         const int bb = i / nrows, rl = i - bb * nrows;
-        Y[(long long)bb * rows + row0 + rl] = acc[bb * rows_per_cta + rl];
+        float sum = acc[(bb * rows_per_cta + rl) * 32 + lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (lane == 0) Y[(long long)bb * rows + row0 + rl] = sum;
     }
-    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, LLVQ_FLAG_INDEX_RANGE);
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(flags, LLVQ_FLAG_INDEX_RANGE);
 }
 
 }  // namespace llvq
@@ -371,9 +393,16 @@ llvq_status build_image48(const HostTables &T, Smem48 &S, std::string &err) {
             cum |= (uint32_t)std::min(acc, 24) << (8 * g);
             if (g < (int)c.vals.size()) vals |= (uint32_t)c.vals[g] << (8 * g);
         }
+        uint32_t gflag = 0;
+        for (int g = 0; g < 4 && g < (int)c.vals.size(); g++) {
+            int v = c.vals[g];
+            gflag |= (uint32_t)(c.odd ? (v % 4 == 1) : (v != 0)) << (8 * g);
+        }
         R.cum = cum;
         R.vals = vals;
+        R.gflag = gflag;
         R.val4 = c.vals.size() > 4 ? (uint8_t)c.vals[4] : 0;
+        R.gflag4 = c.vals.size() > 4 ? (uint8_t)(c.odd ? (c.vals[4] % 4 == 1) : (c.vals[4] != 0)) : 0;
         R.nS = (uint8_t)(c.odd ? 24 : c.k);
         R.B = (uint8_t)c.B;
         R.flags = (uint8_t)((c.odd ? 1 : 0) | (((c.sum_abs / 4) & 1) << 1));
@@ -399,7 +428,7 @@ thread_local std::string g_last_error;
 
 int grid_for(const llvq_codec *c, long long work, int threads) {
     long long want = (work + threads - 1) / threads;
-    long long cap = (long long)c->num_sms * 2;
+    long long cap = (long long)c->num_sms * 3;
     return (int)std::max(1LL, std::min(want, cap));
 }
 
@@ -421,11 +450,14 @@ template <int B>
 cudaError_t launch_gemm48(const llvq_codec *c, const llvq_weight *w, const void *X, float *Y,
                           cudaStream_t st) {
     const int threads = 512;
-    int grid = c->num_sms * 2;
-    int rpc = (w->rows + grid - 1) / grid;
-    rpc = std::max(rpc, 1);
+    int grid = c->num_sms * gemm_ctas_per_sm<B>();
+    int rpc = std::max((w->rows + grid - 1) / grid, 1);
     grid = (w->rows + rpc - 1) / rpc;
-    size_t smem = sizeof(Smem48) + (size_t)B * rpc * sizeof(float);
+    const size_t smem = sizeof(Smem48) + (size_t)B * rpc * 32 * sizeof(float);
+    const int nb = w->blocks_per_row;
+    // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
+    if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
+    const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
     static bool attr_set[17] = {false};
     if (!attr_set[B]) {
         cudaFuncSetAttribute(k_gemm48<B>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -435,7 +467,7 @@ cudaError_t launch_gemm48(const llvq_codec *c, const llvq_weight *w, const void 
     k_gemm48<B><<<grid, threads, smem, st>>>(c->d_image48, (int)c->nclasses,
                                              (unsigned long long)c->npoints,
                                              (const unsigned long long *)w->words, w->row_pitch_words,
-                                             w->rows, w->blocks_per_row, w->gain_mode,
+                                             w->rows, nb, recip, w->gain_mode,
                                              (const __half_raw *)w->gains, (const __half_raw *)X, Y, rpc,
                                              c->d_flags);
     return cudaGetLastError();

@@ -5,7 +5,7 @@ none of the method's decode or product arithmetic.  Quantities that depend on th
 number of coded points N_M, per-block vector norms) are passed in by the caller.
 
 Recipe (seeds numpy.random.default_rng([20260313, config_id, stream])):
-  stream 0  indices, uniform over [0, N_M) by rejection from index_bits random bits
+  stream 0  indices, uniform over [0, N_M) (rejection from N_M.bit_length() random bits)
   stream 1  8-bit gain codes (uniform; equiprobable quantile bins) or direct gains
   stream 2  per-row scale sigma_r ~ U[0.5, 2) of the chi(24) gain tables
   stream 3  activations x ~ N(0, 1) rounded to fp16, zero tail from K to K_pad
@@ -30,24 +30,23 @@ def k_pad(K: int) -> int:
 
 
 def uniform_indices(g: np.random.Generator, n: int, n_points: int, index_bits: int):
-    """n indices uniform over [0, n_points) as (lo, hi) uint64 arrays (hi = 0 for <= 64 bits)."""
+    """n indices uniform over [0, n_points) as (lo, hi) uint64 arrays (hi = 0 below 2^64).
+    Draws n_points.bit_length() random bits per index and rejects values >= n_points."""
+    assert 0 < n_points <= 2 ** index_bits
     lo = np.empty(n, np.uint64)
     hi = np.zeros(n, np.uint64)
+    if n_points <= 2 ** 63:
+        lo[:] = g.integers(0, n_points, size=n, dtype=np.uint64)
+        return lo, hi
+    hi_bits = max(n_points.bit_length() - 64, 0)
+    np_lo, np_hi = n_points & (2**64 - 1), n_points >> 64
     filled = 0
-    hi_bits = max(index_bits - 64, 0)
-    np_lo = n_points & (2**64 - 1)
-    np_hi = n_points >> 64
     while filled < n:
-        want = int((n - filled) * 1.1) + 16
+        want = 2 * (n - filled) + 16
         a = g.integers(0, 2**63, size=want, dtype=np.uint64) << np.uint64(1)
         a |= g.integers(0, 2, size=want, dtype=np.uint64)
-        if index_bits < 64:
-            a &= np.uint64((1 << index_bits) - 1)
-            ok = a < np.uint64(n_points)
-            b = np.zeros(want, np.uint64)
-        else:
-            b = g.integers(0, 2**hi_bits, size=want, dtype=np.uint64)
-            ok = (b < np.uint64(np_hi)) | ((b == np.uint64(np_hi)) & (a < np.uint64(np_lo)))
+        b = g.integers(0, 2**hi_bits, size=want, dtype=np.uint64) if hi_bits else np.zeros(want, np.uint64)
+        ok = (b < np.uint64(np_hi)) | ((b == np.uint64(np_hi)) & (a < np.uint64(np_lo)))
         a, b = a[ok], b[ok]
         take = min(n - filled, a.shape[0])
         lo[filled:filled + take] = a[:take]
