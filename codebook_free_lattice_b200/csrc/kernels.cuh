@@ -1,0 +1,118 @@
+// kernels.cuh -- decode and fused decode-and-multiply kernels, generic over the index budget's
+// decoder (Dec48 / Dec72).  "Leech Lattice Vector Quantization for Efficient LLM Compression",
+// papernotes.org notes, 方法详解 / 关键设计 4: each block is decoded to its 24-dim integer
+// vector in registers and multiplied with the activations; dequantized weights never reach
+// global memory.
+#pragma once
+#include "codec48.cuh"
+#include "codec72.cuh"
+
+namespace llvq {
+
+constexpr unsigned kFlagIndexRange = 0x1u;   // an index >= N_M was met (LLVQ_FLAG_INDEX_RANGE)
+
+// Decode n packed words into int8 [n][24].
+template <class D>
+__global__ void __launch_bounds__(512, D::kCtasPerSm) k_decode(typename D::Args args,
+                                                  const typename D::Word *__restrict__ words,
+                                                  long long n, int8_t *__restrict__ out,
+                                                  unsigned *__restrict__ flags) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    typename D::Smem &S = *reinterpret_cast<typename D::Smem *>(smem_raw);
+    load_smem_image(&S, args.image, sizeof(typename D::Smem));
+    __syncthreads();
+    bool bad = false;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n;
+         t += (long long)gridDim.x * blockDim.x) {
+        uint32_t v[6];
+        int m;
+        bad |= !D::decode(D::load(words + t), S, args, v, m);
+        uint2 *o = reinterpret_cast<uint2 *>(out + t * 24);
+        o[0] = make_uint2(v[0], v[1]);
+        o[1] = make_uint2(v[2], v[3]);
+        o[2] = make_uint2(v[4], v[5]);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagIndexRange);
+}
+
+template <class D, int BATCH>
+constexpr int gemm_ctas_per_sm() { return BATCH == 1 ? D::kCtasPerSm : 2; }
+
+// Fused decode and multiply, batch BATCH (1..16).  Each CTA owns a contiguous range of rows;
+// its threads walk the range's blocks in row-major order (each warp reads 32 consecutive
+// packed words), decode each block once and form scale * <v, x_b> for every batch row.
+// Contributions go to shared-memory accumulators acc[b][row][lane] by atomic add (the lanes of a
+// warp hit distinct words, so only warps of the same CTA can meet on a word); at the end one
+// warp per (b, row) sums the 32 lane slots and writes the output.
+// gain: direct mode -> fp16 gains[row][nb]; table mode -> fp16 gains[row][256] indexed by the
+// word's 8-bit code, times 1/|v| = 1/(4 sqrt(m)) (shape-gain: unit direction times gain).
+template <class D, int BATCH>
+__global__ void __launch_bounds__(512, gemm_ctas_per_sm<D, BATCH>()) k_gemm(
+    typename D::Args args, const typename D::Word *__restrict__ words, long long pitch, int rows, int nb,
+    uint32_t nb_recip, int gain_mode, const __half *__restrict__ gains, const __half *__restrict__ X,
+    float *__restrict__ Y, int rows_per_cta, unsigned *__restrict__ flags) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    typename D::Smem &S = *reinterpret_cast<typename D::Smem *>(smem_raw);
+    float *acc = reinterpret_cast<float *>(smem_raw + sizeof(typename D::Smem));  // [BATCH][rpc][32]
+    load_smem_image(&S, args.image, sizeof(typename D::Smem));
+    for (int i = threadIdx.x; i < BATCH * rows_per_cta * 32; i += blockDim.x) acc[i] = 0.f;
+    __syncthreads();
+    const int row0 = blockIdx.x * rows_per_cta;
+    const int nrows = min(rows_per_cta, rows - row0);
+    const long long K = (long long)nb * 24;
+    const int lane = threadIdx.x & 31;
+    bool bad = false;
+    if (nrows > 0) {
+        const int total = nrows * nb;
+        for (int t = threadIdx.x; t < total; t += blockDim.x) {
+            // row of block t: t / nb by a multiply-high with ceil(2^32 / nb) (exact for t < 2^32 / nb)
+            const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
+            const int j = t - rl * nb;
+            const int r = row0 + rl;
+            const typename D::Word w = D::load(words + (long long)r * pitch + j);
+            uint32_t v[6];
+            int m;
+            bad |= !D::decode(w, S, args, v, m);
+            float scale;
+            if (gain_mode == 0) {
+                scale = __half2float(__ldg(gains + (long long)r * nb + j));
+            } else {
+                scale = __half2float(__ldg(gains + (long long)r * 256 + D::gain_code(w))) * D::invnorm(S, m);
+            }
+            float wv[24];
+#pragma unroll
+            for (int q = 0; q < 6; q++)
+#pragma unroll
+                for (int e = 0; e < 4; e++) wv[4 * q + e] = (float)(int8_t)(v[q] >> (8 * e));
+#pragma unroll
+            for (int bb = 0; bb < BATCH; bb++) {
+                const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
+                float dot = 0.f;
+#pragma unroll
+                for (int c = 0; c < 3; c++) {
+                    const uint4 raw = __ldg(xp + c);
+                    const uint32_t h[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+                    for (int e = 0; e < 4; e++) {
+                        const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&h[e]));
+                        dot = fmaf(wv[8 * c + 2 * e], xf.x, dot);
+                        dot = fmaf(wv[8 * c + 2 * e + 1], xf.y, dot);
+                    }
+                }
+                atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * dot);
+            }
+        }
+    }
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    for (int i = warp; i < BATCH * nrows; i += blockDim.x >> 5) {
+        const int bb = i / nrows, rl = i - bb * nrows;
+        float sum = acc[(bb * rows_per_cta + rl) * 32 + lane];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+        if (lane == 0) Y[(long long)bb * rows + row0 + rl] = sum;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(flags, kFlagIndexRange);
+}
+
+}  // namespace llvq

@@ -39,10 +39,21 @@ def ocodec():
     return oracle.Codec(48)
 
 
+@pytest.fixture(scope="module")
+def gcodec72(dev):
+    import codebook_free_lattice_b200 as L
+    return L.Codec(72)
+
+
+@pytest.fixture(scope="module")
+def ocodec72():
+    return oracle.Codec(72)
+
+
 def gpu_decode(gcodec, words_np):
-    w = torch.from_numpy(words_np.view(np.int64)).cuda()
+    w = torch.from_numpy(np.ascontiguousarray(words_np).view(np.int64)).cuda()
     out = torch.empty((words_np.shape[0], 24), dtype=torch.int8, device="cuda")
-    gcodec.decode(w, out)
+    gcodec.decode(w, out, n=words_np.shape[0])
     torch.cuda.synchronize()
     return out.cpu().numpy()
 
@@ -214,3 +225,67 @@ def test_argument_errors(gcodec):
     bad.index_bits = 72
     assert lib.llvq_gemv(gcodec.handle, C.byref(bad), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()), s) == L.LLVQ_ERR_ARG
     assert L.Codec(48).get_error() == 0
+
+
+# ------------------------------------------------------------------ 72-bit budget ----------
+def split128(vals):
+    lo = np.array([v & (2**64 - 1) for v in vals], dtype=np.uint64)
+    hi = np.array([v >> 64 for v in vals], dtype=np.uint64)
+    return lo, hi
+
+
+def test_codec72_info_matches_oracle(gcodec72, ocodec72):
+    assert gcodec72.max_shell == ocodec72.max_shell == 53
+    assert gcodec72.n_points == ocodec72.n_points
+    assert gcodec72.n_classes == 114976
+
+
+def test_decode72_uniform(gcodec72, ocodec72):
+    lo, hi = synth.uniform_indices(synth.rng(11, 0), 200_000, ocodec72.n_points, 72)
+    codes = synth.gain_codes(synth.rng(11, 1), lo.shape[0])
+    words = synth.pack_words(lo, hi, codes, 72)              # gain bits must be ignored
+    got = gpu_decode(gcodec72, words)
+    assert np.array_equal(got, ocodec72.decode_batch(lo, hi))
+    assert gcodec72.get_error() == 0
+
+
+def test_decode72_every_class(gcodec72, ocodec72):
+    """First, middle and last index of all 114,976 classes (nine-group classes included) and
+    all of shell 2."""
+    idx = list(range(196560))
+    for c in ocodec72.classes():
+        idx += [c.offset, c.offset + c.size // 2, c.offset + c.size - 1]
+    lo, hi = split128(idx)
+    got = gpu_decode(gcodec72, synth.pack_words(lo, hi, None, 72))
+    assert np.array_equal(got, ocodec72.decode_batch(lo, hi))
+
+
+def test_decode72_out_of_range(gcodec72, ocodec72):
+    N = ocodec72.n_points
+    idx = [0, N - 1, N, N + 7, 2**72 - 1]
+    lo, hi = split128(idx)
+    got = gpu_decode(gcodec72, synth.pack_words(lo, hi, None, 72))
+    assert gcodec72.get_error() == 1
+    assert np.array_equal(got, ocodec72.decode_batch(lo, hi))
+    assert (got[2:] == 0).all()
+
+
+@pytest.mark.parametrize("rows,K,batch,mode", [(97, 1000, 1, 1), (64, 24 * 37, 4, 0), (40, 2000, 16, 1)])
+def test_gemm72_ragged(gcodec72, ocodec72, rows, K, batch, mode):
+    def norms(lo, hi):
+        v = ocodec72.decode_batch(lo, hi).astype(np.float64)
+        return np.sqrt((v ** 2).sum(1))
+    layer = Layer(72, rows, K, batch, 30 + batch, ocodec72.n_points, mode, norms_fn=norms)
+    y = run_gemm(gcodec72, layer)
+    ref = oracle_gemm(ocodec72, layer)
+    assert max_rel_err(y, ref) < GEMV_RTOL
+
+
+@pytest.mark.parametrize("rows,K,batch", [(28672, 8192, 1), (8192, 28672, 8)])
+def test_gemm72_full_size_sampled_rows(gcodec72, ocodec72, rows, K, batch):
+    """Llama-2-70B layer shapes at 3 bits (72-bit indices in 16-byte words); 64 sampled rows."""
+    layer = Layer(72, rows, K, batch, 40 + batch, ocodec72.n_points, 1)
+    y = run_gemm(gcodec72, layer)
+    rs = np.sort(np.random.default_rng(rows).choice(rows, 64, replace=False))
+    ref = oracle_gemm(ocodec72, layer, rows=rs)
+    assert max_rel_err(y[:, rs], ref) < GEMV_RTOL
