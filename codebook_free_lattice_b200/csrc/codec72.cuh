@@ -35,7 +35,7 @@ static_assert(sizeof(Rec72) == 80, "Rec72 layout");
 
 constexpr int kGuideBits72 = 16;                  // 65536 buckets over [0, 2^72)
 
-struct Smem72 {
+struct alignas(16) Smem72 {
     uint32_t golay_mask[4096];
     uint32_t golay_weight[4096];
     unsigned long long rc[32];                    // ceil(2^64 / c), c = 2..24 (0 for c <= 1)

@@ -12,6 +12,7 @@
 
 #include "../../include/llvq.h"
 #include "kernels.cuh"
+#include "kernels_tc.cuh"
 #include "tables.h"
 
 using namespace llvq;
@@ -32,6 +33,9 @@ struct llvq_codec {
 namespace {
 
 thread_local std::string g_last_error;
+
+// batches from this size up run on the tensor cores (k_gemm_tc); smaller ones on the CUDA cores
+constexpr int kTensorCoreMinBatch = 8;
 
 // smallest double >= n / d for small positive integers (directed rounding of the host division)
 double round_up_ratio(double n, double d) {
@@ -217,9 +221,29 @@ void set_gemm_attrs(std::integer_sequence<int, Bs...>) {
     (cudaFuncSetAttribute(k_gemm<D, Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024), ...);
 }
 
+// Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
+// CTAs; the output is zeroed here because the splits add into it.
+template <class D>
+cudaError_t launch_gemm_tc(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
+                           int batch, float *Y, cudaStream_t st) {
+    const int mt = (w->rows + kTcRows - 1) / kTcRows;
+    const int nchunks = (w->blocks_per_row + kTcBlocks - 1) / kTcBlocks;
+    const int target = c->num_sms * tc_ctas_per_sm<D>();
+    int splits = std::max(1, std::min(nchunks, (target + mt - 1) / mt));
+    const int cps = (nchunks + splits - 1) / splits;
+    splits = (nchunks + cps - 1) / cps;
+    cudaError_t e = cudaMemsetAsync(Y, 0, (size_t)batch * w->rows * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    k_gemm_tc<D><<<dim3(mt, splits), 512, sizeof(TcSmem<D>), st>>>(
+        a, (const typename D::Word *)w->words, w->row_pitch_words, w->rows, w->blocks_per_row, batch, w->gain_mode,
+        (const __half *)w->gains, (const __half *)X, Y, cps, c->d_flags);
+    return cudaGetLastError();
+}
+
 template <class D>
 cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
                           int batch, float *Y, cudaStream_t s) {
+    if (batch >= kTensorCoreMinBatch) return launch_gemm_tc<D>(c, a, w, X, batch, Y, s);
     switch (batch) {
         case 1: return launch_gemm<D, 1>(c, a, w, X, Y, s);
         case 2: return launch_gemm<D, 2>(c, a, w, X, Y, s);
@@ -312,6 +336,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::call_once(once, [] {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
+        cudaFuncSetAttribute(k_gemm_tc<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec48>));
+        cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
         set_gemm_attrs<Dec48>(std::make_integer_sequence<int, 16>{});
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, 16>{});
     });

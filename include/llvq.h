@@ -53,7 +53,9 @@ typedef enum {
 } llvq_gain_mode;
 
 /* Sticky device flags returned by llvq_get_error. */
-#define LLVQ_FLAG_INDEX_RANGE 0x1u /* some index was >= N_M (its block decoded to zero) */
+#define LLVQ_FLAG_INDEX_RANGE 0x1u  /* some index was >= N_M (its block decoded to zero) */
+#define LLVQ_FLAG_WAIT_TIMEOUT 0x2u /* a bounded wait for the tensor cores gave up; the output of
+                                       that call is incomplete */
 
 /* Opaque codec: owns the decode tables of one index budget on one device. */
 typedef struct llvq_codec llvq_codec;
@@ -96,14 +98,17 @@ llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t wo
                         int8_t *d_out, void *stream);
 
 /* Fused decode-and-multiply, batch 1: d_y[r] = sum_j scale(r, j) * <v(r, j), x[24 j .. 24 j + 23]>
- * with fp32 accumulation.  d_x: device fp16 [blocks_per_row * 24] (zero beyond cols), 4-byte
- * aligned.  d_y: device fp32 [rows], overwritten. */
+ * with fp32 accumulation.  d_x: device fp16 [blocks_per_row * 24] (zero beyond cols), 16-byte
+ * aligned.  d_y: device fp32 [rows], 4-byte aligned, overwritten. */
 llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void *d_x, float *d_y,
                       void *stream);
 
 /* Fused decode-and-multiply for 1 <= batch <= 16: d_Y[b][r] for activations d_X [batch][nb*24]
- * (fp16, row stride nb*24, zero beyond cols).  Each block is decoded once for the whole batch.
- * d_Y: device fp32 [batch][rows], overwritten. */
+ * (fp16, row stride nb*24, zero beyond cols, 16-byte aligned).  Each block is decoded once for the
+ * whole batch.  d_Y: device fp32 [batch][rows], overwritten.  Batches of 8 or more run on the
+ * tensor cores: decoded 128-row tiles (exact fp16 integers) times a block-diagonal activation
+ * tile, per-block partial dots in TMEM, gains applied in fp32; that path zeroes d_Y on the stream
+ * first and adds K-split partial sums atomically (summation order not fixed). */
 llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, const void *d_X,
                                  int32_t batch, float *d_Y, void *stream);
 

@@ -189,7 +189,23 @@ def test_gemm_batch_equals_gemv_columns(gcodec, ocodec):
         assert max_rel_err(yb[0], Y[b]) < 1e-5
 
 
-@pytest.mark.parametrize("rows,K,batch", [(4096, 4096, 1), (11008, 4096, 4), (4096, 11008, 1)])
+@pytest.mark.parametrize("bits,rows,K", [(48, 300, 24 * 45 + 5), (72, 130, 24 * 9)])
+def test_tensor_core_batch_equals_column_gemvs(gcodec, gcodec72, ocodec, ocodec72, bits, rows, K):
+    """Batch 16 (tensor-core path, ragged 128-row tile and ragged 4-block chunk) against 16
+    separate batch-1 products (CUDA-core path)."""
+    g, o = (gcodec, ocodec) if bits == 48 else (gcodec72, ocodec72)
+    layer = Layer(bits, rows, K, 16, 60 + bits, o.n_points, 1)
+    Y = run_gemm(g, layer)
+    for b in range(16):
+        sub = Layer(bits, rows, K, 16, 60 + bits, o.n_points, 1)
+        sub.x = layer.x[b:b + 1].copy()
+        sub.batch = 1
+        assert max_rel_err(run_gemm(g, sub)[0], Y[b]) < 1e-4
+    assert max_rel_err(Y, oracle_gemm(o, layer)) < GEMV_RTOL
+
+
+@pytest.mark.parametrize("rows,K,batch", [(4096, 4096, 1), (11008, 4096, 4), (4096, 11008, 1),
+                                          (28672, 8192, 16)])
 def test_gemm_full_size_sampled_rows(gcodec, ocodec, rows, K, batch):
     """Llama-2-7B layer shapes at the bench's launch configuration; the oracle checks a seeded
     sample of 256 rows."""
