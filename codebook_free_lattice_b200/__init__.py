@@ -56,19 +56,29 @@ def lib() -> C.CDLL:
         L.llvq_gemm_smallbatch.argtypes = [C.c_void_p, C.POINTER(llvq_weight), C.c_void_p, C.c_int32,
                                            C.c_void_p, C.c_void_p]
         L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
+        L.llvq_decode_noalloc.argtypes = [C.c_int32, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
         for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
-                  "llvq_gemm_smallbatch", "llvq_get_error"):
+                  "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
 
 
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
-            "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string")
+            "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
+            "llvq_decode_noalloc")
 
 
 def llvq_status_string(status: int) -> str:
     return lib().llvq_status_string(status).decode()
+
+
+def llvq_decode_noalloc(words, out, n: int | None = None, stream=None):
+    """48-bit decode through the entry point that allocates no device memory (its tables live
+    in a static device array; see include/llvq.h).  words: device int64 words; out: int8 [n, 24]."""
+    n = out.shape[0] if n is None else n
+    _check(lib().llvq_decode_noalloc(48, C.c_void_p(words.data_ptr()), 8, n, C.c_void_p(out.data_ptr()),
+                                     _stream(stream)), "llvq_decode_noalloc")
 
 
 def _check(status: int, what: str):

@@ -278,7 +278,79 @@ llvq_status check_weight(const llvq_codec *c, const llvq_weight *w) {
 
 }  // namespace
 
+// ---- decode without any device allocation -----------------------------------------------
+// A caller that cannot allocate device memory (inside a CUDA-graph capture, under a framework's
+// memory pool that owns every byte, in a plug-in with a fixed device budget) cannot create a
+// codec, because llvq_codec_create allocates its tables with cudaMalloc.  llvq_decode_noalloc
+// keeps the decode kernel's non-input, non-output global memory -- the 48-bit table image and
+// the sticky flag word -- in this file-scope device array instead.  Every GPU that loads the
+// library holds it (kNoAllocScratchBytes) until the process exits.
+constexpr size_t kNoAllocFlagOffset = (sizeof(Smem48) + 255) / 256 * 256;
+constexpr size_t kNoAllocScratchBytes = kNoAllocFlagOffset + 256;     // 66,304 B
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+unsigned char *g_noalloc_ptr[kNoAllocMaxDevices] = {};   // device address of the array, per device
+unsigned long long g_noalloc_npoints = 0;
+
+// Once per device, with that device current: build the 48-bit table image on the host, find the
+// array's device address and copy the image in (synchronous; no allocation on the device).
+llvq_status noalloc_setup(int dev, unsigned char **out) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev]) { *out = g_noalloc_ptr[dev]; return LLVQ_OK; }
+    HostTables T;
+    std::string err;
+    if (!build_host_tables(48, T, err)) { g_last_error = err; return LLVQ_ERR_UNSUPPORTED; }
+    std::vector<unsigned char> image(sizeof(Smem48));
+    const llvq_status st = build_image48(T, *reinterpret_cast<Smem48 *>(image.data()), err);
+    if (st != LLVQ_OK) { g_last_error = err; return st; }
+    unsigned char *ptr = nullptr;
+    if (cudaGetSymbolAddress((void **)&ptr, g_noalloc_scratch) != cudaSuccess || !ptr ||
+        cudaMemcpy(ptr, image.data(), image.size(), cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48)) !=
+            cudaSuccess) {
+        cudaGetLastError();
+        return LLVQ_ERR_CUDA;
+    }
+    g_noalloc_npoints = (unsigned long long)T.n_points;
+    g_noalloc_ptr[dev] = ptr;
+    *out = ptr;
+    return LLVQ_OK;
+}
+}  // namespace
+
 extern "C" {
+
+llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t word_bytes, int64_t n,
+                                int8_t *d_out, void *stream) {
+    if (index_bits != 48) {
+        g_last_error = "llvq_decode_noalloc holds only the 48-bit table image (64.4 KiB); larger budgets need a codec";
+        return LLVQ_ERR_UNSUPPORTED;
+    }
+    if (n < 0 || word_bytes != 8) return LLVQ_ERR_ARG;
+    if (n == 0) return LLVQ_OK;
+    if (!d_words || !d_out || !aligned(d_words, 8) || !aligned(d_out, 8)) return LLVQ_ERR_ARG;
+    int dev = -1, nsm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNoAllocMaxDevices ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LLVQ_ERR_CUDA;
+    unsigned char *ptr = nullptr;
+    const llvq_status st = noalloc_setup(dev, &ptr);
+    if (st != LLVQ_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned *flags = reinterpret_cast<unsigned *>(ptr + kNoAllocFlagOffset);
+    if (cudaMemsetAsync(flags, 0, sizeof(unsigned), s) != cudaSuccess) return LLVQ_ERR_CUDA;
+    const int threads = 512;
+    const long long want = (n + threads - 1) / threads;
+    const int grid = (int)std::max(1LL, std::min(want, (long long)nsm * Dec48::kCtasPerSm));
+    k_decode<Dec48><<<grid, threads, sizeof(Smem48), s>>>(
+        Dec48::Args{reinterpret_cast<const Smem48 *>(ptr), g_noalloc_npoints},
+        (const Dec48::Word *)d_words, n, d_out, flags);
+    return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
+}
+
 
 const char *llvq_status_string(llvq_status s) {
     switch (s) {

@@ -112,6 +112,20 @@ llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void 
 llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, const void *d_X,
                                  int32_t batch, float *d_Y, void *stream);
 
+/* Decode without any device allocation, for callers that cannot call cudaMalloc -- for
+ * example code running inside a CUDA-graph capture, or a plug-in whose device memory is owned by
+ * a framework allocator.  The paper has no counterpart; this is a packaging variant of
+ * llvq_decode for the 48-bit budget only (index_bits must be 48, word_bytes 8; anything else is
+ * LLVQ_ERR_UNSUPPORTED / LLVQ_ERR_ARG).  The decode tables and the status word live in one
+ * static device array inside the library (66,304 bytes on every device that loads it, held until
+ * the process exits) instead of a codec.  The first call on a device builds the tables on the
+ * host and copies them in synchronously, so make that first call before any stream capture.
+ * Calls share the array: indices >= N_M still decode to the zero vector (a coded point is never
+ * zero), and the shared status word is cleared by every call, so calls that overlap on the GPU
+ * race on it.  Arguments as for llvq_decode. */
+llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t word_bytes, int64_t n,
+                                int8_t *d_out, void *stream);
+
 /* Synchronise `stream`, return the sticky device flags raised since the last call in *flags
  * and clear them.  Returns LLVQ_ERR_DEVICE_FLAG when any flag was set, LLVQ_OK otherwise. */
 llvq_status llvq_get_error(const llvq_codec *codec, void *stream, uint32_t *flags);
