@@ -106,7 +106,7 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def make_layer_copies(torch, codec, R, dev):
+def make_layer_copies(torch, codec, R, dev, batch=1):
     from codebook_free_lattice_b200 import synth
     n = ROWS * NB
     lo, _ = synth.uniform_indices(synth.rng(CONFIG_ID, 0), n * R, codec.n_points, 48)
@@ -114,7 +114,7 @@ def make_layer_copies(torch, codec, R, dev):
     words = torch.from_numpy(synth.pack_words(lo, None, codes, 48).view(np.int64)).to(dev)
     words = words.view(R, ROWS, NB)
     gains = torch.from_numpy(synth.chi24_tables(synth.rng(CONFIG_ID, 2), ROWS).view(np.int16)).to(dev)
-    xs = synth.activations(synth.rng(CONFIG_ID, 3), R, K)       # one activation row per copy
+    xs = synth.activations(synth.rng(CONFIG_ID, 3), R * batch, K).reshape(R, batch, -1)  # per copy
     return words, gains, xs
 
 
@@ -167,6 +167,123 @@ def cpu_baseline(steps_seconds=12.0):
             "vectors_per_s": done_rows * NB / el}
 
 
+# ------------------------------------------------------------------ secondary measurements
+SWEEP_CASES = [
+    # (name, rows, K, index_bits, batch)
+    ("4096x4096", 4096, 4096, 48, 1),
+    ("11008x4096 (gate/up)", 11008, 4096, 48, 1),
+    ("11008x4096 (gate/up)", 11008, 4096, 48, 4),
+    ("4096x11008 (down)", 4096, 11008, 48, 1),
+    ("4096x11008 (down)", 4096, 11008, 48, 4),
+    ("28672x8192", 28672, 8192, 48, 1),
+    ("28672x8192", 28672, 8192, 48, 8),
+    ("28672x8192", 28672, 8192, 48, 16),
+    ("8192x28672", 8192, 28672, 48, 1),
+    ("8192x28672", 8192, 28672, 48, 16),
+    ("28672x8192", 28672, 8192, 72, 1),
+    ("28672x8192", 28672, 8192, 72, 16),
+    ("8192x28672", 8192, 28672, 72, 1),
+    ("8192x28672", 8192, 28672, 72, 8),
+]
+LLAMA7B_LAYER = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
+                 ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
+
+
+def _graph_time(torch, stream, body, reps=10, warm=3):
+    with torch.cuda.stream(stream):
+        body()
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        body()
+    with torch.cuda.stream(stream):
+        for _ in range(warm):
+            g.replay()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        for _ in range(reps):
+            g.replay()
+        e.record(stream)
+    torch.cuda.synchronize()
+    del g
+    return s.elapsed_time(e) / 1e3 / reps
+
+
+def _layers(torch, codec, dev, shapes, bits, batch, seed):
+    """Packed words, table gains and activations for each (rows, K) in shapes (distinct data)."""
+    import codebook_free_lattice_b200 as L
+    from codebook_free_lattice_b200 import synth
+    out = []
+    for i, (rows, K) in enumerate(shapes):
+        nb = -(-K // 24)
+        lo, hi = synth.uniform_indices(synth.rng(seed + i, 0), rows * nb, codec.n_points, bits)
+        codes = synth.gain_codes(synth.rng(seed + i, 1), rows * nb)
+        w = torch.from_numpy(np.ascontiguousarray(synth.pack_words(lo, hi, codes, bits)).view(np.int64)).to(dev)
+        g = torch.from_numpy(synth.chi24_tables(synth.rng(seed + i, 2), rows).view(np.int16)).to(dev)
+        x = torch.from_numpy(synth.activations(synth.rng(seed + i, 3), batch, K).view(np.int16)).to(dev)
+        y = torch.empty((batch, rows), dtype=torch.float32, device=dev)
+        out.append((codec.weight(w, g, rows, K, L.LLVQ_GAIN_U8_TABLE), w, g, x, y))
+    return out
+
+
+def _run_layers(codec, layers, batch, stream):
+    for wt, _, _, x, y in layers:
+        if batch == 1:
+            codec.gemv(wt, x, y, stream=stream)
+        else:
+            codec.gemm(wt, x, y, batch, stream=stream)
+
+
+def sweep(torch, dev):
+    """One JSON line per (layer, bits, batch): fused LLVQ product time against cuBLAS fp16
+    (torch.matmul on identical shapes), inputs larger than L2 in both arms; then the full
+    Llama-2-7B-shaped decoder stack (32 layers x q,k,v,o,gate,up,down) at 2 and 3 bits."""
+    import codebook_free_lattice_b200 as L
+    peak, _ = measured_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    stream = torch.cuda.Stream(device=dev)
+    codecs = {48: L.Codec(48), 72: L.Codec(72)}
+    for name, rows, K, bits, batch in SWEEP_CASES:
+        codec = codecs[bits]
+        nb = -(-K // 24)
+        wb = 8 if bits == 48 else 16
+        copies = max(1, int(np.ceil(3 * l2 / (rows * nb * wb))))
+        layers = _layers(torch, codec, dev, [(rows, K)] * copies, bits, batch, 500 + rows % 97)
+        t = _graph_time(torch, stream, lambda: _run_layers(codec, layers, batch, stream)) / copies
+        assert codec.get_error(stream) == 0
+        alg = rows * nb * wb + rows * 512 + batch * nb * 48 + batch * rows * 4
+        del layers
+        fcopies = max(1, int(np.ceil(3 * l2 / (rows * K * 2))))
+        Ws = [torch.randn(rows, K, dtype=torch.float16, device=dev) for _ in range(fcopies)]
+        xs = torch.randn(batch, K, dtype=torch.float16, device=dev)
+        tc = _graph_time(torch, stream, lambda: [torch.matmul(xs, W.t()) for W in Ws]) / fcopies
+        del Ws
+        print(json.dumps({"sweep": name, "index_bits": bits, "batch": batch, "us": t * 1e6,
+                          "GBps": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / peak,
+                          "decoded_vectors_per_s": rows * nb / t, "cublas_fp16_us": tc * 1e6,
+                          "speedup_vs_fp16": tc / t, "layer_copies": copies}), flush=True)
+        torch.cuda.empty_cache()
+    for bits in (48, 72):
+        codec = codecs[bits]
+        shapes = [(r, k) for _ in range(32) for (_, r, k) in LLAMA7B_LAYER]
+        layers = _layers(torch, codec, dev, shapes, bits, 1, 900 + bits)
+        t = _graph_time(torch, stream, lambda: _run_layers(codec, layers, 1, stream), reps=5)
+        assert codec.get_error(stream) == 0
+        wb = 8 if bits == 48 else 16
+        alg = sum(r * -(-k // 24) * wb + r * 512 + -(-k // 24) * 48 + r * 4 for r, k in shapes)
+        del layers
+        torch.cuda.empty_cache()
+        Ws = [torch.randn(r, k, dtype=torch.float16, device=dev) for r, k in shapes]
+        xs = {k: torch.randn(1, k, dtype=torch.float16, device=dev) for k in (4096, 11008)}
+        tc = _graph_time(torch, stream, lambda: [torch.matmul(xs[W.shape[1]], W.t()) for W in Ws], reps=5)
+        del Ws
+        torch.cuda.empty_cache()
+        print(json.dumps({"sweep": "llama-2-7b stack (224 GEMVs)", "index_bits": bits, "batch": 1,
+                          "ms": t * 1e3, "GBps": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / peak,
+                          "cublas_fp16_ms": tc * 1e3, "speedup_vs_fp16": tc / t}), flush=True)
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -200,8 +317,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-n", type=int, default=28672 * 342,
                     help="indices for the llvq_decode throughput line (default: the 28672x8192 layer)")
-    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode"],
-                    help="decode: time llvq_decode alone (profiling aid)")
+    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "sweep"],
+                    help="decode: time llvq_decode alone (profiling aid); sweep: every layer shape, "
+                         "budget and batch against cuBLAS fp16, plus the full 7B stack")
+    ap.add_argument("--batch", type=int, default=1, help="gemv mode: batch (1 = the metric's workload)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -226,25 +345,35 @@ def main():
         if rank == 0:
             print(json.dumps({"mode": "decode", **r}), flush=True)
         return 0
+    if args.mode == "sweep":
+        if rank == 0:
+            sweep(torch, dev)
+        return 0
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     layer_bytes = ROWS * NB * 8
     R = args.copies or int(np.ceil(3 * l2 / layer_bytes)) + 1
-    words, gains, xs = make_layer_copies(torch, codec, R, dev)
-    x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)                 # [R, K_pad]
-    y_dev = torch.empty((R, ROWS), dtype=torch.float32, device=dev)
+    B = args.batch
+    words, gains, xs = make_layer_copies(torch, codec, R, dev, B)
+    x_dev = torch.from_numpy(xs.view(np.int16)).to(dev)                 # [R, B, K_pad]
+    y_dev = torch.empty((R, B, ROWS), dtype=torch.float32, device=dev)
     ws = [codec.weight(words[i], gains, ROWS, K, L.LLVQ_GAIN_U8_TABLE) for i in range(R)]
+
+    def run_all():
+        for i in range(R):
+            if B == 1:
+                codec.gemv(ws[i], x_dev[i], y_dev[i], stream=stream)
+            else:
+                codec.gemm(ws[i], x_dev[i], y_dev[i], B, stream=stream)
 
     stream = torch.cuda.Stream(device=dev)
     with torch.cuda.stream(stream):
-        for i in range(R):                                              # warm the path once
-            codec.gemv(ws[i], x_dev[i], y_dev[i], stream=stream)
+        run_all()                                                       # warm the path once
     stream.synchronize()
     assert codec.get_error(stream) == 0
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
-        for i in range(R):
-            codec.gemv(ws[i], x_dev[i], y_dev[i], stream=stream)
+        run_all()
 
     def barrier():
         if world > 1:
@@ -271,7 +400,7 @@ def main():
 
     # end to end through the public API: pinned host activations in, outputs back out
     x_host = torch.from_numpy(xs.view(np.int16)).pin_memory()
-    y_host = torch.empty((R, ROWS), dtype=torch.float32).pin_memory()
+    y_host = torch.empty((R, B, ROWS), dtype=torch.float32).pin_memory()
 
     def e2e_step():
         x_dev.copy_(x_host, non_blocking=True)
@@ -289,13 +418,13 @@ def main():
         secs, secs_e2e = t.tolist()
 
     launches = args.steps * R
-    bytes_launch = algorithmic_bytes()
+    bytes_launch = algorithmic_bytes(batch=B)
     per_launch_s = secs / launches
     gbs = bytes_launch / per_launch_s / 1e9
     value = gbs * world
     peak, peak_kind = measured_peaks()
-    h2d = R * NB * 24 * 2
-    d2h = R * ROWS * 4
+    h2d = R * B * NB * 24 * 2
+    d2h = R * B * ROWS * 4
     e2e_gbs = bytes_launch * launches / secs_e2e / 1e9 * world
 
     if rank == 0:
@@ -303,8 +432,9 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "rows": ROWS, "cols": K, "blocks_per_row": NB,
-                       "batch": 1, "index_bits": 48, "layer_copies_per_step": R,
+            "config": {"workload": WORKLOAD if B == 1 else WORKLOAD.replace("batch 1", f"batch {B}"),
+                       "rows": ROWS, "cols": K, "blocks_per_row": NB,
+                       "batch": B, "index_bits": 48, "layer_copies_per_step": R,
                        "l2_policy": f"inputs larger than L2: {R} distinct layer copies "
                                     f"({R * layer_bytes / 2**20:.0f} MiB of words) per step",
                        "parallelism": f"replicas x{world}"},
