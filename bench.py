@@ -42,6 +42,30 @@ def algorithmic_bytes(rows=ROWS, nb=NB, batch=1) -> int:
     return rows * nb * 8 + rows * 512 + batch * nb * 24 * 2 + batch * rows * 4
 
 
+def kernel_sources_hash() -> str:
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "codebook_free_lattice_b200", "csrc", "*"))):
+        h.update(os.path.basename(f).encode())
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """DRAM bytes per launch of the metric's kernel from the committed ncu capture, or None when
+    the kernel sources changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f)
+        if rec.get("kernel_sources_sha256") == kernel_sources_hash():
+            return int(rec["traffic_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -441,7 +465,7 @@ def main():
             "us_per_layer": per_launch_s * 1e6,
             "decoded_vectors_per_s": ROWS * NB / per_launch_s * world,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": None,
+                         "frac": gbs / peak, "traffic": measured_traffic() if B == 1 else None,
                          "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
             "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
