@@ -9,13 +9,16 @@
 //   2. r, s, I'' by one fp64 division by A with an exact integer correction;
 //   3. codeword from the shared-memory Golay tables (odd: T by mask order; even: S among the
 //      codewords of weight k);
-//   4. the lexicographic rank I'' of the magnitude arrangement is unranked coordinate by
-//      coordinate as exact arithmetic decoding: f = I''/P in fp64 rounded upward; at a
-//      coordinate whose side (codeword side or not) has L places left, the slot floor(f * L)
-//      picks the magnitude group among that side's remaining items (byte-SIMD search of the
-//      cumulative counts) and f <- (f * L - start(group)) / count(group).  Directed rounding keeps
-//      f above the exact rational with an error far below 1/(remaining arrangements) for
-//      P < 2^33, so every slot is exact.  The loop stays on the FMA, ALU and fp64 pipes;
+//   4. the arrangement rank I'' is unranked coordinate by coordinate as exact arithmetic
+//      decoding.  An even class ranks the magnitudes on its codeword S and on the other
+//      positions separately, I'' = p_S + P_S p_C, each lexicographically; an odd class has one
+//      coordinate set.  f_C = I''/P (fp64, rounded upward) equals (p_C + p_S/P_S)/P_C from above
+//      and decodes the positions off S; f_S = f_C P_C - p_C = p_S/P_S from above decodes S.  At a
+//      coordinate whose set has L places left, the slot floor(f * L) picks the magnitude group
+//      among that set's remaining items (byte-SIMD search of the cumulative counts) and
+//      f <- (f * L - start(group)) / count(group).  Directed rounding keeps each f above its exact
+//      rational with an error far below 1/(remaining arrangements) for P < 2^33, so every slot
+//      is exact.  The loop stays on the FMA, ALU and fp64 pipes;
 //   5. magnitudes and sign flags by byte permutation of the class's group tables, then signs.
 #pragma once
 #include "device_common.cuh"
@@ -38,13 +41,15 @@ struct alignas(16) Rec48 {
     uint8_t flags;             // bit0 odd coset, bit1 parity target (sum|x|/4 odd)
     uint8_t m;                 // shell
     uint16_t wbase;            // even: first by-weight Golay slot of weight k
+    double PC;                 // arrangements off S (even; exact, < 2^24), 1 for odd classes
+    double pad;
 };
-static_assert(sizeof(Rec48) == 48, "Rec48 layout");
+static_assert(sizeof(Rec48) == 64, "Rec48 layout");
 
 constexpr int kGuideBits48 = 11;                  // 2048 buckets over [0, 2^48)
 constexpr int kGuideShift48 = 48 - kGuideBits48;
 
-// Shared-memory image of the 48-bit decode tables (one copy per CTA, 66 KB).
+// Shared-memory image of the 48-bit decode tables (one copy per CTA, 72 KB).
 struct Smem48 {
     uint32_t golay_mask[4096];
     uint32_t golay_weight[4096];
@@ -65,7 +70,7 @@ struct Dec48 {
         unsigned long long npoints;
     };
     static constexpr int kWordBytes = 8;
-    static constexpr int kCtasPerSm = 3;          // 40 registers, 66 KB shared per CTA
+    static constexpr int kCtasPerSm = 3;          // 40 registers, 72 KB shared per CTA
 
     __device__ static Word load(const Word *p) { return __ldg(p); }
     __device__ static int gain_code(const Word &w) { return (int)((w >> 48) & 0xFFu); }
@@ -101,7 +106,9 @@ struct Dec48 {
         const uint32_t side0 = odd ? 0xFFFFFFu : word;
         // 4. arrangement.  Byte b of cumB is 0x7F + C_<=b (remaining items of groups 0..b),
         //    biased one below the guard bit so the byte-wise subtraction of the slot never borrows.
-        double f = __dmul_ru((double)p, R.invP);
+        double fC = __dmul_ru((double)p, R.invP);                   // (p_C + p_S/P_S) / P_C
+        const double g0 = __dmul_ru(fC, R.PC);                       // p_C + p_S/P_S
+        double fS = __dadd_ru(g0, 0x1p52 - __dadd_rz(g0, 0x1p52));   // p_S / P_S
         uint32_t cumB = R.cum + 0x7F7F7F7Fu;
         int L0 = R.nS, L1 = 24 - R.nS;
         uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u,
@@ -111,7 +118,7 @@ struct Dec48 {
             const bool on0 = side0 & (1u << i);
             const int L = on0 ? L0 : L1;
             const int off = on0 ? 0 : L0;
-            const double g = __dmul_ru(f, small_to_double((uint32_t)L));
+            const double g = __dmul_ru(on0 ? fS : fC, small_to_double((uint32_t)L));
             const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52)) + (uint32_t)off;
             const uint32_t u = cumB - slot * 0x01010101u;            // bit 7 of byte b: C_<=b > slot
             const uint32_t dm = (u >> 7) & 0x01010101u;              // one per group >= grp
@@ -121,7 +128,8 @@ struct Dec48 {
             const uint32_t enB = __byte_perm(cumB, 0x7F7F7F7Fu + (uint32_t)(24 - i), esel);
             const uint32_t cnt = min(enB - stB, 31u);                        // in 1..24
             const uint32_t stl = stB - 0x7F7F7F7Fu - (uint32_t)off;
-            f = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), S.invc[cnt]);
+            const double fn = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), S.invc[cnt]);
+            if (on0) fS = fn; else fC = fn;
             cumB -= dm;                                              // groups >= grp lose one item
             L0 -= on0 ? 1 : 0;
             L1 -= on0 ? 0 : 1;

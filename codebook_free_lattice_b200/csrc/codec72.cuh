@@ -4,15 +4,17 @@
 // Same hierarchy as the 48-bit decoder ("Leech Lattice Vector Quantization for Efficient LLM
 // Compression", papernotes.org notes, 方法详解 / 关键设计 2), with wider arithmetic:
 //   - indices are 72-bit (word = two little-endian 64-bit halves; gain code in bits 72..79);
-//   - class records (80 B) and the guide table on the top 16 index bits live in global memory
+//   - class records (96 B) and the guide table on the top 16 index bits live in global memory
 //     (L2-resident, 9.5 MB), the Golay tables in shared memory;
 //   - I_class < 2^63, so r, s, I'' come from one 64-bit division by A;
 //   - arrangement counts reach P ~ 2^50.2, beyond fp64, so the arithmetic decoding state is
-//     a 64-bit fixed-point fraction phi ~ 2^64 I''/P kept above the exact value: slot =
-//     high word of phi * L, and phi <- (slot_in_group * 2^64 + low word) * R_c with
-//     R_c = ceil(2^64 / c) (plus one).  Each step adds at most c + 1 units of error, and
-//     24 * 577 * P <= 2^64 for every class, so every slot is exact (the bound argument is
-//     in the design notes);
+//     a 64-bit fixed-point fraction kept above the exact value: slot = high word of phi * L,
+//     and phi <- (slot_in_group * 2^64 + low word) * R_c with R_c = ceil(2^64 / c) (plus one).
+//     An even class ranks S and the other positions separately (I'' = p_S + P_S p_C):
+//     phi_C ~ 2^64 I''/P decodes the positions off S and phi_S = phi_C * P_C mod 2^64
+//     ~ 2^64 p_S/P_S decodes S.  Each step adds at most c + 1 units of error, the start
+//     error of phi_S is below 2 P_C units, and 24 * 577 * P <= 2^64 for every class, so every
+//     slot is exact (the bound argument is in the design notes);
 //   - up to 9 magnitude groups: cumulative counts in 8 bytes; group 8 patched in when present.
 #pragma once
 #include "device_common.cuh"
@@ -30,8 +32,10 @@ struct alignas(16) Rec72 {
     uint8_t nS, B, flags, m, ngroups, pad0;  // flags: bit0 odd coset, bit1 parity target
     uint16_t wbase, pad1;
     uint32_t pad2;
+    unsigned long long PC;                   // arrangements off S (even), 1 for odd classes
+    unsigned long long pad3;
 };
-static_assert(sizeof(Rec72) == 80, "Rec72 layout");
+static_assert(sizeof(Rec72) == 96, "Rec72 layout");
 
 constexpr int kGuideBits72 = 16;                  // 65536 buckets over [0, 2^72)
 
@@ -86,7 +90,8 @@ struct Dec72 {
         const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min(R.wbase + r, 4095u)];
         const uint32_t side0 = odd ? 0xFFFFFFu : word;
         // 4. arrangement in 64-bit fixed point
-        unsigned long long phi = p * R.Rint + __umul64hi(p, R.Rfrac) + 1ull;
+        unsigned long long phiC = p * R.Rint + __umul64hi(p, R.Rfrac) + 1ull;   // off S
+        unsigned long long phiS = phiC * R.PC;                                    // on S
         uint32_t clo4 = (uint32_t)R.cum + 0x7F7F7F7Fu, chi4 = (uint32_t)(R.cum >> 32) + 0x7F7F7F7Fu;
         int L0 = R.nS, L1 = 24 - R.nS;
         uint32_t sel[6] = {0, 0, 0, 0, 0, 0};
@@ -95,6 +100,7 @@ struct Dec72 {
             const bool on0 = side0 & (1u << i);
             const uint32_t L = (uint32_t)(on0 ? L0 : L1);
             const uint32_t off = on0 ? 0u : (uint32_t)L0;
+            const unsigned long long phi = on0 ? phiS : phiC;
             const unsigned long long frac = phi * L;
             const uint32_t slot = (uint32_t)__umul64hi(phi, L) + off;
             const uint32_t ulo = clo4 - slot * 0x01010101u, uhi = chi4 - slot * 0x01010101u;
@@ -107,7 +113,8 @@ struct Dec72 {
             const uint32_t cnt = min(en - st, 31u);                            // in 1..24
             const unsigned long long rc = S.rc[cnt];
             const unsigned long long within = slot - st;                       // < cnt
-            phi = cnt == 1u ? frac + 1ull : within * rc + __umul64hi(frac, rc) + 1ull;
+            const unsigned long long phn = cnt == 1u ? frac + 1ull : within * rc + __umul64hi(frac, rc) + 1ull;
+            if (on0) phiS = phn; else phiC = phn;
             clo4 -= dlo;
             chi4 -= dhi;
             L0 -= on0 ? 1 : 0;

@@ -87,10 +87,12 @@ llvq_status build_image48(const HostTables &T, Smem48 &S, std::string &err) {
     for (int i = 0; i < nc; i++) {
         const HostClass &c = T.classes[i];
         if (c.vals.size() > 5) { err = "more than 5 magnitude groups at 48 bits"; return LLVQ_ERR_UNSUPPORTED; }
+        if (c.P >= ((u128)1 << 33) || c.P_C >= ((u128)1 << 24)) { err = "48-bit arrangement count out of range"; return LLVQ_ERR_UNSUPPORTED; }
         Rec48 &R = S.recs[i];
         R.start = (unsigned long long)c.start;
         R.invP = round_up_ratio(1.0, (double)c.P);    // P < 2^33: exact as a double
         R.invA = 1.0 / (double)c.A;
+        R.PC = (double)c.P_C;                         // < 2^24 for every 48-bit class: exact
         R.A = c.A;
         uint32_t vals = 0, gflag = 0;
         for (int g = 0; g < 4 && g < (int)c.vals.size(); g++) {
@@ -146,6 +148,7 @@ llvq_status build_image72(const HostTables &T, Smem72 &S, std::vector<Rec72> &re
             const u128 rem = two64 % c.P;               // fraction rem / P, times 2^64, rounded up
             R.Rfrac = (unsigned long long)(((rem << 64) + c.P - 1) / c.P);
         }
+        R.PC = (unsigned long long)c.P_C;
         R.cum = cum_bytes(c, 8);
         for (int g = 0; g < 8 && g < (int)c.vals.size(); g++) {
             R.vals |= (unsigned long long)c.vals[g] << (8 * g);

@@ -104,6 +104,8 @@ void shell_classes(int m, const int words_of_weight[25], std::vector<HostClass> 
                 for (auto &g : side0) p0 /= factorial(g.second);
                 for (auto &g : side1) p1 /= factorial(g.second);
                 c.P = p0 * p1;
+                c.P_S = p0;
+                c.P_C = p1;
             } else {
                 int r8 = ((signed_sum % 8) + 8) % 8;                   // sum with T empty
                 if (r8 != 4) continue;
@@ -112,6 +114,8 @@ void shell_classes(int m, const int words_of_weight[25], std::vector<HostClass> 
                 u128 p = factorial(24);
                 for (auto &g : side0) p /= factorial(g.second);
                 c.P = p;
+                c.P_S = p;
+                c.P_C = 1;
             }
             for (auto &g : side0) { c.vals.push_back(g.first); c.cnts.push_back(g.second); }
             for (auto &g : side1) { c.vals.push_back(g.first); c.cnts.push_back(g.second); }

@@ -5,7 +5,8 @@
 // and the per-class constants of the decode.  Method: "Leech Lattice Vector Quantization for
 // Efficient LLM Compression", papernotes.org notes, 方法详解 / 关键设计 2 (shell by cumulative
 // offsets, classes = magnitude multiset + even/odd coset in contiguous ranges, digits
-// r = I_class mod A, s = I' mod 2^B, I'' = lexicographic arrangement rank).
+// r = I_class mod A, s = I' mod 2^B, I'' = lexicographic arrangement rank; an even class ranks
+// its codeword positions and the other positions separately, I'' = p_S + P_S p_C).
 #pragma once
 #include <stdint.h>
 
@@ -26,7 +27,8 @@ struct HostClass {
     int n_side0 = 0;           // groups on the codeword side (even: 2-mod-4 groups; odd: all)
     uint32_t A = 0;            // Golay refinements
     int B = 0;                 // free sign bits
-    u128 P = 0;                // admissible arrangements
+    u128 P = 0;                // admissible arrangements, P_S * P_C
+    u128 P_S = 1, P_C = 1;     // even: arrangements on S / on its complement; odd: P, 1
     u128 size = 0, start = 0;  // A * 2^B * P and first global index
     int sum_abs = 0;           // sum of magnitudes
 };

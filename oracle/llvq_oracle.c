@@ -243,10 +243,14 @@ int ora_shell_counts_dp(int32_t mmax, uint64_t *lo, uint64_t *hi) {
 }
 
 /* ===================================================================================== */
-/* Lexicographic ranking of arrangements of a multiset ([notes-K2]: "I'' indexes the       */
-/* permutation in lexicographic order").  Each group of equal magnitudes has a side and   */
-/* each position a side; a group may only occupy positions of its own side.  The number   */
-/* of completions is the product of the multinomials of the two sides.                     */
+/* Lexicographic ranking of arrangements of a multiset ([notes-K2]: I'' is the rank of the */
+/* coordinate permutation in lexicographic order).  Groups are numbered in ascending       */
+/* magnitude; an arrangement is a sequence of group numbers, and sequences compare         */
+/* position by position.                                                                   */
+/* An even class has two independent coordinate sets (the codeword S carries the 2-mod-4   */
+/* magnitudes, its complement the 0-mod-4 ones); each set's sequence is ranked on its own  */
+/* and the two ranks form p = p_S + P_S * p_C (the pages do not say how the two sets       */
+/* combine; this is the reading the index format fixes).                                   */
 /* ===================================================================================== */
 static u128 fact128(int n) {
     u128 f = 1;
@@ -266,33 +270,27 @@ static void ensure_binom(void) {
     g_binom_ready = 1;
 }
 
-/* number of distinct arrangements of the remaining groups of one side:
+/* number of distinct arrangements of a multiset with counts rem[0..ng):
  * n! / prod(c_g!) = C(n, c_0) * C(n - c_0, c_1) * ... */
-static u128 multinomial_side(int ng, const int *rem, const int *gside, int side) {
+static u128 multinomial(int ng, const int *rem) {
     int n = 0;
-    for (int g = 0; g < ng; g++) if (gside[g] == side) n += rem[g];
+    for (int g = 0; g < ng; g++) n += rem[g];
     u128 r = 1;
-    for (int g = 0; g < ng; g++)
-        if (gside[g] == side) { r *= g_binom[n][rem[g]]; n -= rem[g]; }
+    for (int g = 0; g < ng; g++) { r *= g_binom[n][rem[g]]; n -= rem[g]; }
     return r;
 }
 
-static u128 completions(int ng, const int *rem, const int *gside) {
-    return multinomial_side(ng, rem, gside, 0) * multinomial_side(ng, rem, gside, 1);
-}
-
-/* unrank: position i (0..n) of side pside[i]; writes group indices to seq */
-static int arr_unrank(int ng, const int *cnt, const int *gside, int n, const int *pside, u128 p,
-                      int *seq) {
-    int rem[ORA_DIM];
-    for (int g = 0; g < ng; g++) rem[g] = cnt[g];
-    if (p >= completions(ng, rem, gside)) return -1;
+/* unrank: the p-th arrangement (lexicographic, from 0) of the multiset cnt; n = sum cnt */
+static int lex_unrank(int ng, const int *cnt, u128 p, int *seq) {
+    int rem[ORA_DIM], n = 0;
+    for (int g = 0; g < ng; g++) { rem[g] = cnt[g]; n += cnt[g]; }
+    if (p >= multinomial(ng, rem)) return -1;
     for (int i = 0; i < n; i++) {
         int chosen = -1;
-        for (int g = 0; g < ng; g++) {                    /* groups in ascending magnitude */
-            if (gside[g] != pside[i] || rem[g] == 0) continue;
+        for (int g = 0; g < ng; g++) {                    /* smallest group first */
+            if (rem[g] == 0) continue;
             rem[g]--;
-            u128 c = completions(ng, rem, gside);
+            u128 c = multinomial(ng, rem);                /* arrangements that put g at i */
             rem[g]++;
             if (p < c) { chosen = g; break; }
             p -= c;
@@ -304,35 +302,35 @@ static int arr_unrank(int ng, const int *cnt, const int *gside, int n, const int
     return 0;
 }
 
-static int arr_rank(int ng, const int *cnt, const int *gside, int n, const int *pside,
-                    const int *seq, u128 *out) {
+/* rank: number of arrangements of cnt that precede seq[0..n) lexicographically */
+static int lex_rank(int ng, const int *cnt, int n, const int *seq, u128 *out) {
     int rem[ORA_DIM];
     for (int g = 0; g < ng; g++) rem[g] = cnt[g];
     u128 p = 0;
     for (int i = 0; i < n; i++) {
         int gi = seq[i];
-        if (gi < 0 || gi >= ng || rem[gi] == 0 || gside[gi] != pside[i]) return -1;
-        for (int g = 0; g < gi; g++) {                    /* smaller magnitudes at position i */
-            if (gside[g] != pside[i] || rem[g] == 0) continue;
+        if (gi < 0 || gi >= ng || rem[gi] == 0) return -1;
+        for (int g = 0; g < gi; g++) {                    /* smaller groups at position i */
+            if (rem[g] == 0) continue;
             rem[g]--;
-            p += completions(ng, rem, gside);
+            p += multinomial(ng, rem);
             rem[g]++;
         }
         rem[gi]--;
     }
+    for (int g = 0; g < ng; g++) if (rem[g]) return -1;
     *out = p;
     return 0;
 }
 
 int ora_unrank_arrangement(int32_t nv, const int32_t *cnt, uint64_t lo, uint64_t hi, int32_t *seq) {
     ensure_binom();
-    int c[ORA_DIM], gs[ORA_DIM], ps[ORA_DIM] = {0}, s[ORA_DIM];
+    int c[ORA_DIM], s[ORA_DIM];
     int n = 0;
     if (nv < 1 || nv > ORA_DIM) return -1;
-    for (int g = 0; g < nv; g++) { c[g] = cnt[g]; gs[g] = 0; n += cnt[g]; }
+    for (int g = 0; g < nv; g++) { c[g] = cnt[g]; n += cnt[g]; }
     if (n > ORA_DIM) return -1;
-    for (int i = 0; i < n; i++) ps[i] = 0;
-    if (arr_unrank(nv, c, gs, n, ps, mk128(lo, hi), s)) return -1;
+    if (lex_unrank(nv, c, mk128(lo, hi), s)) return -1;
     for (int i = 0; i < n; i++) seq[i] = s[i];
     return 0;
 }
@@ -340,19 +338,20 @@ int ora_unrank_arrangement(int32_t nv, const int32_t *cnt, uint64_t lo, uint64_t
 int ora_rank_arrangement(int32_t nv, const int32_t *cnt, int32_t n, const int32_t *seq,
                          uint64_t *lo, uint64_t *hi) {
     ensure_binom();
-    int c[ORA_DIM], gs[ORA_DIM], ps[ORA_DIM], s[ORA_DIM];
+    int c[ORA_DIM], s[ORA_DIM];
     if (nv < 1 || nv > ORA_DIM || n > ORA_DIM) return -1;
-    for (int g = 0; g < nv; g++) { c[g] = cnt[g]; gs[g] = 0; }
-    for (int i = 0; i < n; i++) { ps[i] = 0; s[i] = seq[i]; }
+    for (int g = 0; g < nv; g++) c[g] = cnt[g];
+    for (int i = 0; i < n; i++) s[i] = seq[i];
     u128 p;
-    if (arr_rank(nv, c, gs, n, ps, s, &p)) return -1;
+    if (lex_rank(nv, c, n, s, &p)) return -1;
     split128(p, lo, hi);
     return 0;
 }
 
 /* ===================================================================================== */
-/* Classes ([notes-K2] "leader = multiset of absolute coordinates plus even/odd coset",     */
-/* contiguous index ranges).  Readings: within a shell, even-coset classes come first,    */
+/* Classes ([notes-K2]: a class is a leader's multiset of absolute coordinates together    */
+/* with its even/odd coset; classes take contiguous index ranges).  Readings: within a    */
+/* shell, even-coset classes come first,                                                  */
 /* then odd; inside a coset, classes are ordered by their magnitudes sorted descending,   */
 /* compared lexicographically ascending.                                                  */
 /*   even: k = #{|x_i| = 2 mod 4} must be a Golay weight (0, 8, 12, 16, 24); when k = 0   */
@@ -614,12 +613,64 @@ static int find_class(ora_codec *c, u128 I, ocls *out) {
     return 0;
 }
 
-/* position sides: even class -> 0 on the codeword S, 1 elsewhere; odd -> all 0 */
-static void class_sides(const ocls *o, uint32_t S, int *gside, int *pside) {
-    for (int g = 0; g < o->nvals; g++)
-        gside[g] = o->odd ? 0 : (o->vals[g] % 4 == 2 ? 0 : 1);
+/* Magnitudes a[0..24) of the p-th arrangement of class o, given its codeword word.
+ * odd: p is the lexicographic rank of (a_0, ..., a_23) over the whole multiset.
+ * even: p_S = p mod P_S and p_C = floor(p / P_S); p_S ranks the magnitudes on the positions of
+ * S (ascending position) among the arrangements of the 2-mod-4 groups, p_C ranks those on the
+ * other positions among the arrangements of the 0-mod-4 groups. */
+static int class_unrank(const ocls *o, uint32_t word, u128 p, int a[ORA_DIM]) {
+    if (o->odd) {
+        int cnt[ORA_DIM], seq[ORA_DIM];
+        for (int g = 0; g < o->nvals; g++) cnt[g] = o->cnts[g];
+        if (lex_unrank(o->nvals, cnt, p, seq)) return -1;
+        for (int i = 0; i < ORA_DIM; i++) a[i] = o->vals[seq[i]];
+        return 0;
+    }
+    int vS[ORA_DIM], cS[ORA_DIM], vC[ORA_DIM], cC[ORA_DIM], nS = 0, nC = 0;
+    for (int g = 0; g < o->nvals; g++) {          /* ascending magnitude within each set */
+        if (o->vals[g] % 4 == 2) { vS[nS] = o->vals[g]; cS[nS++] = o->cnts[g]; }
+        else { vC[nC] = o->vals[g]; cC[nC++] = o->cnts[g]; }
+    }
+    const u128 PS = multinomial(nS, cS);
+    int seqS[ORA_DIM], seqC[ORA_DIM];
+    if (lex_unrank(nS, cS, p % PS, seqS)) return -1;
+    if (lex_unrank(nC, cC, p / PS, seqC)) return -1;
+    int iS = 0, iC = 0;
     for (int i = 0; i < ORA_DIM; i++)
-        pside[i] = o->odd ? 0 : ((S >> i & 1u) ? 0 : 1);
+        a[i] = (word >> i & 1u) ? vS[seqS[iS++]] : vC[seqC[iC++]];
+    return 0;
+}
+
+/* inverse of class_unrank: the arrangement rank p of the magnitudes a */
+static int class_rank(const ocls *o, uint32_t word, const int a[ORA_DIM], u128 *p) {
+    int seq[ORA_DIM];
+    if (o->odd) {
+        int cnt[ORA_DIM];
+        for (int g = 0; g < o->nvals; g++) cnt[g] = o->cnts[g];
+        for (int i = 0; i < ORA_DIM; i++) {
+            seq[i] = -1;
+            for (int g = 0; g < o->nvals; g++) if (o->vals[g] == a[i]) seq[i] = g;
+        }
+        return lex_rank(o->nvals, cnt, ORA_DIM, seq, p);
+    }
+    int vS[ORA_DIM], cS[ORA_DIM], vC[ORA_DIM], cC[ORA_DIM], nS = 0, nC = 0;
+    for (int g = 0; g < o->nvals; g++) {
+        if (o->vals[g] % 4 == 2) { vS[nS] = o->vals[g]; cS[nS++] = o->cnts[g]; }
+        else { vC[nC] = o->vals[g]; cC[nC++] = o->cnts[g]; }
+    }
+    int seqS[ORA_DIM], seqC[ORA_DIM], lS = 0, lC = 0;
+    for (int i = 0; i < ORA_DIM; i++) {
+        const int inS = (int)(word >> i & 1u);
+        const int *v = inS ? vS : vC;
+        const int nv = inS ? nS : nC;
+        int gi = -1;
+        for (int g = 0; g < nv; g++) if (v[g] == a[i]) gi = g;
+        if (inS) seqS[lS++] = gi; else seqC[lC++] = gi;
+    }
+    u128 pS, pC;
+    if (lex_rank(nS, cS, lS, seqS, &pS) || lex_rank(nC, cC, lC, seqC, &pC)) return -1;
+    *p = pS + multinomial(nS, cS) * pC;
+    return 0;
 }
 
 /* decode ([notes-K2]): shell -> class -> r, s, I'' by division and remainder, then the
@@ -637,12 +688,8 @@ static int decode_one(ora_codec *c, u128 I, int32_t x[ORA_DIM], int *shell) {
     if (o.odd) word = c->golay_mask[(int)r];                 /* T: r-th codeword by mask */
     else word = c->golay_weight[c->wbase[o.k] + (int)r];     /* S: r-th word of weight k */
 
-    int cnt[ORA_DIM], gside[ORA_DIM], pside[ORA_DIM], seq[ORA_DIM];
-    for (int g = 0; g < o.nvals; g++) cnt[g] = o.cnts[g];
-    class_sides(&o, word, gside, pside);
-    if (arr_unrank(o.nvals, cnt, gside, ORA_DIM, pside, p, seq)) return -1;
     int a[ORA_DIM];
-    for (int i = 0; i < ORA_DIM; i++) a[i] = o.vals[seq[i]];
+    if (class_unrank(&o, word, p, a)) return -1;
 
     if (o.odd) {
         /* x_i = 1 (mod 4) exactly on T */
@@ -736,15 +783,8 @@ int ora_encode(ora_codec *c, const int32_t x[ORA_DIM], uint64_t *lo, uint64_t *h
             j++;
         }
     }
-    int cnt[ORA_DIM], gside[ORA_DIM], pside[ORA_DIM], seq[ORA_DIM];
-    for (int g = 0; g < o.nvals; g++) cnt[g] = o.cnts[g];
-    class_sides(&o, word, gside, pside);
-    for (int i = 0; i < ORA_DIM; i++) {
-        seq[i] = -1;
-        for (int g = 0; g < o.nvals; g++) if (o.vals[g] == a[i]) seq[i] = g;
-    }
     u128 p;
-    if (arr_rank(o.nvals, cnt, gside, ORA_DIM, pside, seq, &p)) return -1;
+    if (class_rank(&o, word, a, &p)) return -1;
     u128 I = o.offset + r + (u128)o.A * (s + ((u128)1 << o.B) * p);
     split128(I, lo, hi);
     return 0;
