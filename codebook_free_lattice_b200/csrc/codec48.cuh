@@ -5,7 +5,8 @@
 // notes, 方法详解 / 关键设计 2 (shell and class by cumulative offsets; r = I_class mod A,
 // I' = floor(I_class / A), s = I' mod 2^B, I'' = floor(I' / 2^B)).
 //
-//   1. class: a guide table on the top index bits narrows a binary search of the class starts;
+//   1. class: a guide table on the top index bits gives the candidate classes, almost always one
+//      or two, decided by comparing with the class starts;
 //   2. r, s, I'' by one fp64 division by A with an exact integer correction;
 //   3. codeword from the shared-memory Golay tables (odd: T by mask order; even: S among the
 //      codewords of weight k);
@@ -18,49 +19,253 @@
 //      among that set's remaining items (byte-SIMD search of the cumulative counts) and
 //      f <- (f * L - start(group)) / count(group).  Directed rounding keeps each f above its exact
 //      rational with an error far below 1/(remaining arrangements) for P < 2^33, so every slot
-//      is exact.  The loop stays on the FMA, ALU and fp64 pipes;
+//      is exact.  The loop stays on the FMA, ALU and fp64 pipes.  Most even classes skip the
+//      loop: p_S and p_C index precomputed arrangement tables of the two coordinate sets;
 //   5. magnitudes and sign flags by byte permutation of the class's group tables, then signs.
+//
+// The per-class constants are stored one array per field, so that a warp reading one field for
+// 32 different classes spreads over the shared-memory banks.
 #pragma once
 #include "device_common.cuh"
 
 namespace llvq {
 
-struct alignas(16) Rec48 {
-    unsigned long long start;  // first global index of the class
-    double invP;               // 1/P rounded toward +inf
-    double invA;               // 1/A rounded to nearest
-    uint32_t cum;              // bytes: cumulative counts C_<=g, g = 0..3 (saturating at 24)
-    uint32_t vals;             // bytes: magnitudes of groups 0..3
-    uint32_t A;                // 1, 759, 2576 or 4096
-    uint32_t gflag;            // bytes: per-group sign flag, groups 0..3 (odd: |x| = 1 mod 4;
-                               //        even: |x| != 0)
-    uint8_t val4;              // magnitude of group 4
-    uint8_t gflag4;            // sign flag of group 4
-    uint8_t nS;                // places on the codeword side: k (even) or 24 (odd)
-    uint8_t B;                 // free sign bits
-    uint8_t flags;             // bit0 odd coset, bit1 parity target (sum|x|/4 odd)
-    uint8_t m;                 // shell
-    uint16_t wbase;            // even: first by-weight Golay slot of weight k
-    double PC;                 // arrangements off S (even; exact, < 2^24), 1 for odd classes
-    double pad;
-};
-static_assert(sizeof(Rec48) == 64, "Rec48 layout");
-
-constexpr int kGuideBits48 = 11;                  // 2048 buckets over [0, 2^48)
+constexpr int kClasses48 = 384;
+constexpr int kGuideBits48 = 12;                  // 4096 buckets over [0, 2^48)
 constexpr int kGuideShift48 = 48 - kGuideBits48;
 
-// Shared-memory image of the 48-bit decode tables (one copy per CTA, 72 KB).
-struct Smem48 {
+// c_info: A (bits 0..12) | B (13..17) | odd coset (18) | parity target sum|x|/4 odd (19) |
+//         table path (20) | shell m (21..24) | magnitude of group 4 (25..28) | its sign flag (29)
+constexpr uint32_t kInfoOdd = 1u << 18;
+constexpr uint32_t kInfoParity = 1u << 19;
+constexpr uint32_t kInfoTable = 1u << 20;
+__host__ __device__ constexpr uint32_t info_A(uint32_t i) { return i & 0x1FFFu; }
+__host__ __device__ constexpr uint32_t info_B(uint32_t i) { return (i >> 13) & 0x1Fu; }
+__host__ __device__ constexpr int info_m(uint32_t i) { return (int)((i >> 21) & 0xFu); }
+__host__ __device__ constexpr uint32_t info_val4(uint32_t i) { return (i >> 25) & 0xFu; }
+__host__ __device__ constexpr uint32_t info_flag4(uint32_t i) { return (i >> 29) & 1u; }
+// c_info2: first by-weight Golay slot of weight k (bits 0..11) | places on S: k or 24 (12..16) |
+//          table path: arrangements on S, P_S (17..27)
+// c_offs:  table path: first entry of the complement's table (bits 0..18) | of S's table (19..31)
+
+constexpr int kTabS48 = 8192;                     // S-side arrangement entries (7964 used)
+
+// Shared-memory image of the 48-bit decode tables (one copy per CTA, 70 KB).  16-byte aligned
+// size: it is copied in 16-byte units, and tables placed after it are read in 16-byte units.
+struct alignas(16) Smem48 {
     uint32_t golay_mask[4096];
     uint32_t golay_weight[4096];
     double invc[32];                              // 1/c rounded up, c = 1..24
     unsigned long long starts[400];               // class starts, [nclasses] = N_M
-    Rec48 recs[384];
+    double c_invA[kClasses48];                    // 1/A rounded up
+    double c_invP[kClasses48];                    // 1/P rounded up
+    double c_PC[kClasses48];                      // arrangements off S (even; exact), 1 for odd
+    uint32_t c_info[kClasses48];
+    uint32_t c_info2[kClasses48];
+    uint32_t c_offs[kClasses48];
+    uint32_t c_cum[kClasses48];                   // bytes: cumulative counts C_<=g, g = 0..3 (sat. 24)
+    uint32_t c_vals[kClasses48];                  // bytes: magnitudes of groups 0..3
+    uint32_t c_gflag[kClasses48];                 // bytes: per-group sign flag (odd: |x| = 1 mod 4;
+                                                  //        even: |x| != 0)
     uint16_t guide[(1 << kGuideBits48) + 1];
     uint16_t pdep_off[256];
     uint8_t pdep[kPdepEntries];
     float invnorm[16];                            // 1 / (4 sqrt(m))
 };
+
+// Tables of the even-coset table path.  An arrangement entry lists the value codes of one
+// coordinate set in ascending position, two bits each (code = (|x| - 2)/4 on S, |x|/4 off S),
+// in lexicographic order per multiset of codes.  merge[mq << 8 | bits] places the next symbols of
+// the two sets on the four coordinates of one nibble whose S positions are mq: bits holds the
+// popcount(mq) S symbols, then the C symbols; the entry is the four magnitude bytes with the
+// nibble's nonzero mask in bits 28..31.
+struct alignas(16) SmemEven48 {
+    uint32_t tabS[kTabS48];
+    uint32_t merge[4096];
+};
+static_assert(sizeof(Smem48) % 16 == 0 && sizeof(SmemEven48) % 16 == 0, "16-byte table images");
+
+// Steps 1-2 of the decode: the class of one packed word and its digits r, s and p = I''.
+struct Cls48 {
+    unsigned long long p;      // arrangement rank I''
+    uint32_t r, s;             // Golay refinement, sign bits
+    uint32_t info;             // c_info of the class
+    int cls;                   // class index
+    bool ok;                   // index < N_M (otherwise the digits describe index 0)
+};
+
+__device__ __forceinline__ Cls48 classify48(unsigned long long w, const Smem48 &S, unsigned long long npoints) {
+    Cls48 c;
+    unsigned long long idx = w & 0xFFFFFFFFFFFFull;
+    c.ok = idx < npoints;
+    if (!c.ok) idx = 0;
+    // 1. class: the guide bucket of the top index bits holds classes lo..hi; almost always
+    //    hi <= lo + 1, decided by one comparison; wider buckets take a binary search
+    const uint32_t b = (uint32_t)(idx >> kGuideShift48);
+    int lo = S.guide[b];
+    const int hi = S.guide[b + 1];
+    if (hi > lo + 1) {
+        int h = hi;
+        while (lo < h) {
+            const int mid = (lo + h + 1) >> 1;
+            if (S.starts[mid] <= idx) lo = mid; else h = mid - 1;
+        }
+    } else {
+        lo += (hi > lo && S.starts[hi] <= idx) ? 1 : 0;
+    }
+    c.cls = lo;
+    c.info = S.c_info[lo];
+    const uint32_t A = info_A(c.info), B = info_B(c.info);
+    // 2. I_class = r + A (s + 2^B I'').  I_class < 2^48 is exact as the double 2^52 + I_class
+    //    minus 2^52; q = floor(I_class / A) comes from the product with 1/A rounded up (q or
+    //    q + 1) and one correction, its 2^52-biased double giving q's bits directly.
+    const unsigned long long Ic = idx - S.starts[lo];
+    const double Icd = __hiloint2double(0x43300000 | (int)(Ic >> 32), (int)(uint32_t)Ic) - 0x1p52;
+    const double t = __dadd_rz(__dmul_ru(Icd, S.c_invA[lo]), 0x1p52);
+    uint32_t q_lo = (uint32_t)__double2loint(t);
+    uint32_t q_hi = (uint32_t)__double2hiint(t) & 0xFFFFFu;
+    int rem = (int)((uint32_t)Ic - q_lo * A);
+    if (rem < 0) {
+        rem += (int)A;
+        q_hi -= q_lo == 0u ? 1u : 0u;
+        q_lo -= 1u;
+    }
+    c.r = (uint32_t)rem;
+    c.s = q_lo & ((1u << B) - 1u);
+    c.p = ((unsigned long long)q_hi << 32 | q_lo) >> B;
+    return c;
+}
+
+// Step 5 after the arrangement: magnitudes and sign flags from the class's group tables by the
+// recorded group nibbles, then the signs.
+__device__ __forceinline__ void finish48(const Smem48 &S, int cls, uint32_t info, bool odd, uint32_t word,
+                                         uint32_t s, bool ok, const uint32_t sel[6], uint32_t v[6]) {
+    const uint32_t vals = S.c_vals[cls], gflag = S.c_gflag[cls];
+    const uint32_t val4 = info_val4(info), flag4 = info_flag4(info);
+    uint32_t mag[6], F = 0;
+#pragma unroll
+    for (int q2 = 0; q2 < 6; q2++) {
+        mag[q2] = __byte_perm(vals, val4, sel[q2]);
+        F |= bytes_to_nibble(__byte_perm(gflag, flag4, sel[q2])) << (4 * q2);
+    }
+    apply_signs(odd, word, s, F, (info & kInfoParity) ? 1u : 0u, mag, ok, S.pdep_off, S.pdep, v);
+}
+
+// Steps 3-5 for any class: codeword, the arrangement of both coordinate sets, signs.
+__device__ __forceinline__ void arrange48(const Smem48 &S, int cls, uint32_t info, unsigned long long p,
+                                          uint32_t r, uint32_t s, bool ok, uint32_t v[6]) {
+    const uint32_t info2 = S.c_info2[cls];
+    const int nS = (int)((info2 >> 12) & 0x1Fu);
+    // 3. codeword
+    const bool odd = info & kInfoOdd;
+    const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
+    const uint32_t side0 = odd ? 0xFFFFFFu : word;
+    // 4. arrangement.  Byte b of cumB is 0x7F + C_<=b (remaining items of groups 0..b),
+    //    biased one below the guard bit so the byte-wise subtraction of the slot never borrows.
+    double fC = __dmul_ru((double)p, S.c_invP[cls]);            // (p_C + p_S/P_S) / P_C
+    const double g0 = __dmul_ru(fC, S.c_PC[cls]);                 // p_C + p_S/P_S
+    double fS = __dadd_ru(g0, 0x1p52 - __dadd_rz(g0, 0x1p52));   // p_S / P_S
+    uint32_t cumB = S.c_cum[cls] + 0x7F7F7F7Fu;
+    int L0 = nS, L1 = 24 - nS;
+    uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u,
+                       0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
+#pragma unroll
+    for (int i = 0; i < 24; i++) {
+        const bool on0 = side0 & (1u << i);
+        const int L = on0 ? L0 : L1;
+        const int off = on0 ? 0 : L0;
+        const double g = __dmul_ru(on0 ? fS : fC, small_to_double((uint32_t)L));
+        const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52)) + (uint32_t)off;
+        const uint32_t u = cumB - slot * 0x01010101u;            // bit 7 of byte b: C_<=b > slot
+        const uint32_t dm = (u >> 7) & 0x01010101u;              // one per group >= grp
+        const uint32_t ssel = (uint32_t)__dp4a((int)dm, -1, 7);          // grp + 3
+        const uint32_t esel = (uint32_t)__dp4a((int)dm, -1, 0x5554);     // 0x5550 + grp
+        const uint32_t stB = __byte_perm(0x7F7F7F7Fu, cumB, ssel);       // 0x7F7F7F7F + C_<grp
+        const uint32_t enB = __byte_perm(cumB, 0x7F7F7F7Fu + (uint32_t)(24 - i), esel);
+        const uint32_t cnt = min(enB - stB, 31u);                        // in 1..24
+        const uint32_t stl = stB - 0x7F7F7F7Fu - (uint32_t)off;
+        const double fn = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), S.invc[cnt]);
+        if (on0) fS = fn; else fC = fn;
+        cumB -= dm;                                              // groups >= grp lose one item
+        L0 -= on0 ? 1 : 0;
+        L1 -= on0 ? 0 : 1;
+        sel[i >> 2] += ssel << (4 * (i & 3));                    // nibble = grp (bias -0x3333)
+    }
+    finish48(S, cls, info, odd, word, s, ok, sel, v);
+}
+
+// One coordinate of the odd-class loop: at coordinate i the set has 24 - i places left and the
+// slot needs no offset.
+__device__ __forceinline__ void odd_step48(int i, double &f, uint32_t &cumB, uint32_t sel[6], const double *invc) {
+    const double g = __dmul_ru(f, (double)(24 - i));
+    const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52));
+    const uint32_t u = cumB - slot * 0x01010101u;
+    const uint32_t dm = (u >> 7) & 0x01010101u;
+    const uint32_t ssel = (uint32_t)__dp4a((int)dm, -1, 7);
+    const uint32_t esel = (uint32_t)__dp4a((int)dm, -1, 0x5554);
+    const uint32_t stB = __byte_perm(0x7F7F7F7Fu, cumB, ssel);
+    const uint32_t enB = __byte_perm(cumB, 0x7F7F7F7Fu + (uint32_t)(24 - i), esel);
+    const uint32_t cnt = min(enB - stB, 31u);
+    const uint32_t stl = stB - 0x7F7F7F7Fu;
+    f = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), invc[cnt]);
+    cumB -= dm;
+    sel[i >> 2] += ssel << (4 * (i & 3));
+}
+
+// Steps 3-5 for an odd class only: one coordinate set, so the places left at coordinate i are
+// 24 - i and the slot needs no offset.
+__device__ __forceinline__ void arrange_odd48(const Smem48 &S, int cls, uint32_t info, unsigned long long p,
+                                              uint32_t r, uint32_t v[6]) {
+    const uint32_t T = S.golay_mask[r & 4095u];
+    double f = __dmul_ru((double)p, S.c_invP[cls]);
+    uint32_t cumB = S.c_cum[cls] + 0x7F7F7F7Fu;
+    uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u,
+                       0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
+#pragma unroll
+    for (int i = 0; i < 24; i++) odd_step48(i, f, cumB, sel, S.invc);
+    finish48(S, cls, info, true, T, 0u, true, sel, v);
+}
+
+// Steps 3-5 for an even class on the table path: p_C = floor(f_C P_C) and p_S from the scaled
+// fraction as in the loop, both sets' code sequences from the arrangement tables, merged
+// nibble by nibble along the codeword S.
+__device__ __forceinline__ void arrange_even48_table(const Smem48 &S, const SmemEven48 &E,
+                                                     const uint32_t *__restrict__ tabC, int cls, uint32_t info,
+                                                     unsigned long long p, uint32_t r, uint32_t s, uint32_t v[6]) {
+    const uint32_t info2 = S.c_info2[cls], offs = S.c_offs[cls];
+    const uint32_t word = S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
+    const double fC = __dmul_ru((double)p, S.c_invP[cls]);       // (p_C + p_S/P_S) / P_C
+    const double g0 = __dmul_ru(fC, S.c_PC[cls]);                 // p_C + p_S/P_S
+    const double t0 = __dadd_rz(g0, 0x1p52);                      // 2^52 + p_C
+    const uint32_t pC = (uint32_t)__double2loint(t0);
+    const double fS = __dadd_ru(g0, 0x1p52 - t0);                 // p_S / P_S
+    const double h = __dmul_ru(fS, small_to_double(info2 >> 17));
+    const uint32_t pS = (uint32_t)__double2loint(__dadd_rz(h, 0x1p52));
+    uint32_t sS = E.tabS[(offs >> 19) + pS];
+    uint32_t cS = __ldg(tabC + (offs & 0x7FFFFu) + pC);
+    uint32_t mag[6], F = 0, Sw = word;
+#pragma unroll
+    for (int q = 0; q < 6; q++) {
+        const uint32_t mq = Sw & 0xFu;
+        Sw >>= 4;
+        const uint32_t n2 = 2u * (uint32_t)__popc(mq);
+        const uint32_t bits = ((sS & ((1u << n2) - 1u)) | (cS << n2)) & 0xFFu;
+        const uint32_t e = E.merge[(mq << 8) | bits];
+        mag[q] = e & 0x0F0F0F0Fu;
+        F |= (e >> 28) << (4 * q);
+        sS >>= n2;
+        cS >>= 8u - n2;
+    }
+    apply_signs(false, word, s, F, (info & kInfoParity) ? 1u : 0u, mag, true, S.pdep_off, S.pdep, v);
+}
+
+// The complement-table position of an even table-path block (to fetch its entry ahead of use).
+__device__ __forceinline__ const uint32_t *even48_tabC_entry(const Smem48 &S, const uint32_t *tabC, int cls,
+                                                             unsigned long long p) {
+    const double g0 = __dmul_ru(__dmul_ru(small_to_double((uint32_t)p), S.c_invP[cls]), S.c_PC[cls]);
+    const uint32_t pC = (uint32_t)__double2loint(__dadd_rz(g0, 0x1p52));
+    return tabC + (S.c_offs[cls] & 0x7FFFFu) + pC;
+}
 
 struct Dec48 {
     using Word = unsigned long long;
@@ -70,7 +275,7 @@ struct Dec48 {
         unsigned long long npoints;
     };
     static constexpr int kWordBytes = 8;
-    static constexpr int kCtasPerSm = 3;          // 40 registers, 72 KB shared per CTA
+    static constexpr int kCtasPerSm = 3;          // 40 registers, 70 KB shared per CTA
 
     __device__ static Word load(const Word *p) { return __ldg(p); }
     __device__ static int gain_code(const Word &w) { return (int)((w >> 48) & 0xFFu); }
@@ -79,71 +284,10 @@ struct Dec48 {
     // Decode one packed word into 24 signed int8 coordinates (v[q] byte b = coordinate 4q+b).
     // Returns false (and v = 0) for an index >= N_M.  m receives the shell.
     __device__ static bool decode(const Word &w, const Smem &S, const Args &a, uint32_t v[6], int &m) {
-        unsigned long long idx = w & 0xFFFFFFFFFFFFull;
-        const bool ok = idx < a.npoints;
-        if (!ok) idx = 0;
-        // 1. class
-        int lo = S.guide[idx >> kGuideShift48];
-        int hi = S.guide[(idx >> kGuideShift48) + 1];
-        while (lo < hi) {
-            const int mid = (lo + hi + 1) >> 1;
-            if (S.starts[mid] <= idx) lo = mid; else hi = mid - 1;
-        }
-        const Rec48 R = S.recs[lo];
-        m = R.m;
-        // 2. I_class = r + A (s + 2^B I'')
-        const unsigned long long Ic = idx - R.start;
-        unsigned long long q = (unsigned long long)((double)Ic * R.invA);
-        long long rem = (long long)(Ic - q * R.A);
-        if (rem < 0) { q -= 1; rem += R.A; }
-        else if (rem >= (long long)R.A) { q += 1; rem -= R.A; }
-        const uint32_t r = (uint32_t)rem;
-        const uint32_t s = (uint32_t)(q & ((1ull << R.B) - 1ull));
-        const unsigned long long p = q >> R.B;
-        // 3. codeword
-        const bool odd = R.flags & 1u;
-        const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min(R.wbase + r, 4095u)];
-        const uint32_t side0 = odd ? 0xFFFFFFu : word;
-        // 4. arrangement.  Byte b of cumB is 0x7F + C_<=b (remaining items of groups 0..b),
-        //    biased one below the guard bit so the byte-wise subtraction of the slot never borrows.
-        double fC = __dmul_ru((double)p, R.invP);                   // (p_C + p_S/P_S) / P_C
-        const double g0 = __dmul_ru(fC, R.PC);                       // p_C + p_S/P_S
-        double fS = __dadd_ru(g0, 0x1p52 - __dadd_rz(g0, 0x1p52));   // p_S / P_S
-        uint32_t cumB = R.cum + 0x7F7F7F7Fu;
-        int L0 = R.nS, L1 = 24 - R.nS;
-        uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u,
-                           0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
-#pragma unroll
-        for (int i = 0; i < 24; i++) {
-            const bool on0 = side0 & (1u << i);
-            const int L = on0 ? L0 : L1;
-            const int off = on0 ? 0 : L0;
-            const double g = __dmul_ru(on0 ? fS : fC, small_to_double((uint32_t)L));
-            const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52)) + (uint32_t)off;
-            const uint32_t u = cumB - slot * 0x01010101u;            // bit 7 of byte b: C_<=b > slot
-            const uint32_t dm = (u >> 7) & 0x01010101u;              // one per group >= grp
-            const uint32_t ssel = (uint32_t)__dp4a((int)dm, -1, 7);          // grp + 3
-            const uint32_t esel = (uint32_t)__dp4a((int)dm, -1, 0x5554);     // 0x5550 + grp
-            const uint32_t stB = __byte_perm(0x7F7F7F7Fu, cumB, ssel);       // 0x7F7F7F7F + C_<grp
-            const uint32_t enB = __byte_perm(cumB, 0x7F7F7F7Fu + (uint32_t)(24 - i), esel);
-            const uint32_t cnt = min(enB - stB, 31u);                        // in 1..24
-            const uint32_t stl = stB - 0x7F7F7F7Fu - (uint32_t)off;
-            const double fn = __dmul_ru(__dadd_ru(g, -small_to_double(stl)), S.invc[cnt]);
-            if (on0) fS = fn; else fC = fn;
-            cumB -= dm;                                              // groups >= grp lose one item
-            L0 -= on0 ? 1 : 0;
-            L1 -= on0 ? 0 : 1;
-            sel[i >> 2] += ssel << (4 * (i & 3));                    // nibble = grp (bias -0x3333)
-        }
-        // 5. magnitudes, sign flags, signs
-        uint32_t mag[6], F = 0;
-#pragma unroll
-        for (int q2 = 0; q2 < 6; q2++) {
-            mag[q2] = __byte_perm(R.vals, (uint32_t)R.val4, sel[q2]);
-            F |= bytes_to_nibble(__byte_perm(R.gflag, (uint32_t)R.gflag4, sel[q2])) << (4 * q2);
-        }
-        apply_signs(odd, word, s, F, (uint32_t)(R.flags >> 1), mag, ok, S.pdep_off, S.pdep, v);
-        return ok;
+        const Cls48 c = classify48(w, S, a.npoints);
+        m = info_m(c.info);
+        arrange48(S, c.cls, c.info, c.p, c.r, c.s, c.ok, v);
+        return c.ok;
     }
 };
 

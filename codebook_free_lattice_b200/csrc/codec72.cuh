@@ -48,6 +48,8 @@ struct alignas(16) Smem72 {
     float invnorm[64];                            // 1 / (4 sqrt(m)), m <= 53
 };
 
+static_assert(sizeof(Smem72) % 16 == 0, "16-byte table image");
+
 struct Dec72 {
     using Word = ulonglong2;                      // x = bits 0..63, y = bits 64..127
     using Smem = Smem72;

@@ -5,13 +5,16 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
+#include <type_traits>
 #include <utility>
 #include <vector>
 
 #include "../../include/llvq.h"
 #include "kernels.cuh"
+#include "kernels_bin48.cuh"
 #include "kernels_tc.cuh"
 #include "tables.h"
 
@@ -27,6 +30,8 @@ struct llvq_codec {
     void *d_image = nullptr;       // Smem48 / Smem72 image (copied to shared memory per CTA)
     Rec72 *d_recs72 = nullptr;     // 72-bit class records (global memory)
     uint32_t *d_guide72 = nullptr; // 72-bit guide table
+    void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
+    uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
     unsigned *d_flags = nullptr;   // sticky device flags
 };
 
@@ -88,27 +93,27 @@ llvq_status build_image48(const HostTables &T, Smem48 &S, std::string &err) {
         const HostClass &c = T.classes[i];
         if (c.vals.size() > 5) { err = "more than 5 magnitude groups at 48 bits"; return LLVQ_ERR_UNSUPPORTED; }
         if (c.P >= ((u128)1 << 33) || c.P_C >= ((u128)1 << 24)) { err = "48-bit arrangement count out of range"; return LLVQ_ERR_UNSUPPORTED; }
-        Rec48 &R = S.recs[i];
-        R.start = (unsigned long long)c.start;
-        R.invP = round_up_ratio(1.0, (double)c.P);    // P < 2^33: exact as a double
-        R.invA = 1.0 / (double)c.A;
-        R.PC = (double)c.P_C;                         // < 2^24 for every 48-bit class: exact
-        R.A = c.A;
+        S.c_invP[i] = round_up_ratio(1.0, (double)c.P);    // P < 2^33: exact as a double
+        S.c_invA[i] = round_up_ratio(1.0, (double)c.A);
+        S.c_PC[i] = (double)c.P_C;                           // < 2^24 for every 48-bit class: exact
         uint32_t vals = 0, gflag = 0;
         for (int g = 0; g < 4 && g < (int)c.vals.size(); g++) {
             vals |= (uint32_t)c.vals[g] << (8 * g);
             gflag |= (uint32_t)sign_flag(c, g) << (8 * g);
         }
-        R.cum = (uint32_t)cum_bytes(c, 4);
-        R.vals = vals;
-        R.gflag = gflag;
-        R.val4 = c.vals.size() > 4 ? (uint8_t)c.vals[4] : 0;
-        R.gflag4 = c.vals.size() > 4 ? sign_flag(c, 4) : 0;
-        R.nS = (uint8_t)(c.odd ? 24 : c.k);
-        R.B = (uint8_t)c.B;
-        R.flags = (uint8_t)((c.odd ? 1 : 0) | (((c.sum_abs / 4) & 1) << 1));
-        R.m = (uint8_t)c.m;
-        R.wbase = (uint16_t)(c.odd ? 0 : T.weight_base[c.k]);
+        S.c_cum[i] = (uint32_t)cum_bytes(c, 4);
+        S.c_vals[i] = vals;
+        S.c_gflag[i] = gflag;
+        const uint32_t val4 = c.vals.size() > 4 ? (uint32_t)c.vals[4] : 0u;
+        const uint32_t flag4 = c.vals.size() > 4 ? sign_flag(c, 4) : 0u;
+        const uint32_t wbase = c.odd ? 0u : (uint32_t)T.weight_base[c.k];
+        if (c.A > 0x1FFFu || c.B > 31 || c.m > 15 || val4 > 15 || wbase > 0xFFFu) {
+            err = "48-bit class constant out of its field";
+            return LLVQ_ERR_UNSUPPORTED;
+        }
+        S.c_info[i] = c.A | (uint32_t)c.B << 13 | (c.odd ? kInfoOdd : 0u) |
+                      (((c.sum_abs / 4) & 1) ? kInfoParity : 0u) | (uint32_t)c.m << 21 | val4 << 25 | flag4 << 29;
+        S.c_info2[i] = wbase | (uint32_t)(c.odd ? 24 : c.k) << 12;
         S.starts[i] = (unsigned long long)c.start;
     }
     S.starts[nc] = (unsigned long long)T.n_points;
@@ -122,6 +127,68 @@ llvq_status build_image48(const HostTables &T, Smem48 &S, std::string &err) {
     }
     fill_pdep(S.pdep_off, S.pdep);
     for (int m = 1; m < 16; m++) S.invnorm[m] = (float)(1.0 / (4.0 * std::sqrt((double)m)));
+    return LLVQ_OK;
+}
+
+// Arrangement tables of the even-coset table path (see SmemEven48).  Classes whose codeword has
+// weight 8, 12 or 16 and whose complement has at most kTabCMax arrangements are marked in their
+// class info; every code sequence table is generated once per multiset of codes, in lexicographic
+// order, by stepping through the distinct permutations.
+constexpr uint64_t kTabCMax = 1u << 17;
+
+uint32_t side_table(const std::vector<int> &codes_sorted, std::map<std::vector<int>, uint32_t> &index,
+                    std::vector<uint32_t> &tab) {
+    auto it = index.find(codes_sorted);
+    if (it != index.end()) return it->second;
+    const uint32_t off = (uint32_t)tab.size();
+    std::vector<int> seq = codes_sorted;
+    do {
+        uint32_t e = 0;
+        for (size_t i = 0; i < seq.size(); i++) e |= (uint32_t)seq[i] << (2 * i);
+        tab.push_back(e);
+    } while (std::next_permutation(seq.begin(), seq.end()));
+    index[codes_sorted] = off;
+    return off;
+}
+
+llvq_status build_even48(const HostTables &T, Smem48 &S, SmemEven48 &E, std::vector<uint32_t> &tabC,
+                         std::string &err) {
+    std::memset(&E, 0, sizeof E);
+    std::map<std::vector<int>, uint32_t> idxS, idxC;
+    std::vector<uint32_t> tabS;
+    tabC.clear();
+    for (size_t i = 0; i < T.classes.size(); i++) {
+        const HostClass &c = T.classes[i];
+        if (c.odd || (c.k != 8 && c.k != 12 && c.k != 16) || c.P_C > kTabCMax || c.P_S > 0x7FF) continue;
+        std::vector<int> cs, cc;                   // value codes, ascending (groups are ascending)
+        bool fits = true;
+        for (size_t g = 0; g < c.vals.size(); g++) {
+            const int v = c.vals[g];
+            const int code = v % 4 == 2 ? (v - 2) / 4 : v / 4;
+            if (code > 3) fits = false;
+            for (int t = 0; t < c.cnts[g]; t++) (v % 4 == 2 ? cs : cc).push_back(code);
+        }
+        if (!fits) continue;
+        const uint32_t offS = side_table(cs, idxS, tabS), offC = side_table(cc, idxC, tabC);
+        if (offC > 0x7FFFFu || offS > 0x1FFFu || c.P_S > 0x7FFu) { err = "arrangement table offset out of its field"; return LLVQ_ERR_UNSUPPORTED; }
+        S.c_offs[i] = offC | offS << 19;
+        S.c_info2[i] |= (uint32_t)c.P_S << 17;
+        S.c_info[i] |= kInfoTable;
+        if (tabS.size() > (size_t)kTabS48) { err = "S arrangement table overflow"; return LLVQ_ERR_UNSUPPORTED; }
+    }
+    std::copy(tabS.begin(), tabS.end(), E.tabS);
+    for (uint32_t mq = 0; mq < 16; mq++)
+        for (uint32_t bits = 0; bits < 256; bits++) {
+            const int n2 = 2 * __builtin_popcount(mq);
+            uint32_t sb = bits & ((1u << n2) - 1u), cb = bits >> n2, e = 0;
+            for (int pos = 0; pos < 4; pos++) {
+                uint32_t mag, nz;
+                if (mq >> pos & 1u) { mag = 2 + 4 * (sb & 3u); sb >>= 2; nz = 1; }
+                else { mag = 4 * (cb & 3u); cb >>= 2; nz = mag != 0; }
+                e |= mag << (8 * pos) | nz << (28 + pos);
+            }
+            E.merge[mq << 8 | bits] = e;
+        }
     return LLVQ_OK;
 }
 
@@ -224,6 +291,13 @@ void set_gemm_attrs(std::integer_sequence<int, Bs...>) {
     (cudaFuncSetAttribute(k_gemm<D, Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024), ...);
 }
 
+constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per block on sm_100
+
+template <int... Bs>
+void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
+    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+}
+
 // Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
 // CTAs; the output is zeroed here because the splits add into it.
 template <class D>
@@ -243,10 +317,42 @@ cudaError_t launch_gemm_tc(const llvq_codec *c, typename D::Args a, const llvq_w
     return cudaGetLastError();
 }
 
+// 48-bit CUDA-core path with coset sorting: one 1024-thread CTA per SM owning a row range; the
+// range shrinks (more CTAs than SMs) only when its accumulators would not fit in shared memory.
+template <int B>
+cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, float *Y,
+                              cudaStream_t st) {
+    const int nb = w->blocks_per_row;
+    if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
+    int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
+    while (rpc > 1 && bin48_smem_bytes(B, rpc) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (bin48_smem_bytes(B, rpc) > kBinSmemLimit) return cudaErrorInvalidValue;
+    // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
+    if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
+    const int grid = (w->rows + rpc - 1) / rpc;
+    const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
+    k_gemm_bin48<B><<<grid, kBinThreads, bin48_smem_bytes(B, rpc), st>>>(
+        a, (const SmemEven48 *)c->d_even48, c->d_tabC48, (const unsigned long long *)w->words, w->row_pitch_words, w->rows, nb, recip, w->gain_mode,
+        (const __half *)w->gains, (const __half *)X, Y, rpc, c->d_flags);
+    return cudaGetLastError();
+}
+
 template <class D>
 cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
                           int batch, float *Y, cudaStream_t s) {
     if (batch >= kTensorCoreMinBatch) return launch_gemm_tc<D>(c, a, w, X, batch, Y, s);
+    if constexpr (std::is_same<D, Dec48>::value) {
+        switch (batch) {
+            case 1: return launch_gemm_bin48<1>(c, a, w, X, Y, s);
+            case 2: return launch_gemm_bin48<2>(c, a, w, X, Y, s);
+            case 3: return launch_gemm_bin48<3>(c, a, w, X, Y, s);
+            case 4: return launch_gemm_bin48<4>(c, a, w, X, Y, s);
+            case 5: return launch_gemm_bin48<5>(c, a, w, X, Y, s);
+            case 6: return launch_gemm_bin48<6>(c, a, w, X, Y, s);
+            case 7: return launch_gemm_bin48<7>(c, a, w, X, Y, s);
+            default: break;
+        }
+    }
     switch (batch) {
         case 1: return launch_gemm<D, 1>(c, a, w, X, Y, s);
         case 2: return launch_gemm<D, 2>(c, a, w, X, Y, s);
@@ -375,11 +481,15 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     if (!build_host_tables(index_bits, T, err)) { g_last_error = err; return LLVQ_ERR_UNSUPPORTED; }
     std::vector<unsigned char> image;
     std::vector<Rec72> recs;
-    std::vector<uint32_t> guide;
+    std::vector<uint32_t> guide, tabC;
+    std::vector<unsigned char> even(sizeof(SmemEven48));
     llvq_status st;
     if (index_bits == 48) {
         image.resize(sizeof(Smem48));
         st = build_image48(T, *reinterpret_cast<Smem48 *>(image.data()), err);
+        if (st == LLVQ_OK)
+            st = build_even48(T, *reinterpret_cast<Smem48 *>(image.data()), *reinterpret_cast<SmemEven48 *>(even.data()),
+                              tabC, err);
     } else {
         image.resize(sizeof(Smem72));
         st = build_image72(T, *reinterpret_cast<Smem72 *>(image.data()), recs, guide, err);
@@ -396,6 +506,12 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
                cudaMemcpy(c->d_image, image.data(), image.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
                cudaMalloc(&c->d_flags, sizeof(unsigned)) == cudaSuccess &&
                cudaMemset(c->d_flags, 0, sizeof(unsigned)) == cudaSuccess;
+    if (okc && index_bits == 48) {
+        okc = cudaMalloc(&c->d_even48, even.size()) == cudaSuccess &&
+              cudaMemcpy(c->d_even48, even.data(), even.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_tabC48, std::max<size_t>(tabC.size(), 1) * sizeof(uint32_t)) == cudaSuccess &&
+              cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess;
+    }
     if (okc && index_bits == 72) {
         okc = cudaMalloc(&c->d_recs72, recs.size() * sizeof(Rec72)) == cudaSuccess &&
               cudaMemcpy(c->d_recs72, recs.data(), recs.size() * sizeof(Rec72), cudaMemcpyHostToDevice) == cudaSuccess &&
@@ -412,6 +528,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
         cudaFuncSetAttribute(k_gemm_tc<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec48>));
+        set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
         set_gemm_attrs<Dec48>(std::make_integer_sequence<int, 16>{});
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, 16>{});
@@ -426,6 +543,8 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_recs72) cudaFree(c->d_recs72);
     if (c->d_guide72) cudaFree(c->d_guide72);
     if (c->d_flags) cudaFree(c->d_flags);
+    if (c->d_even48) cudaFree(c->d_even48);
+    if (c->d_tabC48) cudaFree(c->d_tabC48);
     delete c;
 }
 

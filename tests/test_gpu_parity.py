@@ -186,7 +186,9 @@ def test_gemm_batch_equals_gemv_columns(gcodec, ocodec):
         sub.x = layer.x[b:b + 1].copy()
         sub.batch = 1
         yb = run_gemm(gcodec, sub)
-        assert max_rel_err(yb[0], Y[b]) < 1e-5
+        # same decoded weights and products; only the fp32 summation order differs (blocks reach
+        # the shared accumulators in an order fixed by atomics), hence a reassociation tolerance
+        assert max_rel_err(yb[0], Y[b]) < 1e-4
 
 
 @pytest.mark.parametrize("bits,rows,K", [(48, 300, 24 * 45 + 5), (72, 130, 24 * 9)])
