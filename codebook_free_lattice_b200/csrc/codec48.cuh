@@ -67,6 +67,8 @@ struct alignas(16) Smem48 {
     uint32_t c_vals[kClasses48];                  // bytes: magnitudes of groups 0..3
     uint32_t c_gflag[kClasses48];                 // bytes: per-group sign flag (odd: |x| = 1 mod 4;
                                                   //        even: |x| != 0)
+    unsigned long long c_vt[kClasses48];          // odd: signed int8 value of groups 0..4 on T
+    unsigned long long c_vn[kClasses48];          // odd: signed int8 value of groups 0..4 off T
     uint16_t guide[(1 << kGuideBits48) + 1];
     uint16_t pdep_off[256];
     uint8_t pdep[kPdepEntries];
@@ -213,7 +215,9 @@ __device__ __forceinline__ void odd_step48(int i, double &f, uint32_t &cumB, uin
 }
 
 // Steps 3-5 for an odd class only: one coordinate set, so the places left at coordinate i are
-// 24 - i and the slot needs no offset.
+// 24 - i and the slot needs no offset.  x_i = a_i exactly when (i in T) equals (a_i = 1 mod 4),
+// so each group has one signed value on T and one off T: a byte permutation of each table by the
+// group nibbles, then a byte select by T.
 __device__ __forceinline__ void arrange_odd48(const Smem48 &S, int cls, uint32_t info, unsigned long long p,
                                               uint32_t r, uint32_t v[6]) {
     const uint32_t T = S.golay_mask[r & 4095u];
@@ -223,26 +227,38 @@ __device__ __forceinline__ void arrange_odd48(const Smem48 &S, int cls, uint32_t
                        0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
 #pragma unroll
     for (int i = 0; i < 24; i++) odd_step48(i, f, cumB, sel, S.invc);
-    finish48(S, cls, info, true, T, 0u, true, sel, v);
+    const unsigned long long vt = S.c_vt[cls], vn = S.c_vn[cls];
+#pragma unroll
+    for (int q = 0; q < 6; q++) {
+        const uint32_t pt = __byte_perm((uint32_t)vt, (uint32_t)(vt >> 32), sel[q]);
+        const uint32_t pn = __byte_perm((uint32_t)vn, (uint32_t)(vn >> 32), sel[q]);
+        const uint32_t tb = nibble_to_bytes((T >> (4 * q)) & 0xFu) * 0xFFu;     // 0xFF on T
+        v[q] = (pt & tb) | (pn & ~tb);
+    }
 }
 
-// Steps 3-5 for an even class on the table path: p_C = floor(f_C P_C) and p_S from the scaled
-// fraction as in the loop, both sets' code sequences from the arrangement tables, merged
-// nibble by nibble along the codeword S.
-__device__ __forceinline__ void arrange_even48_table(const Smem48 &S, const SmemEven48 &E,
-                                                     const uint32_t *__restrict__ tabC, int cls, uint32_t info,
-                                                     unsigned long long p, uint32_t r, uint32_t s, uint32_t v[6]) {
-    const uint32_t info2 = S.c_info2[cls], offs = S.c_offs[cls];
+// Step 4 for an even class on the table path: p_C = floor(f_C P_C) and p_S from the scaled
+// fraction as in the loop; they index the arrangement tables of the complement and of S.
+struct Even48Idx {
+    uint32_t pC, pS;
+};
+__device__ __forceinline__ Even48Idx even48_indices(const Smem48 &S, int cls, unsigned long long p) {
+    Even48Idx x;
+    const double fC = __dmul_ru(small_to_double((uint32_t)p), S.c_invP[cls]);   // (p_C + p_S/P_S) / P_C
+    const double g0 = __dmul_ru(fC, S.c_PC[cls]);                               // p_C + p_S/P_S
+    const double t0 = __dadd_rz(g0, 0x1p52);                                    // 2^52 + p_C
+    x.pC = (uint32_t)__double2loint(t0);
+    const double fS = __dadd_ru(g0, 0x1p52 - t0);                               // p_S / P_S
+    const double h = __dmul_ru(fS, small_to_double(S.c_info2[cls] >> 17));
+    x.pS = (uint32_t)__double2loint(__dadd_rz(h, 0x1p52));
+    return x;
+}
+
+// Steps 3 and 5 for an even class on the table path, given the two sets' code sequences: the
+// codeword S, the sequences merged nibble by nibble along S, then the signs.
+__device__ __forceinline__ void even48_merge(const Smem48 &S, const SmemEven48 &E, uint32_t info, uint32_t info2,
+                                             uint32_t r, uint32_t s, uint32_t sS, uint32_t cS, uint32_t v[6]) {
     const uint32_t word = S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
-    const double fC = __dmul_ru((double)p, S.c_invP[cls]);       // (p_C + p_S/P_S) / P_C
-    const double g0 = __dmul_ru(fC, S.c_PC[cls]);                 // p_C + p_S/P_S
-    const double t0 = __dadd_rz(g0, 0x1p52);                      // 2^52 + p_C
-    const uint32_t pC = (uint32_t)__double2loint(t0);
-    const double fS = __dadd_ru(g0, 0x1p52 - t0);                 // p_S / P_S
-    const double h = __dmul_ru(fS, small_to_double(info2 >> 17));
-    const uint32_t pS = (uint32_t)__double2loint(__dadd_rz(h, 0x1p52));
-    uint32_t sS = E.tabS[(offs >> 19) + pS];
-    uint32_t cS = __ldg(tabC + (offs & 0x7FFFFu) + pC);
     uint32_t mag[6], F = 0, Sw = word;
 #pragma unroll
     for (int q = 0; q < 6; q++) {
@@ -259,12 +275,14 @@ __device__ __forceinline__ void arrange_even48_table(const Smem48 &S, const Smem
     apply_signs(false, word, s, F, (info & kInfoParity) ? 1u : 0u, mag, true, S.pdep_off, S.pdep, v);
 }
 
-// The complement-table position of an even table-path block (to fetch its entry ahead of use).
-__device__ __forceinline__ const uint32_t *even48_tabC_entry(const Smem48 &S, const uint32_t *tabC, int cls,
-                                                             unsigned long long p) {
-    const double g0 = __dmul_ru(__dmul_ru(small_to_double((uint32_t)p), S.c_invP[cls]), S.c_PC[cls]);
-    const uint32_t pC = (uint32_t)__double2loint(__dadd_rz(g0, 0x1p52));
-    return tabC + (S.c_offs[cls] & 0x7FFFFu) + pC;
+// Steps 3-5 for an even class on the table path.
+__device__ __forceinline__ void arrange_even48_table(const Smem48 &S, const SmemEven48 &E,
+                                                     const uint32_t *__restrict__ tabC, int cls, uint32_t info,
+                                                     unsigned long long p, uint32_t r, uint32_t s, uint32_t v[6]) {
+    const Even48Idx x = even48_indices(S, cls, p);
+    const uint32_t offs = S.c_offs[cls];
+    const uint32_t cS = __ldg(tabC + (offs & 0x7FFFFu) + x.pC);
+    even48_merge(S, E, info, S.c_info2[cls], r, s, E.tabS[(offs >> 19) + x.pS], cS, v);
 }
 
 struct Dec48 {

@@ -16,6 +16,74 @@ __device__ __forceinline__ void load_smem_image(void *dst, const void *src, size
     for (size_t i = threadIdx.x; i < n; i += blockDim.x) d[i] = __ldg(s + i);
 }
 
+__device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ bool mbar_try_wait_parity(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Table images into shared memory with the bulk-copy engine: thread 0 initialises the mbarrier
+// `bar`, announces the bytes of all regions and starts one bulk copy per region (sizes multiples
+// of 16 bytes, both addresses 16-byte aligned); every thread then waits for the bytes to land,
+// for at most kBulkWaitTries polls.  Returns false in every thread if any wait gave up (the
+// caller then skips its work and raises a flag).  Ends with a CTA barrier.
+constexpr int kBulkWaitTries = 1 << 22;
+template <int N>
+__device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void *const (&src)[N],
+                                               const uint32_t (&bytes)[N], unsigned long long *bar) {
+    const uint32_t b = smem_u32(bar);
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        uint32_t total = 0;
+#pragma unroll
+        for (int i = 0; i < N; i++) total += bytes[i];
+        asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(b), "r"(total) : "memory");
+#pragma unroll
+        for (int i = 0; i < N; i++)
+            asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                         ::"r"(smem_u32(dst[i])), "l"(src[i]), "r"(bytes[i]), "r"(b) : "memory");
+    }
+    __syncthreads();                               // barrier initialised before anyone polls it
+    bool done = false;
+    for (int it = 0; it < kBulkWaitTries && !done; it++) done = mbar_try_wait_parity(b, 0);
+    return __syncthreads_and(done) != 0;
+}
+
+// int8 x4 -> two half2 (exact): (b ^ 0x80) + 1024 is the fp16 with bits 0x64XX; minus 1152 = b
+__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t l = __byte_perm(u, 0x64646464u, 0x4140);     // coordinates 0, 1
+    const uint32_t h = __byte_perm(u, 0x64646464u, 0x4342);     // coordinates 2, 3
+    const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480),
+                                        __ushort_as_half((unsigned short)0x6480));
+    const __half2 a = __hsub2(*reinterpret_cast<const __half2 *>(&l), bias);
+    const __half2 b = __hsub2(*reinterpret_cast<const __half2 *>(&h), bias);
+    lo = *reinterpret_cast<const uint32_t *>(&a);
+    hi = *reinterpret_cast<const uint32_t *>(&b);
+}
+
+// acc + w.lo * x.lo + w.hi * x.hi for fp16 pairs w, x with fp32 accumulation: each product of two
+// fp16 values is exact in fp32 and is added with one rounding (mixed-precision FMA, sm_100).
+__device__ __forceinline__ float fma2_f16_f32(uint32_t w, uint32_t x, float acc) {
+    asm("{\n\t.reg .f16 w0, w1, x0, x1;\n\t"
+        "mov.b32 {w0, w1}, %1;\n\t"
+        "mov.b32 {x0, x1}, %2;\n\t"
+        "fma.rn.f32.f16 %0, w0, x0, %0;\n\t"
+        "fma.rn.f32.f16 %0, w1, x1, %0;\n\t}"
+        : "+f"(acc)
+        : "r"(w), "r"(x));
+    return acc;
+}
+
 // bit k of a nibble -> byte k (0x01)
 __device__ __forceinline__ uint32_t nibble_to_bytes(uint32_t nib) {
     return (nib * 0x00204081u) & 0x01010101u;

@@ -10,6 +10,7 @@
 namespace llvq {
 
 constexpr unsigned kFlagIndexRange = 0x1u;   // an index >= N_M was met (LLVQ_FLAG_INDEX_RANGE)
+constexpr unsigned kFlagWaitTimeout = 0x2u;  // a bounded wait gave up (LLVQ_FLAG_WAIT_TIMEOUT)
 
 // Decode n packed words into int8 [n][24].
 template <class D>

@@ -19,13 +19,15 @@ constexpr int kBinThreads = 1024;                 // one CTA per SM, 64 register
 constexpr int kBinPer = 4;                        // blocks per thread and chunk
 constexpr int kBinChunk = kBinThreads * kBinPer;  // 4096 blocks = 64 KB of records
 
-// One classified block: x = p bits 0..31; y = p bit 32 | class << 1 | r << 10 | gain code << 22;
-// z = s; w = row within the CTA | block column j << 16.
+// One classified block.  y = class | r << 9 | (see below) << 21; z = s | gain code << 24;
+// w = row within the CTA | block column j << 16.  Odd classes and even classes off the table
+// path: x = p bits 0..31, y bit 21 = p bit 32.  Even classes on the table path: x = the
+// complement's code sequence (fetched while classifying), y bits 21..31 = p_S.
 using BinRec = uint4;
 
 __host__ __device__ constexpr size_t bin48_smem_bytes(int batch, int rows_per_cta) {
     return sizeof(Smem48) + sizeof(SmemEven48) + sizeof(BinRec) * kBinChunk +
-           sizeof(float) * (size_t)batch * rows_per_cta * 32 + 8 * sizeof(int);
+           sizeof(float) * (size_t)batch * rows_per_cta * 32 + 8 * sizeof(int) + 8;
 }
 
 // y contribution of one decoded block: scale * <v, x_b> for every batch row b, added to the
@@ -34,65 +36,48 @@ template <int BATCH>
 __device__ __forceinline__ void accumulate_block(const uint32_t v[6], float scale, const __half *__restrict__ X,
                                                  long long K, int j, float *acc, int rl, int rows_per_cta,
                                                  int lane) {
-    float wv[24];
+    uint32_t wh[12];                                           // exact fp16 coordinates, in pairs
 #pragma unroll
-    for (int q = 0; q < 6; q++)
-#pragma unroll
-        for (int e = 0; e < 4; e++) wv[4 * q + e] = (float)(int8_t)(v[q] >> (8 * e));
+    for (int q = 0; q < 6; q++) i8x4_to_h2x2(v[q], wh[2 * q], wh[2 * q + 1]);
 #pragma unroll
     for (int bb = 0; bb < BATCH; bb++) {
         const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
-        float dot = 0.f;
+        float d0 = 0.f, d1 = 0.f;                              // two chains for latency
 #pragma unroll
         for (int c = 0; c < 3; c++) {
             const uint4 raw = __ldg(xp + c);
-            const uint32_t h[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const float2 xf = __half22float2(*reinterpret_cast<const __half2 *>(&h[e]));
-                dot = fmaf(wv[8 * c + 2 * e], xf.x, dot);
-                dot = fmaf(wv[8 * c + 2 * e + 1], xf.y, dot);
-            }
+            d0 = fma2_f16_f32(wh[4 * c + 0], raw.x, d0);
+            d1 = fma2_f16_f32(wh[4 * c + 1], raw.y, d1);
+            d0 = fma2_f16_f32(wh[4 * c + 2], raw.z, d0);
+            d1 = fma2_f16_f32(wh[4 * c + 3], raw.w, d1);
         }
-        atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * dot);
+        atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * (d0 + d1));
     }
-}
-
-struct BinFields {
-    unsigned long long p;
-    uint32_t r, s;
-    int cls, code, rl, j;
-};
-
-__device__ __forceinline__ BinFields bin_unpack(const BinRec e) {
-    BinFields f;
-    f.p = (unsigned long long)(e.y & 1u) << 32 | e.x;
-    f.cls = (int)((e.y >> 1) & 0x1FFu);
-    f.r = (e.y >> 10) & 0xFFFu;
-    f.code = (int)(e.y >> 22);
-    f.s = e.z;
-    f.rl = (int)(e.w & 0xFFFFu);
-    f.j = (int)(e.w >> 16);
-    return f;
 }
 
 // Phase 2 for one record of the coset ODD.
 template <bool ODD, int BATCH>
-__device__ __forceinline__ void bin48_process(const BinRec e, const Smem48 &S, const SmemEven48 &E,
-                                              const uint32_t *__restrict__ tabC, int gain_mode,
+__device__ __forceinline__ void bin48_process(const BinRec e, const Smem48 &S, const SmemEven48 &E, int gain_mode,
                                               const __half *__restrict__ gains, const __half *__restrict__ X,
                                               long long K, int row0, int nb, float *acc, int rows_per_cta,
                                               int lane) {
-    const BinFields f = bin_unpack(e);
-    const uint32_t info = S.c_info[f.cls];
+    const int cls = (int)(e.y & 0x1FFu);
+    const uint32_t r = (e.y >> 9) & 0xFFFu;
+    const uint32_t s = e.z & 0xFFFFFFu;
+    const int code = (int)(e.z >> 24);
+    const int rl = (int)(e.w & 0xFFFFu);
+    const int j = (int)(e.w >> 16);
+    const uint32_t info = S.c_info[cls];
+    const unsigned long long p = (unsigned long long)((e.y >> 21) & 1u) << 32 | e.x;
     uint32_t v[6];
-    if (ODD) arrange_odd48(S, f.cls, info, f.p, f.r, v);
-    else if (info & kInfoTable) arrange_even48_table(S, E, tabC, f.cls, info, f.p, f.r, f.s, v);
-    else arrange48(S, f.cls, info, f.p, f.r, f.s, true, v);
-    const long long row = (long long)row0 + f.rl;
-    const float scale = gain_mode == 0 ? __half2float(__ldg(gains + row * nb + f.j))
-                                       : __half2float(__ldg(gains + row * 256 + f.code)) * S.invnorm[info_m(info)];
-    accumulate_block<BATCH>(v, scale, X, K, f.j, acc, f.rl, rows_per_cta, lane);
+    if (ODD) arrange_odd48(S, cls, info, p, r, v);
+    else if (info & kInfoTable)
+        even48_merge(S, E, info, S.c_info2[cls], r, s, E.tabS[(S.c_offs[cls] >> 19) + (e.y >> 21)], e.x, v);
+    else arrange48(S, cls, info, p, r, s, true, v);
+    const long long row = (long long)row0 + rl;
+    const float scale = gain_mode == 0 ? __half2float(__ldg(gains + row * nb + j))
+                                       : __half2float(__ldg(gains + row * 256 + code)) * S.invnorm[info_m(info)];
+    accumulate_block<BATCH>(v, scale, X, K, j, acc, rl, rows_per_cta, lane);
 }
 
 template <int BATCH>
@@ -106,10 +91,9 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
     SmemEven48 &E = *reinterpret_cast<SmemEven48 *>(smem_raw + sizeof(Smem48));
     BinRec *list = reinterpret_cast<BinRec *>(smem_raw + sizeof(Smem48) + sizeof(SmemEven48));
     float *acc = reinterpret_cast<float *>(list + kBinChunk);              // [BATCH][rows_per_cta][32]
-    // [2 chunk parities][odd count, even count, odd taken, even taken]
+    // [2 chunk parities][odd count | even count << 16, -, odd taken, even taken]
     int *counts = reinterpret_cast<int *>(acc + BATCH * rows_per_cta * 32);
-    load_smem_image(&S, args.image, sizeof(Smem48));
-    load_smem_image(&E, even, sizeof(SmemEven48));
+    unsigned long long *bar = reinterpret_cast<unsigned long long *>(counts + 8);   // 8-byte aligned
     for (int i = threadIdx.x; i < BATCH * rows_per_cta * 32; i += kBinThreads) acc[i] = 0.f;
     if (threadIdx.x < 8) counts[threadIdx.x] = 0;
     const int row0 = blockIdx.x * rows_per_cta;
@@ -130,44 +114,73 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
         const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
         wnext[k] = t < total ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
     }
+    {
+        void *const dst[2] = {&S, &E};
+        const void *const src[2] = {args.image, even};
+        const uint32_t bytes[2] = {(uint32_t)sizeof(Smem48), (uint32_t)sizeof(SmemEven48)};
+        if (!bulk_load_smem(dst, src, bytes, bar)) {
+            if (threadIdx.x == 0) atomicOr(flags, kFlagWaitTimeout);
+            return;
+        }
+    }
     int parity = 0;
     for (int base = 0; base < total; base += kBinChunk, parity ^= 1) {
         __syncthreads();                       // previous chunk's records consumed; counts reset
         int *cnt = counts + 4 * parity;
         if (threadIdx.x < 4) counts[4 * (parity ^ 1) + threadIdx.x] = 0;
-        // phase 1: classify and sort by coset (warps past the end skip)
+        // phase 1a: classify this thread's blocks of the chunk; an even block on the table path
+        // starts the fetch of its complement code sequence (global memory) right away
+        BinRec rec[kBinPer];
+        bool enq[kBinPer], odd[kBinPer];
 #pragma unroll
         for (int k = 0; k < kBinPer; k++) {
-            if (base + k * kBinThreads + warp_t0 >= total) break;
             const int t = base + k * kBinThreads + threadIdx.x;
-            const bool valid = t < total;
+            enq[k] = false;
+            odd[k] = false;
+            if (base + k * kBinThreads + warp_t0 >= total) continue;         // warp-uniform
             const Cls48 c = classify48(wnext[k], S, args.npoints);
+            const bool valid = t < total;
             bad |= valid && !c.ok;
-            const bool enq = valid && c.ok;
-            const bool odd = c.info & kInfoOdd;
-            const unsigned mo = __ballot_sync(0xFFFFFFFFu, enq && odd);
-            const unsigned me = __ballot_sync(0xFFFFFFFFu, enq && !odd);
-            int bo = 0, be = 0;
-            if (lane == 0) {
-                if (mo) bo = atomicAdd(cnt, __popc(mo));
-                if (me) be = atomicAdd(cnt + 1, __popc(me));
+            enq[k] = valid && c.ok;
+            odd[k] = c.info & kInfoOdd;
+            rec[k].z = c.s;
+            if (!odd[k] && (c.info & kInfoTable)) {
+                const Even48Idx ix = even48_indices(S, c.cls, c.p);
+                rec[k].x = enq[k] ? __ldg(tabC + (S.c_offs[c.cls] & 0x7FFFFu) + ix.pC) : 0u;
+                rec[k].y = (uint32_t)c.cls | c.r << 9 | ix.pS << 21;
+            } else {
+                rec[k].x = (uint32_t)c.p;
+                rec[k].y = (uint32_t)c.cls | c.r << 9 | (uint32_t)(c.p >> 32) << 21;
             }
-            bo = __shfl_sync(0xFFFFFFFFu, bo, 0);
-            be = __shfl_sync(0xFFFFFFFFu, be, 0);
-            if (enq && !odd && (c.info & kInfoTable))   // complement table entry into L1 for phase 2
-                asm volatile("prefetch.global.L1 [%0];" ::"l"(even48_tabC_entry(S, tabC, c.cls, c.p)));
-            if (enq) {
-                const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
-                const int j = t - rl * nb;
-                BinRec e;
-                e.x = (uint32_t)c.p;
-                e.y = (uint32_t)(c.p >> 32) | (uint32_t)c.cls << 1 | c.r << 10 |
-                      (uint32_t)((wnext[k] >> 48) & 0xFFu) << 22;
-                e.z = c.s;
-                e.w = (uint32_t)rl | (uint32_t)j << 16;
-                const int pos = odd ? bo + __popc(mo & lanes_below)
-                                    : kBinChunk - 1 - (be + __popc(me & lanes_below));
-                list[pos] = e;
+        }
+        // phase 1b: one shared-memory atomic per warp reserves its places in both lists
+        {
+            unsigned mo[kBinPer], me[kBinPer];
+            uint32_t no_w = 0, ne_w = 0;
+#pragma unroll
+            for (int k = 0; k < kBinPer; k++) {
+                mo[k] = __ballot_sync(0xFFFFFFFFu, enq[k] && odd[k]);
+                me[k] = __ballot_sync(0xFFFFFFFFu, enq[k] && !odd[k]);
+                no_w += __popc(mo[k]);
+                ne_w += __popc(me[k]);
+            }
+            uint32_t b0 = 0;
+            if (lane == 0 && (no_w | ne_w)) b0 = atomicAdd(reinterpret_cast<unsigned *>(cnt), no_w | ne_w << 16);
+            b0 = __shfl_sync(0xFFFFFFFFu, b0, 0);
+            uint32_t bo = b0 & 0xFFFFu, be = b0 >> 16;
+#pragma unroll
+            for (int k = 0; k < kBinPer; k++) {
+                if (enq[k]) {
+                    const int t = base + k * kBinThreads + threadIdx.x;
+                    const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
+                    rec[k].z |= (uint32_t)((wnext[k] >> 48) & 0xFFu) << 24;
+                    rec[k].w = (uint32_t)rl | (uint32_t)(t - rl * nb) << 16;
+                    const int pos = odd[k] ? (int)(bo + __popc(mo[k] & lanes_below))
+                                           : kBinChunk - 1 - (int)(be + __popc(me[k] & lanes_below));
+                    list[pos] = rec[k];
+                }
+                bo += __popc(mo[k]);
+                be += __popc(me[k]);
             }
         }
         // the next chunk's words load while this chunk decodes
@@ -178,11 +191,10 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
             wnext[k] = t < total ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
         }
         __syncthreads();
-        const int no = cnt[0], ne = cnt[1];
         // phase 2: odd-coset records, then even-coset records; each warp takes the next 32
         // records of a list until both are used up
         for (int list_id = 0; list_id < 2; list_id++) {
-            const int n = cnt[list_id];
+            const int n = list_id == 0 ? (cnt[0] & 0xFFFF) : (cnt[0] >> 16);
             while (true) {
                 int i0 = 0;
                 if (lane == 0) i0 = atomicAdd(cnt + 2 + list_id, 32);
@@ -191,10 +203,10 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
                 const int i = i0 + lane;
                 if (i < n) {
                     if (list_id == 0)
-                        bin48_process<true, BATCH>(list[i], S, E, tabC, gain_mode, gains, X, K, row0, nb, acc,
+                        bin48_process<true, BATCH>(list[i], S, E, gain_mode, gains, X, K, row0, nb, acc,
                                                    rows_per_cta, lane);
                     else
-                        bin48_process<false, BATCH>(list[kBinChunk - 1 - i], S, E, tabC, gain_mode, gains, X, K,
+                        bin48_process<false, BATCH>(list[kBinChunk - 1 - i], S, E, gain_mode, gains, X, K,
                                                     row0, nb, acc, rows_per_cta, lane);
                 }
             }

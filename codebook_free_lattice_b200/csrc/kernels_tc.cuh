@@ -17,12 +17,10 @@
 // step LBO apart (A: 2048 B, B: 1024 B).  One CTA = one 128-row tile x a range of K chunks;
 // several CTAs per tile (split K) add into the zeroed output with atomics.
 #pragma once
-#include "codec48.cuh"
-#include "codec72.cuh"
+#include "kernels.cuh"
 
 namespace llvq {
 
-constexpr unsigned kFlagWaitTimeout = 0x2u;   // a bounded wait gave up (LLVQ_FLAG_WAIT_TIMEOUT)
 
 constexpr int kTcRows = 128;                  // UMMA M
 constexpr int kTcBlocks = 4;                  // 24-weight blocks per K chunk
@@ -63,18 +61,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// int8 x4 -> two half2 (exact): (b ^ 0x80) + 1024 is the fp16 with bits 0x64XX; minus 1152 = b
-__device__ __forceinline__ void i8x4_to_h2x2(uint32_t w, uint32_t &lo, uint32_t &hi) {
-    const uint32_t u = w ^ 0x80808080u;
-    const uint32_t l = __byte_perm(u, 0x64646464u, 0x4140);     // coordinates 0, 1
-    const uint32_t h = __byte_perm(u, 0x64646464u, 0x4342);     // coordinates 2, 3
-    const __half2 bias = __halves2half2(__ushort_as_half((unsigned short)0x6480),
-                                        __ushort_as_half((unsigned short)0x6480));
-    const __half2 a = __hsub2(*reinterpret_cast<const __half2 *>(&l), bias);
-    const __half2 b = __hsub2(*reinterpret_cast<const __half2 *>(&h), bias);
-    lo = *reinterpret_cast<const uint32_t *>(&a);
-    hi = *reinterpret_cast<const uint32_t *>(&b);
-}
 
 template <class D>
 struct TcSmem {

@@ -114,6 +114,15 @@ llvq_status build_image48(const HostTables &T, Smem48 &S, std::string &err) {
         S.c_info[i] = c.A | (uint32_t)c.B << 13 | (c.odd ? kInfoOdd : 0u) |
                       (((c.sum_abs / 4) & 1) ? kInfoParity : 0u) | (uint32_t)c.m << 21 | val4 << 25 | flag4 << 29;
         S.c_info2[i] = wbase | (uint32_t)(c.odd ? 24 : c.k) << 12;
+        if (c.odd) {                                          // signed group values on / off T
+            for (int g = 0; g < (int)c.vals.size(); g++) {
+                const int a = c.vals[g];
+                const unsigned long long on = (unsigned long long)(uint8_t)(int8_t)(a % 4 == 1 ? a : -a);
+                const unsigned long long off = (unsigned long long)(uint8_t)(int8_t)(a % 4 == 3 ? a : -a);
+                S.c_vt[i] |= on << (8 * g);
+                S.c_vn[i] |= off << (8 * g);
+            }
+        }
         S.starts[i] = (unsigned long long)c.start;
     }
     S.starts[nc] = (unsigned long long)T.n_points;

@@ -117,7 +117,7 @@ llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, 
  * a framework allocator.  The paper has no counterpart; this is a packaging variant of
  * llvq_decode for the 48-bit budget only (index_bits must be 48, word_bytes 8; anything else is
  * LLVQ_ERR_UNSUPPORTED / LLVQ_ERR_ARG).  The decode tables and the status word live in one
- * static device array inside the library (70,400 bytes on every device that loads it, held until
+ * static device array inside the library (76,544 bytes on every device that loads it, held until
  * the process exits) instead of a codec.  The first call on a device builds the tables on the
  * host and copies them in synchronously, so make that first call before any stream capture.
  * Calls share the array: indices >= N_M still decode to the zero vector (a coded point is never
