@@ -16,8 +16,8 @@
 namespace llvq {
 
 constexpr int kBinThreads = 1024;                 // one CTA per SM, 64 registers per thread
-constexpr int kBinPer = 4;                        // blocks per thread and chunk
-constexpr int kBinChunk = kBinThreads * kBinPer;  // 4096 blocks = 64 KB of records
+// A chunk holds up to PER blocks per thread (PER = 4 or 5: 64 or 80 KB of records); a CTA splits
+// its blocks into equal chunks so that no chunk is a small remainder.
 
 // One classified block.  y = class | r << 9 | (see below) << 21; z = s | gain code << 24;
 // w = row within the CTA | block column j << 16.  Odd classes and even classes off the table
@@ -25,8 +25,8 @@ constexpr int kBinChunk = kBinThreads * kBinPer;  // 4096 blocks = 64 KB of reco
 // complement's code sequence (fetched while classifying), y bits 21..31 = p_S.
 using BinRec = uint4;
 
-__host__ __device__ constexpr size_t bin48_smem_bytes(int batch, int rows_per_cta) {
-    return sizeof(Smem48) + sizeof(SmemEven48) + sizeof(BinRec) * kBinChunk +
+__host__ __device__ constexpr size_t bin48_smem_bytes(int batch, int rows_per_cta, int per) {
+    return sizeof(Smem48) + sizeof(SmemEven48) + sizeof(BinRec) * kBinThreads * per +
            sizeof(float) * (size_t)batch * rows_per_cta * 32 + 8 * sizeof(int) + 8;
 }
 
@@ -80,7 +80,7 @@ __device__ __forceinline__ void bin48_process(const BinRec e, const Smem48 &S, c
     accumulate_block<BATCH>(v, scale, X, K, j, acc, rl, rows_per_cta, lane);
 }
 
-template <int BATCH>
+template <int BATCH, int PER>
 __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
     Dec48::Args args, const SmemEven48 *even, const uint32_t *__restrict__ tabC,
     const unsigned long long *__restrict__ words, long long pitch, int rows, int nb,
@@ -90,7 +90,8 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
     Smem48 &S = *reinterpret_cast<Smem48 *>(smem_raw);
     SmemEven48 &E = *reinterpret_cast<SmemEven48 *>(smem_raw + sizeof(Smem48));
     BinRec *list = reinterpret_cast<BinRec *>(smem_raw + sizeof(Smem48) + sizeof(SmemEven48));
-    float *acc = reinterpret_cast<float *>(list + kBinChunk);              // [BATCH][rows_per_cta][32]
+    constexpr int kCap = kBinThreads * PER;                                 // records per chunk
+    float *acc = reinterpret_cast<float *>(list + kCap);                    // [BATCH][rows_per_cta][32]
     // [2 chunk parities][odd count | even count << 16, -, odd taken, even taken]
     int *counts = reinterpret_cast<int *>(acc + BATCH * rows_per_cta * 32);
     unsigned long long *bar = reinterpret_cast<unsigned long long *>(counts + 8);   // 8-byte aligned
@@ -99,6 +100,8 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
     const int row0 = blockIdx.x * rows_per_cta;
     const int nrows = max(0, min(rows_per_cta, rows - row0));
     const int total = nrows * nb;
+    const int nchunks = (total + kCap - 1) / kCap;
+    const int chunk = nchunks > 0 ? (total + nchunks - 1) / nchunks : 0;
     const long long K = (long long)nb * 24;
     const int lane = threadIdx.x & 31;
     const unsigned lanes_below = (1u << lane) - 1u;
@@ -107,12 +110,12 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
     // block t of the CTA -> row rl = t / nb (multiply-high with ceil(2^32 / nb)), column t - rl nb
     const unsigned long long *wbase = words + (long long)row0 * pitch;
     const int warp_t0 = threadIdx.x & ~31;
-    unsigned long long wnext[kBinPer];
+    unsigned long long wnext[PER];
 #pragma unroll
-    for (int k = 0; k < kBinPer; k++) {
+    for (int k = 0; k < PER; k++) {
         const int t = k * kBinThreads + threadIdx.x;
         const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
-        wnext[k] = t < total ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
+        wnext[k] = t < min(chunk, total) ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
     }
     {
         void *const dst[2] = {&S, &E};
@@ -124,22 +127,23 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
         }
     }
     int parity = 0;
-    for (int base = 0; base < total; base += kBinChunk, parity ^= 1) {
+    for (int base = 0; base < total; base += chunk, parity ^= 1) {
+        const int end = min(base + chunk, total);
         __syncthreads();                       // previous chunk's records consumed; counts reset
         int *cnt = counts + 4 * parity;
         if (threadIdx.x < 4) counts[4 * (parity ^ 1) + threadIdx.x] = 0;
         // phase 1a: classify this thread's blocks of the chunk; an even block on the table path
         // starts the fetch of its complement code sequence (global memory) right away
-        BinRec rec[kBinPer];
-        bool enq[kBinPer], odd[kBinPer];
+        BinRec rec[PER];
+        bool enq[PER], odd[PER];
 #pragma unroll
-        for (int k = 0; k < kBinPer; k++) {
+        for (int k = 0; k < PER; k++) {
             const int t = base + k * kBinThreads + threadIdx.x;
             enq[k] = false;
             odd[k] = false;
-            if (base + k * kBinThreads + warp_t0 >= total) continue;         // warp-uniform
+            if (base + k * kBinThreads + warp_t0 >= end) continue;           // warp-uniform
             const Cls48 c = classify48(wnext[k], S, args.npoints);
-            const bool valid = t < total;
+            const bool valid = t < end;
             bad |= valid && !c.ok;
             enq[k] = valid && c.ok;
             odd[k] = c.info & kInfoOdd;
@@ -155,10 +159,10 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
         }
         // phase 1b: one shared-memory atomic per warp reserves its places in both lists
         {
-            unsigned mo[kBinPer], me[kBinPer];
+            unsigned mo[PER], me[PER];
             uint32_t no_w = 0, ne_w = 0;
 #pragma unroll
-            for (int k = 0; k < kBinPer; k++) {
+            for (int k = 0; k < PER; k++) {
                 mo[k] = __ballot_sync(0xFFFFFFFFu, enq[k] && odd[k]);
                 me[k] = __ballot_sync(0xFFFFFFFFu, enq[k] && !odd[k]);
                 no_w += __popc(mo[k]);
@@ -169,14 +173,14 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
             b0 = __shfl_sync(0xFFFFFFFFu, b0, 0);
             uint32_t bo = b0 & 0xFFFFu, be = b0 >> 16;
 #pragma unroll
-            for (int k = 0; k < kBinPer; k++) {
+            for (int k = 0; k < PER; k++) {
                 if (enq[k]) {
                     const int t = base + k * kBinThreads + threadIdx.x;
                     const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
                     rec[k].z |= (uint32_t)((wnext[k] >> 48) & 0xFFu) << 24;
                     rec[k].w = (uint32_t)rl | (uint32_t)(t - rl * nb) << 16;
                     const int pos = odd[k] ? (int)(bo + __popc(mo[k] & lanes_below))
-                                           : kBinChunk - 1 - (int)(be + __popc(me[k] & lanes_below));
+                                           : kCap - 1 - (int)(be + __popc(me[k] & lanes_below));
                     list[pos] = rec[k];
                 }
                 bo += __popc(mo[k]);
@@ -185,15 +189,18 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
         }
         // the next chunk's words load while this chunk decodes
 #pragma unroll
-        for (int k = 0; k < kBinPer; k++) {
-            const int t = base + kBinChunk + k * kBinThreads + threadIdx.x;
+        for (int k = 0; k < PER; k++) {
+            const int t = end + k * kBinThreads + threadIdx.x;
             const int rl = nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip);
-            wnext[k] = t < total ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
+            wnext[k] = t < min(end + chunk, total) ? __ldg(wbase + (long long)rl * pitch + (t - rl * nb)) : 0ull;
         }
         __syncthreads();
-        // phase 2: odd-coset records, then even-coset records; each warp takes the next 32
-        // records of a list until both are used up
-        for (int list_id = 0; list_id < 2; list_id++) {
+        // phase 2: each warp takes the next 32 records of a list until both lists are used up;
+        // even-numbered warps start on the odd-coset list and odd-numbered warps on the even-coset
+        // list, so the arithmetic-heavy and the lookup-latency-bound decodes share the SM
+        const int first = (threadIdx.x >> 5) & 1;
+        for (int pass = 0; pass < 2; pass++) {
+            const int list_id = first ^ pass;
             const int n = list_id == 0 ? (cnt[0] & 0xFFFF) : (cnt[0] >> 16);
             while (true) {
                 int i0 = 0;
@@ -206,7 +213,7 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_gemm_bin48(
                         bin48_process<true, BATCH>(list[i], S, E, gain_mode, gains, X, K, row0, nb, acc,
                                                    rows_per_cta, lane);
                     else
-                        bin48_process<false, BATCH>(list[kBinChunk - 1 - i], S, E, gain_mode, gains, X, K,
+                        bin48_process<false, BATCH>(list[kCap - 1 - i], S, E, gain_mode, gains, X, K,
                                                     row0, nb, acc, rows_per_cta, lane);
                 }
             }

@@ -304,7 +304,8 @@ constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per bl
 
 template <int... Bs>
 void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
-    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
 }
 
 // Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
@@ -334,15 +335,19 @@ cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_wei
     const int nb = w->blocks_per_row;
     if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
     int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
-    while (rpc > 1 && bin48_smem_bytes(B, rpc) > kBinSmemLimit) rpc = (rpc + 1) / 2;
-    if (bin48_smem_bytes(B, rpc) > kBinSmemLimit) return cudaErrorInvalidValue;
+    while (rpc > 1 && bin48_smem_bytes(B, rpc, 4) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (bin48_smem_bytes(B, rpc, 4) > kBinSmemLimit) return cudaErrorInvalidValue;
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
     const int grid = (w->rows + rpc - 1) / rpc;
     const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
-    k_gemm_bin48<B><<<grid, kBinThreads, bin48_smem_bytes(B, rpc), st>>>(
-        a, (const SmemEven48 *)c->d_even48, c->d_tabC48, (const unsigned long long *)w->words, w->row_pitch_words, w->rows, nb, recip, w->gain_mode,
-        (const __half *)w->gains, (const __half *)X, Y, rpc, c->d_flags);
+    const bool per5 = bin48_smem_bytes(B, rpc, 5) <= kBinSmemLimit;   // larger chunks when they fit
+    const size_t smem = bin48_smem_bytes(B, rpc, per5 ? 5 : 4);
+    auto kern = per5 ? k_gemm_bin48<B, 5> : k_gemm_bin48<B, 4>;
+    kern<<<grid, kBinThreads, smem, st>>>(a, (const SmemEven48 *)c->d_even48, c->d_tabC48,
+                                          (const unsigned long long *)w->words, w->row_pitch_words, w->rows, nb,
+                                          recip, w->gain_mode, (const __half *)w->gains, (const __half *)X, Y, rpc,
+                                          c->d_flags);
     return cudaGetLastError();
 }
 
