@@ -268,6 +268,21 @@ Dec72::Args args72(const llvq_codec *c) {
 template <class D>
 cudaError_t launch_decode(const llvq_codec *c, typename D::Args a, const void *words, long long n,
                           int8_t *out, cudaStream_t st) {
+    if constexpr (std::is_same<D, Dec48>::value) {
+        // coset-sorted decode: one 1024-thread CTA per SM over a contiguous range of words
+        if (n == 0) return cudaSuccess;
+        const int grid = (int)std::max(1LL, std::min((long long)c->num_sms, (n + kBinThreads - 1) / kBinThreads));
+        const long long per = (n + grid - 1) / grid;
+        if (per >= (1LL << 31)) return cudaErrorInvalidValue;
+        DecodeSink sink{};
+        sink.words = (const unsigned long long *)words;
+        sink.n = n;
+        sink.out = out;
+        sink.per_cta = per;
+        k_bin48<DecodeSink, kBinPer><<<grid, kBinThreads, bin48_base_smem(kBinPer), st>>>(
+            a, (const SmemEven48 *)c->d_even48, c->d_tabC48, sink, c->d_flags);
+        return cudaGetLastError();
+    }
     const int threads = 512;
     const long long want = (n + threads - 1) / threads;
     const int grid = (int)std::max(1LL, std::min(want, (long long)c->num_sms * D::kCtasPerSm));
@@ -304,8 +319,10 @@ constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per bl
 
 template <int... Bs>
 void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
-    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
-    (cudaFuncSetAttribute(k_gemm_bin48<Bs + 1, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          (int)kBinSmemLimit), ...);
+    cudaFuncSetAttribute(k_bin48<DecodeSink, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)kBinSmemLimit);
 }
 
 // Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
@@ -335,19 +352,26 @@ cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_wei
     const int nb = w->blocks_per_row;
     if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
     int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
-    while (rpc > 1 && bin48_smem_bytes(B, rpc, 4) > kBinSmemLimit) rpc = (rpc + 1) / 2;
-    if (bin48_smem_bytes(B, rpc, 4) > kBinSmemLimit) return cudaErrorInvalidValue;
+    while (rpc > 1 && bin48_smem_bytes(B, rpc, kBinPer) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (bin48_smem_bytes(B, rpc, kBinPer) > kBinSmemLimit) return cudaErrorInvalidValue;
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
     const int grid = (w->rows + rpc - 1) / rpc;
     const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
-    const bool per5 = bin48_smem_bytes(B, rpc, 5) <= kBinSmemLimit;   // larger chunks when they fit
-    const size_t smem = bin48_smem_bytes(B, rpc, per5 ? 5 : 4);
-    auto kern = per5 ? k_gemm_bin48<B, 5> : k_gemm_bin48<B, 4>;
-    kern<<<grid, kBinThreads, smem, st>>>(a, (const SmemEven48 *)c->d_even48, c->d_tabC48,
-                                          (const unsigned long long *)w->words, w->row_pitch_words, w->rows, nb,
-                                          recip, w->gain_mode, (const __half *)w->gains, (const __half *)X, Y, rpc,
-                                          c->d_flags);
+    const size_t smem = bin48_smem_bytes(B, rpc, kBinPer);
+    GemvSink<B> sink{};
+    sink.words = (const unsigned long long *)w->words;
+    sink.pitch = w->row_pitch_words;
+    sink.rows = w->rows;
+    sink.nb = nb;
+    sink.nb_recip = recip;
+    sink.gain_mode = w->gain_mode;
+    sink.gains = (const __half *)w->gains;
+    sink.X = (const __half *)X;
+    sink.Y = Y;
+    sink.rows_per_cta = rpc;
+    k_bin48<GemvSink<B>, kBinPer><<<grid, kBinThreads, smem, st>>>(a, (const SmemEven48 *)c->d_even48, c->d_tabC48,
+                                                                  sink, c->d_flags);
     return cudaGetLastError();
 }
 
