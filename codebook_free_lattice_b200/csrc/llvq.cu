@@ -387,27 +387,18 @@ cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_we
             case 4: return launch_gemm_bin48<4>(c, a, w, X, Y, s);
             case 5: return launch_gemm_bin48<5>(c, a, w, X, Y, s);
             case 6: return launch_gemm_bin48<6>(c, a, w, X, Y, s);
-            case 7: return launch_gemm_bin48<7>(c, a, w, X, Y, s);
-            default: break;
+            default: return launch_gemm_bin48<7>(c, a, w, X, Y, s);
         }
-    }
-    switch (batch) {
-        case 1: return launch_gemm<D, 1>(c, a, w, X, Y, s);
-        case 2: return launch_gemm<D, 2>(c, a, w, X, Y, s);
-        case 3: return launch_gemm<D, 3>(c, a, w, X, Y, s);
-        case 4: return launch_gemm<D, 4>(c, a, w, X, Y, s);
-        case 5: return launch_gemm<D, 5>(c, a, w, X, Y, s);
-        case 6: return launch_gemm<D, 6>(c, a, w, X, Y, s);
-        case 7: return launch_gemm<D, 7>(c, a, w, X, Y, s);
-        case 8: return launch_gemm<D, 8>(c, a, w, X, Y, s);
-        case 9: return launch_gemm<D, 9>(c, a, w, X, Y, s);
-        case 10: return launch_gemm<D, 10>(c, a, w, X, Y, s);
-        case 11: return launch_gemm<D, 11>(c, a, w, X, Y, s);
-        case 12: return launch_gemm<D, 12>(c, a, w, X, Y, s);
-        case 13: return launch_gemm<D, 13>(c, a, w, X, Y, s);
-        case 14: return launch_gemm<D, 14>(c, a, w, X, Y, s);
-        case 15: return launch_gemm<D, 15>(c, a, w, X, Y, s);
-        default: return launch_gemm<D, 16>(c, a, w, X, Y, s);
+    } else {
+        switch (batch) {
+            case 1: return launch_gemm<D, 1>(c, a, w, X, Y, s);
+            case 2: return launch_gemm<D, 2>(c, a, w, X, Y, s);
+            case 3: return launch_gemm<D, 3>(c, a, w, X, Y, s);
+            case 4: return launch_gemm<D, 4>(c, a, w, X, Y, s);
+            case 5: return launch_gemm<D, 5>(c, a, w, X, Y, s);
+            case 6: return launch_gemm<D, 6>(c, a, w, X, Y, s);
+            default: return launch_gemm<D, 7>(c, a, w, X, Y, s);
+        }
     }
 }
 
@@ -568,8 +559,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
         cudaFuncSetAttribute(k_gemm_tc<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec48>));
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
-        set_gemm_attrs<Dec48>(std::make_integer_sequence<int, 16>{});
-        set_gemm_attrs<Dec72>(std::make_integer_sequence<int, 16>{});
+        set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
     });
     *out = c;
     return LLVQ_OK;
