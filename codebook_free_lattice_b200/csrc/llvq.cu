@@ -16,6 +16,7 @@
 #include "kernels.cuh"
 #include "kernels_bin48.cuh"
 #include "kernels_tc.cuh"
+#include "kernels_tc48.cuh"
 #include "tables.h"
 
 using namespace llvq;
@@ -375,10 +376,38 @@ cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_wei
     return cudaGetLastError();
 }
 
+// 48-bit tensor-core path: 128-row tiles x K splits of 8-block rounds.  The split is chosen to
+// minimise (waves of CTAs) x (rounds per CTA + one round of fixed cost: tables, TMEM, epilogue).
+cudaError_t launch_gemm_tc48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, int batch,
+                             float *Y, cudaStream_t st) {
+    const int mt = (w->rows + kTcRows - 1) / kTcRows;
+    const int nrounds = (w->blocks_per_row + kTc48Slots - 1) / kTc48Slots;
+    int best_rps = nrounds;
+    long long best_cost = -1;
+    for (int sp = 1; sp <= nrounds; sp++) {
+        const int rps = (nrounds + sp - 1) / sp;
+        const int splits = (nrounds + rps - 1) / rps;
+        const long long waves = ((long long)mt * splits + c->num_sms - 1) / c->num_sms;
+        const long long cost = waves * (rps + 1);
+        if (best_cost < 0 || cost < best_cost) { best_cost = cost; best_rps = rps; }
+    }
+    const int splits = std::max(1, (nrounds + best_rps - 1) / best_rps);
+    cudaError_t e = cudaMemsetAsync(Y, 0, (size_t)batch * w->rows * sizeof(float), st);
+    if (e != cudaSuccess) return e;
+    k_gemm_tc48<<<dim3(mt, splits), kTc48Threads, tc48_smem_bytes(), st>>>(
+        a, (const SmemEven48 *)c->d_even48, c->d_tabC48, (const unsigned long long *)w->words, w->row_pitch_words,
+        w->rows, w->blocks_per_row, batch, w->gain_mode, (const __half *)w->gains, (const __half *)X, Y, best_rps,
+        c->d_flags);
+    return cudaGetLastError();
+}
+
 template <class D>
 cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
                           int batch, float *Y, cudaStream_t s) {
-    if (batch >= kTensorCoreMinBatch) return launch_gemm_tc<D>(c, a, w, X, batch, Y, s);
+    if (batch >= kTensorCoreMinBatch) {
+        if constexpr (std::is_same<D, Dec48>::value) return launch_gemm_tc48(c, a, w, X, batch, Y, s);
+        else return launch_gemm_tc<D>(c, a, w, X, batch, Y, s);
+    }
     if constexpr (std::is_same<D, Dec48>::value) {
         switch (batch) {
             case 1: return launch_gemm_bin48<1>(c, a, w, X, Y, s);
@@ -556,8 +585,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::call_once(once, [] {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
-        cudaFuncSetAttribute(k_gemm_tc<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec48>));
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
+        cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
         cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
     });
