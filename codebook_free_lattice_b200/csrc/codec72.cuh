@@ -6,7 +6,8 @@
 //   - indices are 72-bit (word = two little-endian 64-bit halves; gain code in bits 72..79);
 //   - class records (96 B) and the guide table on the top 16 index bits live in global memory
 //     (L2-resident, 9.5 MB), the Golay tables in shared memory;
-//   - I_class < 2^63, so r, s, I'' come from one 64-bit division by A;
+//   - I_class < 2^63, so r, s, I'' come from one 64-bit division by A (a multiply-high by a
+//     per-class reciprocal and one correction);
 //   - arrangement counts reach P ~ 2^50.2, beyond fp64, so the arithmetic decoding state is
 //     a 64-bit fixed-point fraction kept above the exact value: slot = high word of phi * L,
 //     and phi <- (slot_in_group * 2^64 + low word) * R_c with R_c = ceil(2^64 / c) (plus one).
@@ -33,7 +34,7 @@ struct alignas(16) Rec72 {
     uint16_t wbase, pad1;
     uint32_t pad2;
     unsigned long long PC;                   // arrangements off S (even), 1 for odd classes
-    unsigned long long pad3;
+    unsigned long long mA;                   // floor((2^64 - 1) / A): I_class / A by multiply-high
 };
 static_assert(sizeof(Rec72) == 96, "Rec72 layout");
 
@@ -83,8 +84,10 @@ struct Dec72 {
         m = R.m;
         // 2. I_class = idx - start < 2^63 (the high halves cancel), then r, s, I''
         const unsigned long long Ic = lo - R.start_lo;
-        const unsigned long long q = Ic / R.A;
-        const uint32_t r = (uint32_t)(Ic - q * R.A);
+        // q = floor(I_class / A): the multiply-high by floor((2^64 - 1)/A) is q or q - 1
+        unsigned long long q = __umul64hi(Ic, R.mA);
+        uint32_t r = (uint32_t)(Ic - q * R.A);
+        if (r >= R.A) { q += 1; r -= R.A; }
         const uint32_t s = (uint32_t)(q & ((1ull << R.B) - 1ull));
         const unsigned long long p = q >> R.B;
         // 3. codeword

@@ -226,6 +226,7 @@ llvq_status build_image72(const HostTables &T, Smem72 &S, std::vector<Rec72> &re
             R.Rfrac = (unsigned long long)(((rem << 64) + c.P - 1) / c.P);
         }
         R.PC = (unsigned long long)c.P_C;
+        R.mA = ~0ull / c.A;
         R.cum = cum_bytes(c, 8);
         for (int g = 0; g < 8 && g < (int)c.vals.size(); g++) {
             R.vals |= (unsigned long long)c.vals[g] << (8 * g);
