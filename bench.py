@@ -53,17 +53,37 @@ def kernel_sources_hash() -> str:
     return h.hexdigest()
 
 
-def measured_traffic():
-    """DRAM bytes per launch of the metric's kernel from the committed ncu capture, or None when
-    the kernel sources changed since the capture."""
+def profile_record():
+    """The committed ncu record of the metric's kernel (DRAM bytes and warp instructions per
+    launch), or None when the kernel sources changed since the capture."""
     try:
         with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
             rec = json.load(f)
         if rec.get("kernel_sources_sha256") == kernel_sources_hash():
-            return int(rec["traffic_bytes_per_launch"])
+            return rec
     except Exception:
         pass
     return None
+
+
+def measured_traffic():
+    rec = profile_record()
+    return int(rec["traffic_bytes_per_launch"]) if rec else None
+
+
+def issue_roofline(per_launch_s, sm_mhz):
+    """Instruction-issue roofline of the metric's kernel: thread-instructions per second (ncu count
+    of one launch / the measured launch time) against 148 SMs x 4 schedulers x 32 lanes x the SM
+    clock measured during the timed region (one warp-instruction per scheduler and cycle)."""
+    rec = profile_record()
+    if not rec or "warp_instructions_per_launch" not in rec or not sm_mhz:
+        return None
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    achieved = rec["warp_instructions_per_launch"] * 32 / per_launch_s
+    peak = sms * 4 * 32 * sm_mhz * 1e6
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "thread-instructions/s",
+            "frac": achieved / peak,
+            "peak_source": f"{sms} SMs x 4 schedulers x 32 lanes x {sm_mhz:.0f} MHz (clock measured under load)"}
 
 
 def measured_peaks():
@@ -472,6 +492,8 @@ def main():
             "gpu_launches": launches,
             "clocks": clk,
         }
+        if B == 1:
+            line["issue_roofline"] = issue_roofline(per_launch_s, clk.get("sm_mhz") if clk else None)
         line["decode"] = decode_throughput(torch, codec, dev, args.decode_n, 5, 2)
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()

@@ -214,6 +214,12 @@ __device__ __forceinline__ void odd_step48(int i, double &f, uint32_t &cumB, uin
     sel[i >> 2] += ssel << (4 * (i & 3));
 }
 
+// The last coordinate: one place left, so the slot is 0 and the group is the one item left.
+__device__ __forceinline__ void odd_last_step48(uint32_t cumB, uint32_t sel[6]) {
+    const uint32_t dm = (cumB >> 7) & 0x01010101u;
+    sel[5] += (uint32_t)__dp4a((int)dm, -1, 7) << 12;
+}
+
 // Steps 3-5 for an odd class only: one coordinate set, so the places left at coordinate i are
 // 24 - i and the slot needs no offset.  x_i = a_i exactly when (i in T) equals (a_i = 1 mod 4),
 // so each group has one signed value on T and one off T: a byte permutation of each table by the
@@ -226,7 +232,8 @@ __device__ __forceinline__ void arrange_odd48(const Smem48 &S, int cls, uint32_t
     uint32_t sel[6] = {0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u,
                        0u - 0x3333u, 0u - 0x3333u, 0u - 0x3333u};
 #pragma unroll
-    for (int i = 0; i < 24; i++) odd_step48(i, f, cumB, sel, S.invc);
+    for (int i = 0; i < 23; i++) odd_step48(i, f, cumB, sel, S.invc);
+    odd_last_step48(cumB, sel);
     const unsigned long long vt = S.c_vt[cls], vn = S.c_vn[cls];
 #pragma unroll
     for (int q = 0; q < 6; q++) {

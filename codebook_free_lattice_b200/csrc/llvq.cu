@@ -321,7 +321,9 @@ constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per bl
 
 template <int... Bs>
 void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
-    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                           (int)kBinSmemLimit), ...);
     cudaFuncSetAttribute(k_bin48<DecodeSink, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kBinSmemLimit);
@@ -353,14 +355,16 @@ cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_wei
                               cudaStream_t st) {
     const int nb = w->blocks_per_row;
     if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
+    // one CTA per SM over a row range; 5 blocks per thread and chunk when the row accumulators
+    // leave room, else 4, else the row range shrinks (more CTAs than SMs)
     int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
-    while (rpc > 1 && bin48_smem_bytes(B, rpc, kBinPer) > kBinSmemLimit) rpc = (rpc + 1) / 2;
-    if (bin48_smem_bytes(B, rpc, kBinPer) > kBinSmemLimit) return cudaErrorInvalidValue;
+    int per = bin48_smem_bytes(B, rpc, 5) <= kBinSmemLimit ? 5 : 4;
+    while (rpc > 1 && bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) return cudaErrorInvalidValue;
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
     const int grid = (w->rows + rpc - 1) / rpc;
     const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
-    const size_t smem = bin48_smem_bytes(B, rpc, kBinPer);
     GemvSink<B> sink{};
     sink.words = (const unsigned long long *)w->words;
     sink.pitch = w->row_pitch_words;
@@ -372,8 +376,9 @@ cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_wei
     sink.X = (const __half *)X;
     sink.Y = Y;
     sink.rows_per_cta = rpc;
-    k_bin48<GemvSink<B>, kBinPer><<<grid, kBinThreads, smem, st>>>(a, (const SmemEven48 *)c->d_even48, c->d_tabC48,
-                                                                  sink, c->d_flags);
+    auto kern = per == 5 ? k_bin48<GemvSink<B>, 5> : k_bin48<GemvSink<B>, 4>;
+    kern<<<grid, kBinThreads, bin48_smem_bytes(B, rpc, per), st>>>(a, (const SmemEven48 *)c->d_even48,
+                                                                  c->d_tabC48, sink, c->d_flags);
     return cudaGetLastError();
 }
 
