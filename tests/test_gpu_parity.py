@@ -178,6 +178,29 @@ def test_gemm_table_gains_ragged(gcodec, ocodec, rows, K, batch, pitch):
     assert max_rel_err(y, ref) < GEMV_RTOL
 
 
+@pytest.mark.parametrize("batch", [1, 3, 16])
+def test_gemm_out_of_range_blocks(gcodec, ocodec, batch):
+    """Blocks whose index is >= N_M contribute nothing (the oracle skips them) and raise the
+    index-range flag, on the CUDA-core path (batch 1, 3) and the tensor-core path (batch 16)."""
+    import codebook_free_lattice_b200 as L
+    layer = Layer(48, 150, 24 * 37, batch, 30 + batch, ocodec.n_points, 1)
+    w = layer.words.reshape(-1)
+    w[::17] = (w[::17] & ~np.uint64(0xFFFFFFFFFFFF)) | np.uint64(ocodec.n_points + 99)
+    w[5::23] = (w[5::23] & ~np.uint64(0xFFFFFFFFFFFF)) | np.uint64(2**48 - 1)
+    words = torch.from_numpy(np.ascontiguousarray(layer.words).view(np.int64)).cuda()
+    gains = torch.from_numpy(layer.gains.view(np.int16)).cuda()
+    X = torch.from_numpy(layer.x[:batch].view(np.int16)).cuda()
+    Y = torch.full((batch, layer.rows), float("nan"), dtype=torch.float32, device="cuda")
+    wt = gcodec.weight(words, gains, layer.rows, layer.K, layer.gain_mode, layer.pitch)
+    if batch == 1:
+        gcodec.gemv(wt, X, Y)
+    else:
+        gcodec.gemm(wt, X, Y, batch)
+    assert gcodec.get_error() == L.LLVQ_FLAG_INDEX_RANGE
+    y = Y.cpu().numpy().astype(np.float64)
+    assert max_rel_err(y, oracle_gemm(ocodec, layer)) < GEMV_RTOL
+
+
 def test_gemm_batch_equals_gemv_columns(gcodec, ocodec):
     layer = Layer(48, 200, 24 * 50, 5, 9, ocodec.n_points, 1)
     Y = run_gemm(gcodec, layer)
