@@ -7,18 +7,23 @@
 //
 // A CTA (1024 threads, one per SM) owns a 128-row tile and a range of K rounds.  A round covers
 // 8 blocks of each row (1024 blocks, one per thread to classify):
-//   1. thread t classifies block (row t / 8, slot t % 8) and appends a record to the odd or the
-//      even list, as in k_bin48; blocks outside the matrix or with a bad index get a zero A entry
-//      and a zero gain;
-//   2. warps take 32 records of one list at a time, decode them and write the 24 fp16 values and
-//      the gain of each block to its A position; meanwhile the block-diagonal activation tiles
-//      B_0, B_1 (slots 0..3, 4..7; N = 4 slots x 16 batch columns) are filled;
-//   3. one thread issues 2 x 6 MMAs (M = 128, N = 64, K = 96) into 128 TMEM columns and commits
-//      them to an mbarrier (bounded wait);
-//   4. warp w reads TMEM lanes 32 (w % 4).. (rows) and the 16 columns of slot w / 4, and adds
-//      gain * D into its 16 fp32 accumulators (one per batch column).
-// At the end the 8 slots of each row are summed in shared memory and added into y (zeroed by the
-// launch; K splits add).
+//   1. thread t classifies block (row t / 8, slot t % 8) and appends a record (with the block's
+//      fp16 gain) to the odd or the even list, as in k_bin48; the next round's word, gain and
+//      activation chunk are loaded meanwhile;
+//   -- barrier --
+//   2. the previous round's MMAs have had the whole classify phase to finish: a bounded wait on
+//      their mbarrier, then warp w reads TMEM lanes 32 (w % 4).. (rows) and the 16 columns of
+//      slot w / 4 and adds gain * D into its 16 fp32 accumulators (one per batch column);
+//   3. the block-diagonal activation tiles B_0, B_1 (slots 0..3, 4..7; N = 4 slots x 16 batch
+//      columns) are stored; warps take 32 records of one list at a time, decode them and write
+//      the 24 exact fp16 values and the gain of each block to its A position (blocks outside
+//      the matrix or with a bad index get a zero A entry and a zero gain);
+//   -- barrier --
+//   4. one thread issues 2 x 6 MMAs (M = 128, N = 64, K = 96) into 128 TMEM columns and commits
+//      them to the mbarrier; the CTA goes on with the next round's classify at once.
+// Two CTA barriers per round; the MMA round trip hides behind the classify phase.  At the end
+// the 8 slots of each row are summed in shared memory and added into y (zeroed by the launch;
+// K splits add).
 #pragma once
 #include "kernels_bin48.cuh"
 #include "kernels_tc.cuh"
@@ -61,6 +66,27 @@ __device__ __forceinline__ void tc48_store_a(Tc48Smem &T, int dr, int jj, const 
             make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
 }
 
+// bounded wait for the round's MMAs; the result is the same in every lane of the warp, so the
+// warp-collective TMEM load that follows is taken by all lanes or by none
+__device__ __forceinline__ bool tc48_wait_mma(Tc48Smem &T, uint32_t phase) {
+    bool done = false;
+    for (int it = 0; it < (1 << 20) && !done; it++) done = mbar_try_wait_parity(smem_u32(&T.mbar_mma), phase);
+    return __all_sync(0xFFFFFFFFu, done);
+}
+
+// gain * D of this warp's 32 rows and one slot (16 batch columns) into the accumulators
+__device__ __forceinline__ void tc48_epilogue(uint32_t taddr, float g, float yacc[16]) {
+    uint32_t d[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]), "=r"(d[7]),
+          "=r"(d[8]), "=r"(d[9]), "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]), "=r"(d[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int b = 0; b < 16; b++) yacc[b] = fmaf(g, __uint_as_float(d[b]), yacc[b]);
+}
+
 __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
     Dec48::Args args, const SmemEven48 *even, const uint32_t *__restrict__ tabC,
     const unsigned long long *__restrict__ words, long long pitch, int rows, int nb, int batch, int gain_mode,
@@ -79,11 +105,37 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
     const long long K = (long long)nb * 24;
     const int dr = tid >> 3, djj = tid & 7;                   // classify role: row, slot
     const int row = row0 + dr;
+    const bool row_in = row < rows;
+    const unsigned short *gbits = reinterpret_cast<const unsigned short *>(gains);
+    // activation role: threads 0..383 own one 16-byte chunk (slot, batch column, third) of B
+    constexpr int kXChunks = kTcBlocks * 16 * 3;
+    const bool xrole = tid < 2 * kXChunks;
+    const int xhalf = tid / kXChunks, xu = tid % kXChunks;
+    const int xq = xu % 3, xn = xu / 3;                       // n = 16 slot + b
+    const int xjj = xn >> 4, xb = xn & 15;
+    auto load_x = [&](int ch) {
+        const int j = ch * kTc48Slots + 4 * xhalf + xjj;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (xrole && xb < batch && j < nb) v = __ldg(reinterpret_cast<const uint4 *>(X + xb * K + (long long)j * 24 + 8 * xq));
+        return v;
+    };
+    // this thread's word (and, with per-block gains, its gain) of round ch
+    auto load_word = [&](int ch) {
+        const int j = ch * kTc48Slots + djj;
+        return row_in && j < nb ? __ldg(words + (long long)row * pitch + j) : 0ull;
+    };
+    auto load_gain = [&](int ch) {
+        const int j = ch * kTc48Slots + djj;
+        return gain_mode == 0 && row_in && j < nb ? __ldg(gbits + (long long)row * nb + j) : (unsigned short)0;
+    };
 
-    // first round's word, then the tables (bulk copy, bounded wait)
+    // first round's word, gain and activations, then the tables (bulk copy, bounded wait)
     unsigned long long wcur = 0ull;
-    if (c0 < c1 && row < rows && c0 * kTc48Slots + djj < nb)
-        wcur = __ldg(words + (long long)row * pitch + c0 * kTc48Slots + djj);
+    unsigned short gcur = 0;
+    if (c0 < c1) {
+        wcur = load_word(c0);
+        gcur = load_gain(c0);
+    }
     if (tid < 8) T.counts[tid] = 0;
     // B tiles: only the diagonal chunks are written per round; the rest stays zero
     for (int i = tid; i < 2 * kTcBSize / 16; i += kTc48Threads)
@@ -114,6 +166,7 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
 
     const int lg = warp & 3, eslot = warp >> 2;               // epilogue role: lane quarter, slot
     const int em = lg * 32 + lane;
+    const uint32_t etaddr = tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(eslot * 16);
     float yacc[16];
 #pragma unroll
     for (int b = 0; b < 16; b++) yacc[b] = 0.f;
@@ -124,17 +177,23 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
         const int j0 = ch * kTc48Slots;
         int *cnt = T.counts + 4 * (ch & 1);
         if (tid < 4) T.counts[4 * ((ch & 1) ^ 1) + tid] = 0;
+        // the previous round's gain of this thread's epilogue row and slot (written before the
+        // last barrier; this round's decode overwrites it only after the next one)
+        const float gep = ch > c0 ? T.gain[eslot][em] : 0.f;
         // ---- 1. classify this thread's block; append its record
+        bool zero_a;
         {
-            const int j = j0 + djj;
-            const bool inside = row < rows && j < nb;
+            const bool inside = row_in && j0 + djj < nb;
+            const uint32_t code = (uint32_t)((wcur >> 48) & 0xFFu);
+            const unsigned short gh = gain_mode == 0 ? gcur : inside ? __ldg(gbits + (long long)row * 256 + code) : (unsigned short)0;
             const Cls48 c = classify48(wcur, S, args.npoints);
             bad |= inside && !c.ok;
             const bool enq = inside && c.ok;
             const bool odd = c.info & kInfoOdd;
+            zero_a = !enq;
             BinRec rec;
-            rec.z = c.s | (uint32_t)((wcur >> 48) & 0xFFu) << 24;
-            rec.w = (uint32_t)dr | (uint32_t)djj << 8;
+            rec.z = c.s | code << 24;
+            rec.w = (uint32_t)dr | (uint32_t)djj << 8 | (uint32_t)gh << 16;
             if (!odd && (c.info & kInfoTable)) {
                 const Even48Idx ix = even48_indices(S, c.cls, c.p);
                 rec.x = enq ? __ldg(tabC + (S.c_offs[c.cls] & 0x7FFFFu) + ix.pC) : 0u;
@@ -142,11 +201,6 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
             } else {
                 rec.x = (uint32_t)c.p;
                 rec.y = (uint32_t)c.cls | c.r << 9 | (uint32_t)(c.p >> 32) << 21;
-            }
-            if (!enq) {                                       // zero A entry and gain
-                const uint32_t z[6] = {0x0u, 0x0u, 0x0u, 0x0u, 0x0u, 0x0u};
-                tc48_store_a(T, dr, djj, z);
-                T.gain[djj][dr] = 0.f;
             }
             const unsigned mo = __ballot_sync(0xFFFFFFFFu, enq && odd);
             const unsigned me = __ballot_sync(0xFFFFFFFFu, enq && !odd);
@@ -159,22 +213,31 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
                 T.list[pos] = rec;
             }
         }
-        // the next round's word loads while this round decodes
-        wcur = 0ull;
-        if (ch + 1 < c1 && row < rows && j0 + kTc48Slots + djj < nb)
-            wcur = __ldg(words + (long long)row * pitch + j0 + kTc48Slots + djj);
-        // ---- B tiles: block-diagonal activations, 3 x 16 B per (slot, batch column)
-        if (tid < 2 * kTcBlocks * 16 * 3) {
-            const int half = tid / (kTcBlocks * 16 * 3), u = tid % (kTcBlocks * 16 * 3);
-            const int q = u % 3, nidx = u / 3;                // n = 16 slot + b
-            const int jj = nidx >> 4, b = nidx & 15;
-            const int j = j0 + 4 * half + jj;
-            uint4 val = make_uint4(0, 0, 0, 0);
-            if (b < batch && j < nb) val = __ldg(reinterpret_cast<const uint4 *>(X + b * K + (long long)j * 24 + 8 * q));
-            *reinterpret_cast<uint4 *>(T.B[half] + (3 * jj + q) * kTcBLbo + nidx * 16) = val;
+        // the next round's word and gain load while this round decodes
+        if (ch + 1 < c1) {
+            wcur = load_word(ch + 1);
+            gcur = load_gain(ch + 1);
         }
         __syncthreads();
-        // ---- 2. decode the lists into A (odd-numbered warps start on the even list)
+        const uint4 xnow = load_x(ch);                          // L2-resident; lands during the wait
+        // ---- 2. the previous round's products: bounded wait, then the epilogue
+        if (ch > c0) {
+            if (tc48_wait_mma(T, phase)) {
+                tc_fence_after();
+                tc48_epilogue(etaddr, gep, yacc);
+            } else if (lane == 0) {
+                atomicOr(&T.status, 1u);
+            }
+            phase ^= 1u;
+        }
+        // ---- 3. this round's A and B tiles (the MMAs that read them have completed)
+        if (zero_a) {
+            const uint32_t z[6] = {0x0u, 0x0u, 0x0u, 0x0u, 0x0u, 0x0u};
+            tc48_store_a(T, dr, djj, z);
+            T.gain[djj][dr] = 0.f;
+        }
+        if (xrole) *reinterpret_cast<uint4 *>(T.B[xhalf] + (3 * xjj + xq) * kTcBLbo + xn * 16) = xnow;
+        // decode the lists into A (odd-numbered warps start on the even list)
         const int first = warp & 1;
         for (int pass = 0; pass < 2; pass++) {
             const int list_id = first ^ pass;
@@ -197,19 +260,18 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
                         even48_merge(S, E, info, S.c_info2[cls], r, s, E.tabS[(S.c_offs[cls] >> 19) + (e.y >> 21)],
                                      e.x, v);
                     else arrange48_rare(S, cls, info, p, r, s, v);
-                    const int rr = (int)(e.w & 0xFFu), jj = (int)(e.w >> 8);
+                    const int rr = (int)(e.w & 0xFFu), jj = (int)((e.w >> 8) & 0xFFu);
                     tc48_store_a(T, rr, jj, v);
-                    const long long grow = (long long)row0 + rr;
-                    T.gain[jj][rr] = gain_mode == 0
-                                         ? __half2float(__ldg(gains + grow * nb + j0 + jj))
-                                         : __half2float(__ldg(gains + grow * 256 + (e.z >> 24))) * S.invnorm[info_m(info)];
+                    const float g = __half2float(__ushort_as_half((unsigned short)(e.w >> 16)));
+                    T.gain[jj][rr] = gain_mode == 0 ? g : g * S.invnorm[info_m(info)];
                 }
             }
         }
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");   // generic writes -> MMA reads
         tc_fence_before();
         __syncthreads();
-        // ---- 3. one thread issues 2 x 6 MMA steps and commits them to the barrier
+        if (T.status) break;                                   // uniform: set only before the barrier
+        // ---- 4. one thread issues 2 x 6 MMA steps and commits them to the barrier
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
@@ -229,28 +291,17 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          ::"r"(smem_u32(&T.mbar_mma)) : "memory");
         }
-        // ---- 4. bounded wait for the MMAs, then this warp's 32 rows x 16 columns
-        {
-            bool done = false;
-            for (int it = 0; it < (1 << 20) && !done; it++) done = mbar_try_wait_parity(smem_u32(&T.mbar_mma), phase);
-            if (!done) atomicOr(&T.status, 1u);
+    }
+    // ---- the last round's products (T.status is uniform here: nothing wrote it since the
+    // last barrier)
+    if (c0 < c1 && !T.status) {
+        const float gep = T.gain[eslot][em];
+        if (tc48_wait_mma(T, phase)) {
+            tc_fence_after();
+            tc48_epilogue(etaddr, gep, yacc);
+        } else if (lane == 0) {
+            atomicOr(&T.status, 1u);
         }
-        phase ^= 1u;
-        __syncthreads();
-        if (T.status) break;                                   // uniform: read after the barrier
-        tc_fence_after();
-        uint32_t d[16];
-        asm volatile(
-            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-            : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3]), "=r"(d[4]), "=r"(d[5]), "=r"(d[6]), "=r"(d[7]),
-              "=r"(d[8]), "=r"(d[9]), "=r"(d[10]), "=r"(d[11]), "=r"(d[12]), "=r"(d[13]), "=r"(d[14]), "=r"(d[15])
-            : "r"(tmem + ((uint32_t)(lg * 32) << 16) + (uint32_t)(eslot * 16)));
-        asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-        const float g = T.gain[eslot][em];
-#pragma unroll
-        for (int b = 0; b < 16; b++) yacc[b] = fmaf(g, __uint_as_float(d[b]), yacc[b]);
-        tc_fence_before();
-        __syncthreads();                                       // A, B, gains and TMEM free
     }
     // ---- sum the 8 slots of each row (in the A tiles, free now) and add the row sums into y
     __syncthreads();
