@@ -476,6 +476,7 @@ struct ora_codec {
     int64_t ncls[MAXM + 1];          /* classes per shell (-1: not built) */
     ocls *cls[MAXM + 1];
     int store_all;                   /* 1: keep every shell's class list */
+    int cached;                      /* store_all = 0: the one shell kept after its use (-1: none) */
 };
 
 typedef struct { ocls *v; int64_t n, cap; u128 next; } clist;
@@ -506,12 +507,16 @@ static int build_shell(ora_codec *c, int m) {
     return 0;
 }
 
+/* Budgets with shells built on demand keep the shell used last, so that indices of one shell
+ * in a row build its class list once. */
 static void drop_shell(ora_codec *c, int m) {
-    if (!c->store_all && c->ncls[m] >= 0) {
-        free(c->cls[m]);
-        c->cls[m] = NULL;
-        c->ncls[m] = -1;
+    if (c->store_all || c->ncls[m] < 0) return;
+    if (c->cached >= 0 && c->cached != m) {
+        free(c->cls[c->cached]);
+        c->cls[c->cached] = NULL;
+        c->ncls[c->cached] = -1;
     }
+    c->cached = m;
 }
 
 ora_codec *ora_codec_create(int32_t index_bits) {
@@ -525,6 +530,7 @@ ora_codec *ora_codec_create(int32_t index_bits) {
     ora_golay_by_weight(c->golay_weight, c->wbase);
     for (int i = 0; i < 4096; i++) c->nk[popcount24(c->golay_mask[i])]++;
     for (int m = 0; m <= MAXM; m++) c->ncls[m] = -1;
+    c->cached = -1;
 
     /* shell sizes far enough to pass 2^index_bits (M = 13, 53, 214 for 48, 72, 96 bits) */
     int mbound = index_bits == 48 ? 20 : (index_bits == 72 ? 64 : 230);
@@ -790,14 +796,25 @@ int ora_encode(ora_codec *c, const int32_t x[ORA_DIM], uint64_t *lo, uint64_t *h
     return 0;
 }
 
-int64_t ora_decode_batch_shell(ora_codec *c, int64_t n, const uint64_t *lo, const uint64_t *hi,
-                               int8_t *out, int32_t *shell) {
+/* Decodes in ascending index order (the results land at their original positions), so a
+ * budget with shells built on demand builds each shell once. */
+typedef struct { u128 I; int64_t pos; } idx_pos;
+static int cmp_idx_pos(const void *a, const void *b) {
+    const u128 x = ((const idx_pos *)a)->I, y = ((const idx_pos *)b)->I;
+    return x < y ? -1 : (x > y ? 1 : 0);
+}
+
+static int64_t decode_sorted(ora_codec *c, int64_t n, const u128 *idx, int8_t *out, int32_t *shell) {
+    idx_pos *o = malloc((size_t)(n > 0 ? n : 1) * sizeof(idx_pos));
+    if (!o) return -1;
+    for (int64_t t = 0; t < n; t++) { o[t].I = idx[t]; o[t].pos = t; }
+    if (!c->store_all) qsort(o, (size_t)n, sizeof(idx_pos), cmp_idx_pos);
     int64_t bad = 0;
-    for (int64_t t = 0; t < n; t++) {
+    for (int64_t u = 0; u < n; u++) {
         int32_t x[ORA_DIM];
         int m = 0;
-        u128 I = mk128(lo[t], hi ? hi[t] : 0);
-        if (decode_one(c, I, x, &m)) {
+        const int64_t t = o[u].pos;
+        if (decode_one(c, o[u].I, x, &m)) {
             memset(x, 0, sizeof x);
             m = 0;
             bad++;
@@ -805,6 +822,17 @@ int64_t ora_decode_batch_shell(ora_codec *c, int64_t n, const uint64_t *lo, cons
         for (int i = 0; i < ORA_DIM; i++) out[t * ORA_DIM + i] = (int8_t)x[i];
         if (shell) shell[t] = m;
     }
+    free(o);
+    return bad;
+}
+
+int64_t ora_decode_batch_shell(ora_codec *c, int64_t n, const uint64_t *lo, const uint64_t *hi,
+                               int8_t *out, int32_t *shell) {
+    u128 *idx = malloc((size_t)(n > 0 ? n : 1) * sizeof(u128));
+    if (!idx) return -1;
+    for (int64_t t = 0; t < n; t++) idx[t] = mk128(lo[t], hi ? hi[t] : 0);
+    const int64_t bad = decode_sorted(c, n, idx, out, shell);
+    free(idx);
     return bad;
 }
 
@@ -848,6 +876,8 @@ typedef struct {
     double *y;
     int32_t r0, r1;
     int64_t bad;
+    const int8_t *vecs;            /* on-demand budgets: every block decoded beforehand */
+    const int32_t *shells;         /* (shell 0 = bad index) */
 } gemm_job;
 
 static void gemm_rows(gemm_job *J) {
@@ -863,7 +893,15 @@ static void gemm_rows(gemm_job *J) {
             unpack_word(W + ((int64_t)r * J->pitch + j) * J->word_bytes, J->word_bytes, c->bits, &I,
                         &code);
             int32_t v[ORA_DIM];
-            if (decode_one(c, I, v, &m)) { J->bad++; continue; }
+            if (J->vecs) {
+                const int64_t blk = (int64_t)r * J->nb + j;
+                m = J->shells[blk];
+                if (m == 0) { J->bad++; continue; }
+                for (int t = 0; t < ORA_DIM; t++) v[t] = J->vecs[blk * ORA_DIM + t];
+            } else if (decode_one(c, I, v, &m)) {
+                J->bad++;
+                continue;
+            }
             double scale;
             if (J->gain_mode == 0) scale = ora_half_to_double(J->gains[(int64_t)r * J->nb + j]);
             else scale = ora_half_to_double(J->gains[(int64_t)r * 256 + code]) / (4.0 * sqrt((double)m));
@@ -877,13 +915,41 @@ static void gemm_rows(gemm_job *J) {
     }
 }
 
+/* On-demand budgets (96 bits): decode every block first, in ascending index order. */
+static int predecode(ora_codec *c, int32_t rows, int32_t nb, const void *words, int32_t word_bytes,
+                     int64_t pitch, int8_t **vecs, int32_t **shells) {
+    const int64_t n = (int64_t)rows * nb;
+    u128 *idx = malloc((size_t)(n > 0 ? n : 1) * sizeof(u128));
+    *vecs = malloc((size_t)(n > 0 ? n : 1) * ORA_DIM);
+    *shells = malloc((size_t)(n > 0 ? n : 1) * sizeof(int32_t));
+    if (!idx || !*vecs || !*shells) { free(idx); return -1; }
+    for (int32_t r = 0; r < rows; r++)
+        for (int32_t j = 0; j < nb; j++) {
+            int code;
+            unpack_word((const uint8_t *)words + ((int64_t)r * pitch + j) * word_bytes, word_bytes, c->bits,
+                        &idx[(int64_t)r * nb + j], &code);
+        }
+    decode_sorted(c, n, idx, *vecs, *shells);
+    free(idx);
+    return 0;
+}
+
 int64_t ora_gemm(ora_codec *c, int32_t rows, int32_t nb, const void *words, int32_t word_bytes,
                  int64_t row_pitch_words, int32_t gain_mode, const uint16_t *gains,
                  const uint16_t *x, int32_t batch, double *y) {
     if ((c->bits == 48) != (word_bytes == 8)) return -1;
     gemm_job J = {c, rows, nb, word_bytes, gain_mode, batch, words, row_pitch_words, gains, x, y,
-                  0, rows, 0};
+                  0, rows, 0, NULL, NULL};
+    int8_t *vecs = NULL;
+    int32_t *shells = NULL;
+    if (!c->store_all) {
+        if (predecode(c, rows, nb, words, word_bytes, row_pitch_words, &vecs, &shells)) return -1;
+        J.vecs = vecs;
+        J.shells = shells;
+    }
     gemm_rows(&J);
+    free(vecs);
+    free(shells);
     return J.bad;
 }
 
@@ -894,14 +960,17 @@ int64_t ora_gemm_mt(const ora_codec *c, int32_t rows, int32_t nb, const void *wo
                     const uint16_t *gains, const uint16_t *x, int32_t batch, double *y,
                     int32_t nthreads) {
     if ((c->bits == 48) != (word_bytes == 8)) return -1;
-    if (!c->store_all) nthreads = 1;     /* on-demand shell lists are not shared safely */
+    if (!c->store_all)                   /* on-demand shell lists are not shared safely */
+        return ora_gemm((ora_codec *)c, rows, nb, words, word_bytes, row_pitch_words, gain_mode, gains, x,
+                        batch, y);
     if (nthreads < 1) nthreads = 1;
     if (nthreads > rows) nthreads = rows > 0 ? rows : 1;
     gemm_job *jobs = calloc((size_t)nthreads, sizeof(gemm_job));
     pthread_t *th = calloc((size_t)nthreads, sizeof(pthread_t));
     for (int t = 0; t < nthreads; t++) {
         gemm_job J = {c, rows, nb, word_bytes, gain_mode, batch, words, row_pitch_words, gains, x, y,
-                      (int32_t)((int64_t)rows * t / nthreads), (int32_t)((int64_t)rows * (t + 1) / nthreads), 0};
+                      (int32_t)((int64_t)rows * t / nthreads), (int32_t)((int64_t)rows * (t + 1) / nthreads), 0,
+                      NULL, NULL};
         jobs[t] = J;
         pthread_create(&th[t], NULL, gemm_thread, &jobs[t]);
     }
