@@ -29,9 +29,16 @@ class llvq_weight(C.Structure):
                 ("row_pitch_words", C.c_int64), ("words", C.c_void_p), ("gains", C.c_void_p)]
 
 
+class llvq_class96(C.Structure):
+    _fields_ = [("start_lo", C.c_uint64), ("start_hi", C.c_uint32), ("meta", C.c_uint32),
+                ("rcp_lo", C.c_uint64), ("rcp_hi", C.c_uint64), ("cum", C.c_uint32 * 4),
+                ("vals", C.c_uint32 * 4)]
+
+
 class LLVQError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {llvq_status_string(status)} ({status})")
+        msg = lib().llvq_last_error_message().decode()
+        super().__init__(f"{what}: {llvq_status_string(status)} ({status})" + (f": {msg}" if msg else ""))
         self.status = status
 
 
@@ -57,8 +64,11 @@ def lib() -> C.CDLL:
                                            C.c_void_p, C.c_void_p]
         L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
         L.llvq_decode_noalloc.argtypes = [C.c_int32, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
+        L.llvq_last_error_message.argtypes = []
+        L.llvq_last_error_message.restype = C.c_char_p
+        L.llvq_class_table96.argtypes = [C.c_int32, C.c_void_p, C.c_int64, C.POINTER(C.c_int64)]
         for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
-                  "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc"):
+                  "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc", "llvq_class_table96"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -66,7 +76,7 @@ def lib() -> C.CDLL:
 
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
             "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
-            "llvq_decode_noalloc")
+            "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message")
 
 
 def llvq_status_string(status: int) -> str:
@@ -79,6 +89,21 @@ def llvq_decode_noalloc(words, out, n: int | None = None, stream=None):
     n = out.shape[0] if n is None else n
     _check(lib().llvq_decode_noalloc(48, C.c_void_p(words.data_ptr()), 8, n, C.c_void_p(out.data_ptr()),
                                      _stream(stream)), "llvq_decode_noalloc")
+
+
+def class_table96(m: int):
+    """Host-side 96-bit class records of shell m (no device needed), as a numpy structured array
+    with the fields of llvq_class96 (include/llvq.h)."""
+    import numpy as np
+    n = C.c_int64()
+    _check(lib().llvq_class_table96(m, None, 0, C.byref(n)), f"llvq_class_table96({m})")
+    dt = np.dtype([("start_lo", "<u8"), ("start_hi", "<u4"), ("meta", "<u4"), ("rcp_lo", "<u8"),
+                   ("rcp_hi", "<u8"), ("cum", "u1", 16), ("vals", "u1", 16)])
+    assert dt.itemsize == C.sizeof(llvq_class96) == 64
+    out = np.zeros(n.value, dt)
+    _check(lib().llvq_class_table96(m, out.ctypes.data_as(C.c_void_p), n.value, C.byref(n)),
+           f"llvq_class_table96({m})")
+    return out
 
 
 def _check(status: int, what: str):
@@ -94,7 +119,7 @@ def _stream(stream) -> C.c_void_p:
 
 
 class Codec:
-    """Decode tables of one index budget (48 or 72 bits) on the current CUDA device."""
+    """Decode tables of one index budget (48, 72 or 96 bits) on the current CUDA device."""
 
     def __init__(self, index_bits: int = 48):
         h = C.c_void_p()

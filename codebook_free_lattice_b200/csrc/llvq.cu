@@ -1,13 +1,17 @@
-// llvq.cu -- host side of libllvq: decode-table images for the 48- and 72-bit index budgets,
-// kernel launches, and the C ABI declared in include/llvq.h.  Kernels: kernels.cuh; decoders:
-// codec48.cuh, codec72.cuh; host table construction: tables.cpp.
+// llvq.cu -- host side of libllvq: decode-table images for the 48-, 72- and 96-bit index
+// budgets, kernel launches, and the C ABI declared in include/llvq.h.  Kernels: kernels.cuh;
+// decoders: codec48.cuh, codec72.cuh, codec96.cuh; host table construction: tables.cpp,
+// tables96.cpp.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
 #include <map>
+#include <memory>
 #include <mutex>
 #include <string>
+#include <thread>
 #include <type_traits>
 #include <utility>
 #include <vector>
@@ -17,7 +21,9 @@
 #include "kernels_bin48.cuh"
 #include "kernels_tc.cuh"
 #include "kernels_tc48.cuh"
+#include "codec96.cuh"
 #include "tables.h"
+#include "tables96.h"
 
 using namespace llvq;
 
@@ -31,6 +37,8 @@ struct llvq_codec {
     void *d_image = nullptr;       // Smem48 / Smem72 image (copied to shared memory per CTA)
     Rec72 *d_recs72 = nullptr;     // 72-bit class records (global memory)
     uint32_t *d_guide72 = nullptr; // 72-bit guide table
+    Rec96 *d_recs96 = nullptr;     // 96-bit class records (global memory)
+    uint32_t *d_guide96 = nullptr; // 96-bit guide table (top 28 index bits)
     void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
     unsigned *d_flags = nullptr;   // sticky device flags
@@ -267,6 +275,95 @@ Dec72::Args args72(const llvq_codec *c) {
                        (unsigned long long)c->npoints, (unsigned long long)(c->npoints >> 64)};
 }
 
+Dec96::Args args96(const llvq_codec *c) {
+    return Dec96::Args{(const Smem96 *)c->d_image, c->d_recs96, c->d_guide96, (unsigned long long)c->npoints,
+                       (uint32_t)(c->npoints >> 64)};
+}
+
+// guide[b] = the class holding index b 2^68 (the last class whose start is <= b 2^68)
+__global__ void k_guide96(const Rec96 *__restrict__ recs, long long ncls, uint32_t *__restrict__ guide, long long nb) {
+    const long long b = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (b >= nb) return;
+    const unsigned long long thi = (unsigned long long)b << (kGuideShift96 - 64);
+    if (thi > 0xFFFFFFFFull) { guide[b] = (uint32_t)(ncls - 1); return; }
+    long long lo = 0, hi = ncls - 1;
+    while (lo < hi) {
+        const long long mid = (lo + hi + 1) >> 1;
+        const uint32_t sh = recs[mid].start_hi;
+        const bool le = sh < (uint32_t)thi || (sh == (uint32_t)thi && recs[mid].start_lo == 0ull);
+        if (le) lo = mid; else hi = mid - 1;
+    }
+    guide[b] = (uint32_t)lo;
+}
+
+// The 96-bit tables: shell sizes and class counts on the host, then the class records shell by
+// shell on the host threads, each shell copied to its place in the device table, then the guide
+// on the device.
+llvq_status create96(llvq_codec *c, std::vector<unsigned char> &image, std::string &err) {
+    Tables96 T;
+    const int hw = std::max(1, (int)std::thread::hardware_concurrency());
+    if (!build_tables96(T, hw, err)) return LLVQ_ERR_UNSUPPORTED;
+    c->M = T.M;
+    c->npoints = T.n_points;
+    c->nclasses = T.n_classes;
+    image.assign(sizeof(Smem96), 0);
+    Smem96 &S = *reinterpret_cast<Smem96 *>(image.data());
+    std::memcpy(S.golay_mask, T.golay_by_mask, sizeof S.golay_mask);
+    std::memcpy(S.golay_weight, T.golay_by_weight, sizeof S.golay_weight);
+    for (int d = 2; d < 32; d++) S.mc[d] = (unsigned long long)((((u128)1 << 64) + d - 1) / d);
+    for (int k = 0; k <= 24; k++) {
+        S.nwords[k] = (uint16_t)T.words_of_weight[k];
+        S.wbase[k] = (uint16_t)T.weight_base[k];
+        const int A = T.words_of_weight[k];
+        if (A >= 2) S.mA[k] = (unsigned long long)((((u128)1 << 64) + A - 1) / A);
+    }
+    S.nwords[25] = 4096;
+    S.mA[25] = 1ull << 52;
+    fill_pdep(S.pdep_off, S.pdep);
+    if (T.M > 255) { err = "96-bit shell bound above the table"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int m = 1; m <= T.M; m++) S.invnorm[m] = (float)(1.0 / (4.0 * std::sqrt((double)m)));
+    const long long nb = (long long)((T.n_points - 1) >> kGuideShift96) + 2;
+    if (cudaMalloc(&c->d_recs96, (size_t)T.n_classes * sizeof(Rec96)) != cudaSuccess ||
+        cudaMalloc(&c->d_guide96, (size_t)nb * sizeof(uint32_t)) != cudaSuccess) {
+        err = "device memory for the 96-bit class table (" +
+              std::to_string((size_t)T.n_classes * sizeof(Rec96) + (size_t)nb * 4) + " bytes) not available";
+        cudaGetLastError();
+        return LLVQ_ERR_CUDA;
+    }
+    // fill threads hold one shell each (up to 0.6 GB of records)
+    const int nfill = std::min(hw, 8);
+    std::atomic<int> next(0);
+    std::atomic<bool> failed(false);
+    std::mutex emu;
+    std::vector<std::thread> pool;
+    for (int th = 0; th < nfill; th++)
+        pool.emplace_back([&]() {
+            if (cudaSetDevice(c->device) != cudaSuccess) { failed = true; return; }
+            std::vector<Rec96> buf;
+            std::string e;
+            while (!failed) {
+                const int m = T.M - next.fetch_add(1);
+                if (m < 2) break;
+                buf.resize((size_t)T.shell_classes[m]);
+                if (!fill_shell96(T, m, buf.data(), e) ||
+                    cudaMemcpy(c->d_recs96 + T.class_base[m], buf.data(), buf.size() * sizeof(Rec96),
+                               cudaMemcpyHostToDevice) != cudaSuccess) {
+                    std::lock_guard<std::mutex> g(emu);
+                    if (!failed) err = e.empty() ? "copy of the 96-bit class records failed" : e;
+                    failed = true;
+                }
+            }
+        });
+    for (auto &t : pool) t.join();
+    if (failed) return LLVQ_ERR_UNSUPPORTED;
+    k_guide96<<<(unsigned)((nb + 255) / 256), 256>>>(c->d_recs96, T.n_classes, c->d_guide96, nb);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        err = "96-bit guide construction failed";
+        return LLVQ_ERR_CUDA;
+    }
+    return LLVQ_OK;
+}
+
 template <class D>
 cudaError_t launch_decode(const llvq_codec *c, typename D::Args a, const void *words, long long n,
                           int8_t *out, cudaStream_t st) {
@@ -492,6 +589,52 @@ llvq_status noalloc_setup(int dev, unsigned char **out) {
     *out = ptr;
     return LLVQ_OK;
 }
+void set_kernel_attrs() {
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
+        cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
+        set_bin48_attrs(std::make_integer_sequence<int, 7>{});
+        cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
+        cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
+        set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
+        cudaFuncSetAttribute(k_decode<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem96));
+        cudaFuncSetAttribute(k_gemm_tc<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec96>));
+        set_gemm_attrs<Dec96>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
+    });
+}
+
+llvq_status codec_create96(llvq_codec **out) {
+    llvq_codec *c = new llvq_codec;
+    c->index_bits = 96;
+    std::vector<unsigned char> image;
+    std::string err;
+    llvq_status st = LLVQ_OK;
+    if (cudaGetDevice(&c->device) != cudaSuccess ||
+        cudaDeviceGetAttribute(&c->num_sms, cudaDevAttrMultiProcessorCount, c->device) != cudaSuccess) {
+        err = "no CUDA device";
+        st = LLVQ_ERR_CUDA;
+    }
+    if (st == LLVQ_OK) st = create96(c, image, err);
+    if (st == LLVQ_OK &&
+        !(cudaMalloc(&c->d_image, image.size()) == cudaSuccess &&
+          cudaMemcpy(c->d_image, image.data(), image.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+          cudaMalloc(&c->d_flags, sizeof(unsigned)) == cudaSuccess &&
+          cudaMemset(c->d_flags, 0, sizeof(unsigned)) == cudaSuccess)) {
+        err = "device allocation for the 96-bit codec failed";
+        st = LLVQ_ERR_CUDA;
+    }
+    if (st != LLVQ_OK) {
+        cudaGetLastError();
+        g_last_error = err;
+        llvq_codec_destroy(c);
+        return st;
+    }
+    set_kernel_attrs();
+    *out = c;
+    return LLVQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -525,6 +668,37 @@ llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t
 }
 
 
+const char *llvq_last_error_message(void) { return g_last_error.c_str(); }
+
+llvq_status llvq_class_table96(int32_t m, llvq_class96 *out, int64_t capacity, int64_t *n_classes) {
+    static_assert(sizeof(llvq_class96) == sizeof(Rec96), "llvq_class96 mirrors Rec96");
+    static std::mutex mu;
+    static std::unique_ptr<Tables96> tables;
+    std::lock_guard<std::mutex> g(mu);
+    if (!tables) {
+        auto t = std::make_unique<Tables96>();
+        std::string err;
+        if (!build_tables96(*t, std::max(1, (int)std::thread::hardware_concurrency()), err)) {
+            g_last_error = err;
+            return LLVQ_ERR_UNSUPPORTED;
+        }
+        tables = std::move(t);
+    }
+    if (m < 2 || m > tables->M) return LLVQ_ERR_ARG;
+    const int64_t n = tables->shell_classes[m];
+    if (n_classes) *n_classes = n;
+    if (!out) return LLVQ_OK;
+    if (capacity < n) return LLVQ_ERR_ARG;
+    std::vector<Rec96> buf((size_t)n);
+    std::string err;
+    if (!fill_shell96(*tables, m, buf.data(), err)) {
+        g_last_error = err;
+        return LLVQ_ERR_UNSUPPORTED;
+    }
+    std::memcpy(out, buf.data(), buf.size() * sizeof(Rec96));
+    return LLVQ_OK;
+}
+
 const char *llvq_status_string(llvq_status s) {
     switch (s) {
         case LLVQ_OK: return "ok";
@@ -539,7 +713,8 @@ const char *llvq_status_string(llvq_status s) {
 llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     if (!out) return LLVQ_ERR_ARG;
     *out = nullptr;
-    if (index_bits != 48 && index_bits != 72) return LLVQ_ERR_UNSUPPORTED;
+    if (index_bits != 48 && index_bits != 72 && index_bits != 96) return LLVQ_ERR_UNSUPPORTED;
+    if (index_bits == 96) return codec_create96(out);
     HostTables T;
     std::string err;
     if (!build_host_tables(index_bits, T, err)) { g_last_error = err; return LLVQ_ERR_UNSUPPORTED; }
@@ -587,15 +762,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
         llvq_codec_destroy(c);
         return LLVQ_ERR_CUDA;
     }
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
-        cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
-        set_bin48_attrs(std::make_integer_sequence<int, 7>{});
-        cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
-        cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
-        set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
-    });
+    set_kernel_attrs();
     *out = c;
     return LLVQ_OK;
 }
@@ -605,6 +772,8 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_image) cudaFree(c->d_image);
     if (c->d_recs72) cudaFree(c->d_recs72);
     if (c->d_guide72) cudaFree(c->d_guide72);
+    if (c->d_recs96) cudaFree(c->d_recs96);
+    if (c->d_guide96) cudaFree(c->d_guide96);
     if (c->d_flags) cudaFree(c->d_flags);
     if (c->d_even48) cudaFree(c->d_even48);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
@@ -629,8 +798,9 @@ llvq_status llvq_decode(const llvq_codec *c, const void *d_words, int32_t word_b
     if (word_bytes != (c->index_bits == 48 ? 8 : 16)) return LLVQ_ERR_ARG;
     if (!aligned(d_words, (size_t)word_bytes) || !aligned(d_out, 8)) return LLVQ_ERR_ARG;
     cudaStream_t st = (cudaStream_t)stream;
-    const cudaError_t e = c->index_bits == 48 ? launch_decode<Dec48>(c, args48(c), d_words, n, d_out, st)
-                                              : launch_decode<Dec72>(c, args72(c), d_words, n, d_out, st);
+    const cudaError_t e = c->index_bits == 48   ? launch_decode<Dec48>(c, args48(c), d_words, n, d_out, st)
+                          : c->index_bits == 72 ? launch_decode<Dec72>(c, args72(c), d_words, n, d_out, st)
+                                                : launch_decode<Dec96>(c, args96(c), d_words, n, d_out, st);
     return e == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 
@@ -643,8 +813,9 @@ llvq_status llvq_gemm_smallbatch(const llvq_codec *c, const llvq_weight *w, cons
     if (!aligned(d_X, 16) || !aligned(d_Y, 4)) return LLVQ_ERR_ARG;
     if (w->rows == 0) return LLVQ_OK;
     cudaStream_t s = (cudaStream_t)stream;
-    const cudaError_t e = c->index_bits == 48 ? gemm_dispatch<Dec48>(c, args48(c), w, d_X, batch, d_Y, s)
-                                              : gemm_dispatch<Dec72>(c, args72(c), w, d_X, batch, d_Y, s);
+    const cudaError_t e = c->index_bits == 48   ? gemm_dispatch<Dec48>(c, args48(c), w, d_X, batch, d_Y, s)
+                          : c->index_bits == 72 ? gemm_dispatch<Dec72>(c, args72(c), w, d_X, batch, d_Y, s)
+                                                : gemm_dispatch<Dec96>(c, args96(c), w, d_X, batch, d_Y, s);
     return e == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 

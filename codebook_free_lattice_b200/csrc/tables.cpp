@@ -5,9 +5,6 @@
 #include <cmath>
 
 namespace llvq {
-namespace {
-
-int popc24(uint32_t w) { return __builtin_popcount(w & 0xFFFFFFu); }
 
 // Extended Golay code: every multiple a(x) g(x), deg a < 12, of the generator polynomial
 // g(x) = 1 + x^2 + x^4 + x^5 + x^6 + x^10 + x^11 of the cyclic [23,12] code (carry-less
@@ -18,9 +15,13 @@ void golay_code(uint32_t words[4096]) {
         uint32_t prod = 0;
         for (int i = 0; i < 12; i++)
             if (a >> i & 1u) prod ^= g << i;
-        words[a] = prod | ((uint32_t)(popc24(prod) & 1) << 23);
+        words[a] = prod | ((uint32_t)(__builtin_popcount(prod & 0xFFFFFFu) & 1) << 23);
     }
 }
+
+namespace {
+
+int popc24(uint32_t w) { return __builtin_popcount(w & 0xFFFFFFu); }
 
 u128 factorial(int n) {
     u128 f = 1;

@@ -44,6 +44,9 @@ struct HostTables {
     int weight_base[25];                 // first by-weight slot of each weight
 };
 
+// The 4096 codewords of the extended binary Golay code (24-bit masks), in message order.
+void golay_code(uint32_t words[4096]);
+
 // index_bits 48 or 72.  Returns false and sets err on failure.
 bool build_host_tables(int index_bits, HostTables &out, std::string &err);
 

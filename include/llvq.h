@@ -64,6 +64,7 @@ typedef struct llvq_codec llvq_codec;
  * words: device, [rows][row_pitch_words] packed words of word_bytes bytes (row-major).
  *   word_bytes 8  (index_bits 48): bits [0,48) index, [48,56) gain code, [56,64) zero.
  *   word_bytes 16 (index_bits 72): little-endian; bits [0,72) index, [72,80) gain code.
+ *   word_bytes 16 (index_bits 96): little-endian; bits [0,96) index, [96,104) gain code.
  * Block j of row r covers columns [24 j, 24 j + 24); cols beyond the logical width are
  * padding, and the activations must be zero there.  Alignment: words 8-byte (16-byte for
  * 16-byte words) aligned, gains 2-byte aligned. */
@@ -71,18 +72,22 @@ typedef struct {
     int32_t rows;              /* M */
     int32_t cols;              /* K (logical); blocks_per_row = ceil(K / 24) */
     int32_t blocks_per_row;    /* nb */
-    int32_t index_bits;        /* 48 or 72; must equal the codec's */
-    int32_t word_bytes;        /* 8 for 48-bit, 16 for 72-bit */
+    int32_t index_bits;        /* 48, 72 or 96; must equal the codec's */
+    int32_t word_bytes;        /* 8 for 48-bit, 16 for 72- and 96-bit */
     int32_t gain_mode;         /* llvq_gain_mode */
     int64_t row_pitch_words;   /* >= blocks_per_row */
     const void *words;         /* device */
     const void *gains;         /* device fp16 (see llvq_gain_mode) */
 } llvq_weight;
 
-/* Build the tables for an index budget (48 -> shells 2..13, 72 -> shells 2..53; 96 bits is
- * LLVQ_ERR_UNSUPPORTED) on the current device and upload them.  *out is owned by the caller
- * and released with llvq_codec_destroy.  Thread-safe to use from several streams afterwards
- * (the codec is read-only except for its sticky flag word). */
+/* Build the tables for an index budget (48 -> shells 2..13, 72 -> shells 2..53, 96 -> shells
+ * 2..214) on the current device and upload them.  *out is owned by the caller and released with
+ * llvq_codec_destroy.  Thread-safe to use from several streams afterwards (the codec is
+ * read-only except for its sticky flag word).
+ * 48 and 72 bits: tables of 76 KB / 11 MB, built in well under a second.  96 bits: 304,649,365
+ * class records of 64 bytes plus a 1 GB guide (about 20.5 GB of device memory), built on all host
+ * cores (several seconds; a few GB of host memory while it runs); LLVQ_ERR_CUDA when the device
+ * memory is not available, with the reason in llvq_last_error_message. */
 llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out);
 void llvq_codec_destroy(llvq_codec *codec);
 
@@ -126,12 +131,40 @@ llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, 
 llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t word_bytes, int64_t n,
                                 int8_t *d_out, void *stream);
 
+/* Host-side inspection of the 96-bit class table (no device needed): the class records of shell
+ * m (2 <= m <= 214) in index order, as the decoder reads them.  A class is one multiset of |x_i|
+ * in one coset; its magnitude groups form one list (even coset: the magnitudes 0 mod 4 ascending,
+ * then those 2 mod 4 ascending; odd coset: all ascending).  Fields:
+ *   start (start_lo, low 32 bits of start_hi): first global index of the class (< 2^96);
+ *   meta: bits 0..6 t = bitlen(P - 1) (P = arrangements of the class), 7..14 shell m,
+ *         15..19 k (even: codeword weight), 20..24 B (free sign bits), 25 odd coset,
+ *         26 parity target (even: sum|x|/4 mod 2);
+ *   rcp_lo/rcp_hi: ceil(2^(128 + t) / P) - 2^128;
+ *   cum: byte g = 0x7F + (number of coordinates in groups 0..g), 16 groups (unused: 0x7F + 24);
+ *   vals: byte g = magnitude of group g (unused: 0).
+ * out may be NULL (then only *n_classes is set); otherwise it holds capacity records and the call
+ * returns LLVQ_ERR_ARG when the shell has more.  The first call builds the shell sizes and class
+ * counts (a few seconds on all host cores) and keeps them for later calls. */
+typedef struct {
+    uint64_t start_lo;
+    uint32_t start_hi;
+    uint32_t meta;
+    uint64_t rcp_lo, rcp_hi;
+    uint32_t cum[4];
+    uint32_t vals[4];
+} llvq_class96;
+llvq_status llvq_class_table96(int32_t m, llvq_class96 *out, int64_t capacity, int64_t *n_classes);
+
 /* Synchronise `stream`, return the sticky device flags raised since the last call in *flags
  * and clear them.  Returns LLVQ_ERR_DEVICE_FLAG when any flag was set, LLVQ_OK otherwise. */
 llvq_status llvq_get_error(const llvq_codec *codec, void *stream, uint32_t *flags);
 
 /* Static string for a status code. */
 const char *llvq_status_string(llvq_status status);
+
+/* The reason of the last failed call on this thread that gave one (table construction, device
+ * memory), or an empty string.  Valid until the next call on this thread. */
+const char *llvq_last_error_message(void);
 
 #ifdef __cplusplus
 }

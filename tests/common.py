@@ -25,13 +25,18 @@ class Layer:
     """A synthetic compressed layer: words [rows, nb(, 2)], fp16 gains, fp16 activations."""
 
     def __init__(self, index_bits, rows, K, batch, config_id, n_points, gain_mode,
-                 index_limit=None, norms_fn=None, pitch=None):
+                 index_limit=None, norms_fn=None, pitch=None, index_base=0):
         self.index_bits, self.rows, self.K, self.batch = index_bits, rows, K, batch
         self.nb = -(-K // 24)
         self.pitch = self.nb if pitch is None else pitch
         self.gain_mode = gain_mode
         limit = n_points if index_limit is None else index_limit
-        lo, hi = synth.uniform_indices(synth.rng(config_id, 0), rows * self.pitch, limit, index_bits)
+        lo, hi = synth.uniform_indices(synth.rng(config_id, 0), rows * self.pitch, limit - index_base, index_bits)
+        if index_base:                          # uniform over [index_base, limit)
+            blo = np.uint64(index_base & (2**64 - 1))
+            lo2 = lo + blo
+            hi = hi + np.uint64(index_base >> 64) + (lo2 < lo).astype(np.uint64)
+            lo = lo2
         self.lo, self.hi = lo, hi
         codes = synth.gain_codes(synth.rng(config_id, 1), rows * self.pitch)
         self.codes = codes.reshape(rows, self.pitch)

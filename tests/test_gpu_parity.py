@@ -330,3 +330,103 @@ def test_gemm72_full_size_sampled_rows(gcodec72, ocodec72, rows, K, batch):
     rs = np.sort(np.random.default_rng(rows).choice(rows, 64, replace=False))
     ref = oracle_gemm(ocodec72, layer, rows=rs)
     assert max_rel_err(y[:, rs], ref) < GEMV_RTOL
+
+
+# ------------------------------------------------------------------ 96-bit budget ----------
+# The oracle builds the class list of a 96-bit shell on demand (up to 9.1M classes for shell
+# 214) and decodes in ascending index order, so the cases below draw their indices from a few
+# shells each.
+
+@pytest.fixture(scope="module")
+def gcodec96(dev):
+    import codebook_free_lattice_b200 as L
+    return L.Codec(96)
+
+
+@pytest.fixture(scope="module")
+def ocodec96():
+    return oracle.Codec(96)
+
+
+def split96(idx):
+    lo = np.array([i & (2**64 - 1) for i in idx], np.uint64)
+    hi = np.array([i >> 64 for i in idx], np.uint64)
+    return lo, hi
+
+
+def uniform_in_shells(ocodec, m0, m1, n, seed):
+    """n seeded indices uniform over shells m0..m1 (python ints)."""
+    a, b = ocodec.shell_offset(m0), ocodec.shell_offset(m1 + 1)
+    lo, hi = synth.uniform_indices(synth.rng(seed, 0), n, b - a, 96)
+    return [a + (int(h) << 64 | int(l)) for l, h in zip(lo, hi)]
+
+
+def test_codec96_info_matches_oracle(gcodec96, ocodec96):
+    assert gcodec96.max_shell == ocodec96.max_shell == 214
+    assert gcodec96.n_points == ocodec96.n_points == 74972166705387133681638419280
+    assert gcodec96.n_classes == 304649365
+
+
+def test_decode96_class_boundaries_and_shells(gcodec96, ocodec96):
+    """First, middle and last index of every class of shells 2..9 and of sampled classes of
+    shells 50, 120, 200 and 214; seeded uniform indices inside shells 3, 50, 120, 200 and 214;
+    the last coded index.  Gain-code bits must be ignored."""
+    idx = []
+    for m in range(2, 10):
+        for j in range(ocodec96.shell_nclasses(m)):
+            c = ocodec96.shell_class(m, j)
+            idx += [c.offset, c.offset + c.size // 2, c.offset + c.size - 1]
+    for m in (50, 120, 200, 214):
+        n = ocodec96.shell_nclasses(m)
+        for j in list(range(0, n, max(1, n // 150))) + [n - 1]:
+            c = ocodec96.shell_class(m, j)
+            idx += [c.offset, c.offset + c.size - 1]
+    for seed, m in enumerate((3, 50, 120, 200, 214)):
+        idx += uniform_in_shells(ocodec96, m, m, 400, 40 + seed)
+    idx.append(ocodec96.n_points - 1)
+    lo, hi = split96(idx)
+    codes = synth.gain_codes(synth.rng(45, 1), lo.shape[0])
+    got = gpu_decode(gcodec96, synth.pack_words(lo, hi, codes, 96))
+    assert np.array_equal(got, ocodec96.decode_batch(lo, hi))
+    assert gcodec96.get_error() == 0
+
+
+def test_decode96_top_shells_uniform(gcodec96, ocodec96):
+    """6000 seeded indices uniform over shells 205..214, which hold 38% of the index space."""
+    lo, hi = split96(uniform_in_shells(ocodec96, 205, 214, 6000, 46))
+    got = gpu_decode(gcodec96, synth.pack_words(lo, hi, None, 96))
+    assert np.array_equal(got, ocodec96.decode_batch(lo, hi))
+
+
+def test_decode96_out_of_range(gcodec96, ocodec96):
+    N = ocodec96.n_points
+    lo, hi = split96([0, N - 1, N, N + 7, 2**96 - 1, 5])
+    got = gpu_decode(gcodec96, synth.pack_words(lo, hi, None, 96))
+    assert gcodec96.get_error() == 1
+    assert np.array_equal(got, ocodec96.decode_batch(lo, hi))
+    assert (got[2:5] == 0).all()
+
+
+@pytest.mark.parametrize("batch,rows,K,gain_mode", [(1, 150, 24 * 33 + 7, 1), (3, 70, 24 * 20, 0),
+                                                    (16, 200, 24 * 13, 1)])
+def test_gemm96_low_shells(gcodec96, ocodec96, batch, rows, K, gain_mode):
+    """GEMV, CUDA-core batch 3 and tensor-core batch 16 on indices uniform over shells 2..60."""
+    limit = ocodec96.shell_offset(61)
+    norms = None
+    if gain_mode == 0:
+        def norms(lo, hi):
+            v = ocodec96.decode_batch(lo, hi).astype(np.float64)
+            return np.sqrt((v ** 2).sum(1))
+    layer = Layer(96, rows, K, batch, 50 + batch, ocodec96.n_points, gain_mode, index_limit=limit,
+                  norms_fn=norms)
+    y = run_gemm(gcodec96, layer)
+    assert max_rel_err(y, oracle_gemm(ocodec96, layer)) < GEMV_RTOL
+
+
+@pytest.mark.parametrize("batch", [1, 16])
+def test_gemm96_top_shells(gcodec96, ocodec96, batch):
+    """Products on indices uniform over shells 208..214 (u8 gain tables)."""
+    layer = Layer(96, 64, 24 * 40, batch, 60 + batch, ocodec96.n_points, 1,
+                  index_base=ocodec96.shell_offset(208))
+    y = run_gemm(gcodec96, layer)
+    assert max_rel_err(y, oracle_gemm(ocodec96, layer)) < GEMV_RTOL
