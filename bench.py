@@ -228,6 +228,11 @@ SWEEP_CASES = [
     ("28672x8192", 28672, 8192, 72, 16),
     ("8192x28672", 8192, 28672, 72, 1),
     ("8192x28672", 8192, 28672, 72, 8),
+    ("4096x4096", 4096, 4096, 96, 1),
+    ("28672x8192", 28672, 8192, 96, 1),
+    ("28672x8192", 28672, 8192, 96, 16),
+    ("8192x28672", 8192, 28672, 96, 1),
+    ("8192x28672", 8192, 28672, 96, 8),
 ]
 LLAMA7B_LAYER = [("q", 4096, 4096), ("k", 4096, 4096), ("v", 4096, 4096), ("o", 4096, 4096),
                  ("gate", 11008, 4096), ("up", 11008, 4096), ("down", 4096, 11008)]
@@ -282,12 +287,12 @@ def _run_layers(codec, layers, batch, stream):
 def sweep(torch, dev):
     """One JSON line per (layer, bits, batch): fused LLVQ product time against cuBLAS fp16
     (torch.matmul on identical shapes), inputs larger than L2 in both arms; then the full
-    Llama-2-7B-shaped decoder stack (32 layers x q,k,v,o,gate,up,down) at 2 and 3 bits."""
+    Llama-2-7B-shaped decoder stack (32 layers x q,k,v,o,gate,up,down) at 2, 3 and 4 bits."""
     import codebook_free_lattice_b200 as L
     peak, _ = measured_peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     stream = torch.cuda.Stream(device=dev)
-    codecs = {48: L.Codec(48), 72: L.Codec(72)}
+    codecs = {48: L.Codec(48), 72: L.Codec(72), 96: L.Codec(96)}
     for name, rows, K, bits, batch in SWEEP_CASES:
         codec = codecs[bits]
         nb = -(-K // 24)
@@ -308,7 +313,7 @@ def sweep(torch, dev):
                           "decoded_vectors_per_s": rows * nb / t, "cublas_fp16_us": tc * 1e6,
                           "speedup_vs_fp16": tc / t, "layer_copies": copies}), flush=True)
         torch.cuda.empty_cache()
-    for bits in (48, 72):
+    for bits in (48, 72, 96):
         codec = codecs[bits]
         shapes = [(r, k) for _ in range(32) for (_, r, k) in LLAMA7B_LAYER]
         layers = _layers(torch, codec, dev, shapes, bits, 1, 900 + bits)
