@@ -15,7 +15,10 @@
 //     slot = high word of phi * L and, for the group a holding the slot,
 //     phi <- floor(((slot - C_<a) 2^128 + low words) / c_a) + 1 by long division in 32-bit limbs.
 //     With e_i = (phi_i - 2^128 f_i) P_i / 2^128 (P_i = arrangements left), e_{i+1} <= e_i +
-//     P_{i+1} / 2^128, so e stays below 2^-40 over the 24 steps and every slot is exact;
+//     P_{i+1} / 2^128, so e stays below 2^-40 over the 24 steps and every slot is exact.
+//     Once every lane of the warp has P_i < 2^57 (a running upper bound on log2 P_i), the state
+//     narrows to its top 64 bits plus one and the steps continue in two limbs: the same bound in
+//     units of 2^-64 gives e <= 2^-7 + 24 * 2^-7 < 1.  The last step needs no new state;
 //   - an even class ranks its magnitudes off and on the codeword separately with
 //     I'' = p_S + P_S p_C, which is the lexicographic rank of the concatenated sequence
 //     (positions off S ascending, then positions on S ascending): one state walks the positions
@@ -36,11 +39,15 @@ struct alignas(16) Smem96 {
     unsigned long long mA[32];                    // ceil(2^64 / A) for A = codewords of weight k (k <= 24), [25]: A = 4096
     uint16_t nwords[32];                          // A: codewords of weight k, [25] = 4096
     uint16_t wbase[32];                           // first by-weight slot of weight k
+    float lg2_down[32];                           // log2(L) rounded down, L = 1..24
+    float lg2_up[32];                             // log2(c) rounded up, c = 1..24
     uint16_t pdep_off[256];
     uint8_t pdep[kPdepEntries];
     float invnorm[256];                           // 1 / (4 sqrt(m)), m <= 214
 };
 static_assert(sizeof(Smem96) % 16 == 0, "16-byte table image");
+
+constexpr float kNarrowLog2_96 = 57.0f;           // 64-bit state once every lane has P_i < 2^57
 
 // 64 x 64 -> 128-bit product
 __device__ __forceinline__ void mul64wide(unsigned long long a, unsigned long long b, unsigned long long &lo,
@@ -158,15 +165,30 @@ struct Dec96 {
         const uint32_t nC = odd ? 24u : 24u - k;
         uint32_t cm = odd ? 0xFFFFFFu : (~word & 0xFFFFFFu), sm = word;
         uint32_t sel0 = 0, sel1 = 0, sel2 = 0;
+        float lp = (float)t;                                             // >= log2 P_i
+        bool wide = true;
 #pragma unroll
         for (int i = 0; i < 24; i++) {
             const bool inC = (uint32_t)i < nC;
             const uint32_t L = inC ? nC - (uint32_t)i : 24u - (uint32_t)i;
-            // phi * L: low 128 bits (the fraction) and the slot above them
-            const unsigned long long t0 = (unsigned long long)f0 * L;
-            const unsigned long long t1 = (unsigned long long)f1 * L + (t0 >> 32);
-            const unsigned long long t2 = (unsigned long long)f2 * L + (t1 >> 32);
-            const unsigned long long t3 = (unsigned long long)f3 * L + (t2 >> 32);
+            if (wide && !__any_sync(__activemask(), lp >= kNarrowLog2_96)) {
+                // narrow to the top 64 bits plus one (uniform over the lanes that vote together;
+                // a lane narrows only when its own bound is below the threshold)
+                const unsigned long long h = ((unsigned long long)f3 << 32 | f2) + 1ull;
+                f2 = (uint32_t)h;
+                f3 = (uint32_t)(h >> 32);
+                wide = false;
+            }
+            // phi * L: the fraction (low limbs) and the slot above it
+            unsigned long long t0 = 0, t1 = 0, t2, t3;
+            if (wide) {
+                t0 = (unsigned long long)f0 * L;
+                t1 = (unsigned long long)f1 * L + (t0 >> 32);
+                t2 = (unsigned long long)f2 * L + (t1 >> 32);
+            } else {
+                t2 = (unsigned long long)f2 * L;
+            }
+            t3 = (unsigned long long)f3 * L + (t2 >> 32);
             const uint32_t slot = (uint32_t)(t3 >> 32);
             // group: the number of cumulative counts C_<=g at or below the slot
             const uint32_t sb = slot * 0x01010101u;
@@ -178,23 +200,32 @@ struct Dec96 {
             const uint32_t en = byte16(y0, y1, y2, y3, grp) - 0x7Fu;                    // C_<=grp
             const uint32_t st = grp ? byte16(y0, y1, y2, y3, grp - 1u) - 0x7Fu : 0u;   // C_<grp
             const uint32_t c = min(en - st, 31u);
-            uint32_t rem = slot - st;                                                  // < c
             y0 -= d0;
             y1 -= d1;
             y2 -= d2;
             y3 -= d3;
-            // phi <- floor((rem 2^128 + fraction) / c) + 1
-            const unsigned long long mc = S.mc[c];
-            const uint32_t n3 = divlimb(rem, (uint32_t)t3, c, mc);
-            const uint32_t n2 = divlimb(rem, (uint32_t)t2, c, mc);
-            const uint32_t n1 = divlimb(rem, (uint32_t)t1, c, mc);
-            const uint32_t n0 = divlimb(rem, (uint32_t)t0, c, mc);
-            unsigned long long lo64 = ((unsigned long long)n1 << 32 | n0) + 1ull;
-            unsigned long long hi64 = ((unsigned long long)n3 << 32 | n2) + (lo64 == 0ull ? 1ull : 0ull);
-            f0 = (uint32_t)lo64;
-            f1 = (uint32_t)(lo64 >> 32);
-            f2 = (uint32_t)hi64;
-            f3 = (uint32_t)(hi64 >> 32);
+            if (i < 23) {                                  // the last step needs no new state
+                // phi <- floor((slot - C_<a) 2^W + fraction) / c) + 1, W = 128 or 64
+                uint32_t rem = slot - st;                                  // < c
+                const unsigned long long mc = S.mc[c];
+                const uint32_t n3 = divlimb(rem, (uint32_t)t3, c, mc);
+                const uint32_t n2 = divlimb(rem, (uint32_t)t2, c, mc);
+                if (wide) {
+                    const uint32_t n1 = divlimb(rem, (uint32_t)t1, c, mc);
+                    const uint32_t n0 = divlimb(rem, (uint32_t)t0, c, mc);
+                    const unsigned long long lo64 = ((unsigned long long)n1 << 32 | n0) + 1ull;
+                    const unsigned long long hi64 = ((unsigned long long)n3 << 32 | n2) + (lo64 == 0ull ? 1ull : 0ull);
+                    f0 = (uint32_t)lo64;
+                    f1 = (uint32_t)(lo64 >> 32);
+                    f2 = (uint32_t)hi64;
+                    f3 = (uint32_t)(hi64 >> 32);
+                } else {
+                    const unsigned long long h64 = ((unsigned long long)n3 << 32 | n2) + 1ull;
+                    f2 = (uint32_t)h64;
+                    f3 = (uint32_t)(h64 >> 32);
+                }
+                lp = lp - S.lg2_down[L] + S.lg2_up[c];                     // P_{i+1} = P_i c / L
+            }
             // coordinate of this step: the lowest position left in its set
             const uint32_t mk = inC ? cm : sm;
             const uint32_t pos = (uint32_t)__ffs((int)mk) - 1u;

@@ -319,6 +319,14 @@ llvq_status create96(llvq_codec *c, std::vector<unsigned char> &image, std::stri
     }
     S.nwords[25] = 4096;
     S.mA[25] = 1ull << 52;
+    for (int n = 1; n <= 24; n++) {             // directed roundings keep the log2 P_i bound above
+        const double l = std::log2((double)n);
+        float dn = (float)l, up = (float)l;
+        while ((double)dn > l) dn = std::nextafter(dn, -INFINITY);
+        while ((double)up < l) up = std::nextafter(up, INFINITY);
+        S.lg2_down[n] = dn;
+        S.lg2_up[n] = up;
+    }
     fill_pdep(S.pdep_off, S.pdep);
     if (T.M > 255) { err = "96-bit shell bound above the table"; return LLVQ_ERR_UNSUPPORTED; }
     for (int m = 1; m <= T.M; m++) S.invnorm[m] = (float)(1.0 / (4.0 * std::sqrt((double)m)));
