@@ -39,24 +39,32 @@ __global__ void __launch_bounds__(512, D::kCtasPerSm) k_decode(typename D::Args 
 template <class D, int BATCH>
 constexpr int gemm_ctas_per_sm() { return BATCH == 1 ? D::kCtasPerSm : 2; }
 
-// Fused decode and multiply, batch BATCH (1..16).  Each CTA owns a contiguous range of rows;
+// Shared accumulator slots per (batch row, output row): one per lane up to batch 7; from batch 8
+// up, lanes l, l + 8, l + 16, l + 24 share a slot, which keeps the accumulators of a 97-row tile
+// at batch 16 within 50 KB (two CTAs per SM).
+template <int BATCH>
+constexpr int gemm_acc_slots() { return BATCH <= 7 ? 32 : 8; }
+
+// Fused decode and multiply, batch `batch` <= BATCH (BATCH 1..7 exact, 8 or 16 with a runtime
+// batch).  Each CTA owns a contiguous range of rows;
 // its threads walk the range's blocks in row-major order (each warp reads 32 consecutive
 // packed words), decode each block once and form scale * <v, x_b> for every batch row.
-// Contributions go to shared-memory accumulators acc[b][row][lane] by atomic add (the lanes of a
-// warp hit distinct words, so only warps of the same CTA can meet on a word); at the end one
-// warp per (b, row) sums the 32 lane slots and writes the output.
+// Contributions go to shared-memory accumulators acc[b][row][slot] by atomic add (slot = lane up
+// to batch 7: only warps of the same CTA meet on a word); at the end one warp per (b, row) sums
+// the slots and writes the output.
 // gain: direct mode -> fp16 gains[row][nb]; table mode -> fp16 gains[row][256] indexed by the
 // word's 8-bit code, times 1/|v| = 1/(4 sqrt(m)) (shape-gain: unit direction times gain).
 template <class D, int BATCH>
 __global__ void __launch_bounds__(512, gemm_ctas_per_sm<D, BATCH>()) k_gemm(
     typename D::Args args, const typename D::Word *__restrict__ words, long long pitch, int rows, int nb,
     uint32_t nb_recip, int gain_mode, const __half *__restrict__ gains, const __half *__restrict__ X,
-    float *__restrict__ Y, int rows_per_cta, unsigned *__restrict__ flags) {
+    float *__restrict__ Y, int rows_per_cta, int batch, unsigned *__restrict__ flags) {
+    constexpr int SLOTS = gemm_acc_slots<BATCH>();
     extern __shared__ __align__(16) unsigned char smem_raw[];
     typename D::Smem &S = *reinterpret_cast<typename D::Smem *>(smem_raw);
-    float *acc = reinterpret_cast<float *>(smem_raw + sizeof(typename D::Smem));  // [BATCH][rpc][32]
+    float *acc = reinterpret_cast<float *>(smem_raw + sizeof(typename D::Smem));  // [BATCH][rpc][SLOTS]
     load_smem_image(&S, args.image, sizeof(typename D::Smem));
-    for (int i = threadIdx.x; i < BATCH * rows_per_cta * 32; i += blockDim.x) acc[i] = 0.f;
+    for (int i = threadIdx.x; i < BATCH * rows_per_cta * SLOTS; i += blockDim.x) acc[i] = 0.f;
     __syncthreads();
     const int row0 = blockIdx.x * rows_per_cta;
     const int nrows = min(rows_per_cta, rows - row0);
@@ -87,6 +95,7 @@ __global__ void __launch_bounds__(512, gemm_ctas_per_sm<D, BATCH>()) k_gemm(
                 for (int e = 0; e < 4; e++) wv[4 * q + e] = (float)(int8_t)(v[q] >> (8 * e));
 #pragma unroll
             for (int bb = 0; bb < BATCH; bb++) {
+                if (BATCH >= 8 && bb >= batch) break;
                 const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
                 float dot = 0.f;
 #pragma unroll
@@ -100,15 +109,16 @@ __global__ void __launch_bounds__(512, gemm_ctas_per_sm<D, BATCH>()) k_gemm(
                         dot = fmaf(wv[8 * c + 2 * e + 1], xf.y, dot);
                     }
                 }
-                atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * dot);
+                atomicAdd(&acc[(bb * rows_per_cta + rl) * SLOTS + (lane & (SLOTS - 1))], scale * dot);
             }
         }
     }
     __syncthreads();
     const int warp = threadIdx.x >> 5;
-    for (int i = warp; i < BATCH * nrows; i += blockDim.x >> 5) {
+    const int nbatch = BATCH >= 8 ? batch : BATCH;
+    for (int i = warp; i < nbatch * nrows; i += blockDim.x >> 5) {
         const int bb = i / nrows, rl = i - bb * nrows;
-        float sum = acc[(bb * rows_per_cta + rl) * 32 + lane];
+        float sum = lane < SLOTS ? acc[(bb * rows_per_cta + rl) * SLOTS + lane] : 0.f;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
         if (lane == 0) Y[(long long)bb * rows + row0 + rl] = sum;

@@ -48,7 +48,8 @@ namespace {
 
 thread_local std::string g_last_error;
 
-// batches from this size up run on the tensor cores (k_gemm_tc); smaller ones on the CUDA cores
+// 48-bit batches from this size up run on the tensor cores (k_gemm_tc48); smaller ones, and every
+// 72/96-bit batch, on the CUDA cores
 constexpr int kTensorCoreMinBatch = 8;
 
 // smallest double >= n / d for small positive integers (directed rounding of the host division)
@@ -400,12 +401,12 @@ cudaError_t launch_decode(const llvq_codec *c, typename D::Args a, const void *w
 
 template <class D, int B>
 cudaError_t launch_gemm(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
-                        float *Y, cudaStream_t st) {
+                        float *Y, cudaStream_t st, int batch = B) {
     const int threads = 512;
     int grid = c->num_sms * gemm_ctas_per_sm<D, B>();
     int rpc = std::max((w->rows + grid - 1) / grid, 1);
     grid = (w->rows + rpc - 1) / rpc;
-    const size_t smem = sizeof(typename D::Smem) + (size_t)B * rpc * 32 * sizeof(float);
+    const size_t smem = sizeof(typename D::Smem) + (size_t)B * rpc * gemm_acc_slots<B>() * sizeof(float);
     const int nb = w->blocks_per_row;
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
@@ -413,13 +414,15 @@ cudaError_t launch_gemm(const llvq_codec *c, typename D::Args a, const llvq_weig
     const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
     k_gemm<D, B><<<grid, threads, smem, st>>>(a, (const typename D::Word *)w->words, w->row_pitch_words,
                                              w->rows, nb, recip, w->gain_mode, (const __half *)w->gains,
-                                             (const __half *)X, Y, rpc, c->d_flags);
+                                             (const __half *)X, Y, rpc, batch, c->d_flags);
     return cudaGetLastError();
 }
 
 template <class D, int... Bs>
 void set_gemm_attrs(std::integer_sequence<int, Bs...>) {
     (cudaFuncSetAttribute(k_gemm<D, Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024), ...);
+    cudaFuncSetAttribute(k_gemm<D, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaFuncSetAttribute(k_gemm<D, 16>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
 }
 
 constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per block on sm_100
@@ -436,25 +439,6 @@ void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
 
 // Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
 // CTAs; the output is zeroed here because the splits add into it.
-template <class D>
-cudaError_t launch_gemm_tc(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
-                           int batch, float *Y, cudaStream_t st) {
-    const int mt = (w->rows + kTcRows - 1) / kTcRows;
-    const int nchunks = (w->blocks_per_row + kTcBlocks - 1) / kTcBlocks;
-    const int target = c->num_sms * tc_ctas_per_sm<D>();
-    int splits = std::max(1, std::min(nchunks, (target + mt - 1) / mt));
-    const int cps = (nchunks + splits - 1) / splits;
-    splits = (nchunks + cps - 1) / cps;
-    cudaError_t e = cudaMemsetAsync(Y, 0, (size_t)batch * w->rows * sizeof(float), st);
-    if (e != cudaSuccess) return e;
-    k_gemm_tc<D><<<dim3(mt, splits), 512, sizeof(TcSmem<D>), st>>>(
-        a, (const typename D::Word *)w->words, w->row_pitch_words, w->rows, w->blocks_per_row, batch, w->gain_mode,
-        (const __half *)w->gains, (const __half *)X, Y, cps, c->d_flags);
-    return cudaGetLastError();
-}
-
-// 48-bit CUDA-core path with coset sorting: one 1024-thread CTA per SM owning a row range; the
-// range shrinks (more CTAs than SMs) only when its accumulators would not fit in shared memory.
 template <int B>
 cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, float *Y,
                               cudaStream_t st) {
@@ -516,8 +500,11 @@ template <class D>
 cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_weight *w, const void *X,
                           int batch, float *Y, cudaStream_t s) {
     if (batch >= kTensorCoreMinBatch) {
+        // 48 bits: tensor cores.  72/96 bits: the decode dominates, and the CUDA-core product that
+        // decodes each block once for the whole batch is faster than 128-row tensor-core rounds
         if constexpr (std::is_same<D, Dec48>::value) return launch_gemm_tc48(c, a, w, X, batch, Y, s);
-        else return launch_gemm_tc<D>(c, a, w, X, batch, Y, s);
+        else if (batch == 8) return launch_gemm<D, 8>(c, a, w, X, Y, s);
+        else return launch_gemm<D, 16>(c, a, w, X, Y, s, batch);
     }
     if constexpr (std::is_same<D, Dec48>::value) {
         switch (batch) {
@@ -604,10 +591,8 @@ void set_kernel_attrs() {
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
-        cudaFuncSetAttribute(k_gemm_tc<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec72>));
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
         cudaFuncSetAttribute(k_decode<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem96));
-        cudaFuncSetAttribute(k_gemm_tc<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(TcSmem<Dec96>));
         set_gemm_attrs<Dec96>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
     });
 }

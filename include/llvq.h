@@ -110,10 +110,11 @@ llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void 
 
 /* Fused decode-and-multiply for 1 <= batch <= 16: d_Y[b][r] for activations d_X [batch][nb*24]
  * (fp16, row stride nb*24, zero beyond cols, 16-byte aligned).  Each block is decoded once for the
- * whole batch.  d_Y: device fp32 [batch][rows], overwritten.  Batches of 8 or more run on the
- * tensor cores: decoded 128-row tiles (exact fp16 integers) times a block-diagonal activation
+ * whole batch.  d_Y: device fp32 [batch][rows], overwritten.  48-bit batches of 8 or more run on
+ * the tensor cores: decoded 128-row tiles (exact fp16 integers) times a block-diagonal activation
  * tile, per-block partial dots in TMEM, gains applied in fp32; that path zeroes d_Y on the stream
- * first and adds K-split partial sums atomically (summation order not fixed). */
+ * first and adds K-split partial sums atomically (summation order not fixed).  72/96-bit batches
+ * run on the CUDA cores at every size (their decode dominates). */
 llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, const void *d_X,
                                  int32_t batch, float *d_Y, void *stream);
 
