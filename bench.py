@@ -182,6 +182,30 @@ def decode_throughput(torch, codec, dev, n, steps, warmup):
             "GBps": n * 32 / t / 1e9}
 
 
+def encode_throughput(torch, codec, dev, n, steps, warmup):
+    """llvq_encode on the n lattice points llvq_decode gives for seeded uniform 48-bit indices
+    (int8 [n, 24] in, packed words out), CUDA-event timed; the round trip must return the indices."""
+    from codebook_free_lattice_b200 import synth
+    lo, _ = synth.uniform_indices(synth.rng(5, 0), n, codec.n_points, 48)
+    w = torch.from_numpy(lo.view(np.int64)).to(dev)
+    vecs = torch.empty((n, 24), dtype=torch.int8, device=dev)
+    codec.decode(w, vecs)
+    out = torch.empty(n, dtype=torch.int64, device=dev)
+    for _ in range(max(warmup, 1)):
+        codec.encode(vecs, out)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        codec.encode(vecs, out)
+    e.record()
+    torch.cuda.synchronize()
+    if not torch.equal(out, w) or codec.get_error() != 0:
+        raise RuntimeError("llvq_encode did not invert llvq_decode")
+    t = s.elapsed_time(e) / 1e3 / max(steps, 1)
+    return {"n": n, "us_per_launch": t * 1e6, "encoded_vectors_per_s": n / t, "GBps": n * 32 / t / 1e9}
+
+
 def cpu_baseline(steps_seconds=12.0):
     """The oracle (fp64, plain C) on a bounded sample of the same workload: whole rows of the
     layer, decoded and multiplied on every host core, timed until ~steps_seconds of work."""
@@ -366,7 +390,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-n", type=int, default=28672 * 342,
                     help="indices for the llvq_decode throughput line (default: the 28672x8192 layer)")
-    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "sweep"],
+    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "encode", "sweep"],
                     help="decode: time llvq_decode alone (profiling aid); sweep: every layer shape, "
                          "budget and batch against cuBLAS fp16, plus the full 7B stack")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: batch (1 = the metric's workload)")
@@ -393,6 +417,11 @@ def main():
         r = decode_throughput(torch, codec, dev, args.decode_n, args.steps, args.warmup)
         if rank == 0:
             print(json.dumps({"mode": "decode", **r}), flush=True)
+        return 0
+    if args.mode == "encode":
+        r = encode_throughput(torch, codec, dev, args.decode_n, args.steps, args.warmup)
+        if rank == 0:
+            print(json.dumps({"mode": "encode", **r}), flush=True)
         return 0
     if args.mode == "sweep":
         if rank == 0:
@@ -500,6 +529,7 @@ def main():
         if B == 1:
             line["issue_roofline"] = issue_roofline(per_launch_s, clk.get("sm_mhz") if clk else None)
         line["decode"] = decode_throughput(torch, codec, dev, args.decode_n, 5, 2)
+        line["encode"] = encode_throughput(torch, codec, dev, args.decode_n, 5, 2)
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline()
         print(json.dumps(line), flush=True)

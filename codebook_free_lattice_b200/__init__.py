@@ -21,6 +21,8 @@ LLVQ_ERR_DEVICE_FLAG = 4
 LLVQ_GAIN_FP16_DIRECT = 0
 LLVQ_GAIN_U8_TABLE = 1
 LLVQ_FLAG_INDEX_RANGE = 0x1
+LLVQ_FLAG_WAIT_TIMEOUT = 0x2
+LLVQ_FLAG_NOT_CODED = 0x4
 
 
 class llvq_weight(C.Structure):
@@ -64,11 +66,13 @@ def lib() -> C.CDLL:
                                            C.c_void_p, C.c_void_p]
         L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
         L.llvq_decode_noalloc.argtypes = [C.c_int32, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
+        L.llvq_encode.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_int32, C.c_void_p]
         L.llvq_last_error_message.argtypes = []
         L.llvq_last_error_message.restype = C.c_char_p
         L.llvq_class_table96.argtypes = [C.c_int32, C.c_void_p, C.c_int64, C.POINTER(C.c_int64)]
         for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
-                  "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc", "llvq_class_table96"):
+                  "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc", "llvq_class_table96",
+                  "llvq_encode"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -76,7 +80,7 @@ def lib() -> C.CDLL:
 
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
             "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
-            "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message")
+            "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message", "llvq_encode")
 
 
 def llvq_status_string(status: int) -> str:
@@ -160,6 +164,13 @@ class Codec:
         n = out.shape[0] if n is None else n
         _check(lib().llvq_decode(self._h, C.c_void_p(words.data_ptr()), self.word_bytes, n,
                                  C.c_void_p(out.data_ptr()), _stream(stream)), "llvq_decode")
+
+    def encode(self, vectors, words, n: int | None = None, stream=None):
+        """vectors: device int8 [n, 24] lattice points; words: device int64 [n] (48-bit budget),
+        written with the packed indices (gain code 0)."""
+        n = vectors.shape[0] if n is None else n
+        _check(lib().llvq_encode(self._h, C.c_void_p(vectors.data_ptr()), n, C.c_void_p(words.data_ptr()),
+                                 self.word_bytes, _stream(stream)), "llvq_encode")
 
     def gemv(self, w: llvq_weight, x, y, stream=None):
         _check(lib().llvq_gemv(self._h, C.byref(w), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()),

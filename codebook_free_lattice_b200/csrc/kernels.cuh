@@ -6,11 +6,13 @@
 #pragma once
 #include "codec48.cuh"
 #include "codec72.cuh"
+#include "encode48.cuh"
 
 namespace llvq {
 
 constexpr unsigned kFlagIndexRange = 0x1u;   // an index >= N_M was met (LLVQ_FLAG_INDEX_RANGE)
 constexpr unsigned kFlagWaitTimeout = 0x2u;  // a bounded wait gave up (LLVQ_FLAG_WAIT_TIMEOUT)
+constexpr unsigned kFlagNotCoded = 0x4u;     // an encoded vector is not a coded point (LLVQ_FLAG_NOT_CODED)
 
 // Decode n packed words into int8 [n][24].
 template <class D>
@@ -34,6 +36,28 @@ __global__ void __launch_bounds__(512, D::kCtasPerSm) k_decode(typename D::Args 
         o[2] = make_uint2(v[4], v[5]);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagIndexRange);
+}
+
+// Encode n lattice points (int8 [n][24]) into 48-bit packed words (gain code 0).
+__global__ void __launch_bounds__(512, 2) k_encode48(const EncSmem48 *__restrict__ image, unsigned long long npoints,
+                                                     const int8_t *__restrict__ vecs, long long n,
+                                                     unsigned long long *__restrict__ words,
+                                                     unsigned *__restrict__ flags) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    EncSmem48 &E = *reinterpret_cast<EncSmem48 *>(smem_raw);
+    load_smem_image(&E, image, sizeof(EncSmem48));
+    __syncthreads();
+    bool bad = false;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n;
+         t += (long long)gridDim.x * blockDim.x) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(vecs + t * 24);
+        const uint2 a = __ldg(src), b = __ldg(src + 1), c = __ldg(src + 2);
+        const uint32_t xw[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
+        unsigned long long I;
+        bad |= !encode48(xw, E, npoints, I);
+        words[t] = I;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagNotCoded);
 }
 
 template <class D, int BATCH>

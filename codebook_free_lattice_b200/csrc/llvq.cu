@@ -22,6 +22,7 @@
 #include "kernels_tc.cuh"
 #include "kernels_tc48.cuh"
 #include "codec96.cuh"
+#include "encode48.cuh"
 #include "tables.h"
 #include "tables96.h"
 
@@ -41,6 +42,7 @@ struct llvq_codec {
     uint32_t *d_guide96 = nullptr; // 96-bit guide table (top 28 index bits)
     void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
+    void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
     unsigned *d_flags = nullptr;   // sticky device flags
 };
 
@@ -208,6 +210,68 @@ llvq_status build_even48(const HostTables &T, Smem48 &S, SmemEven48 &E, std::vec
             }
             E.merge[mq << 8 | bits] = e;
         }
+    return LLVQ_OK;
+}
+
+// Encoder tables of the 48-bit budget: per class its count-vector key, digits and the groups of
+// its two coordinate sets (set 0: off S, or all positions of an odd class; set 1: on S).
+llvq_status build_enc48(const HostTables &T, EncSmem48 &E, std::string &err) {
+    std::memset(&E, 0, sizeof E);
+    std::memcpy(E.golay_mask, T.golay_by_mask, sizeof E.golay_mask);
+    std::memcpy(E.golay_weight, T.golay_by_weight, sizeof E.golay_weight);
+    for (int L = 2; L < 32; L++) E.mL[L] = (unsigned long long)((((u128)1 << 64) + L - 1) / L);
+    for (int k = 0; k <= 24; k++) E.wbase[k] = (uint16_t)T.weight_base[k];
+    const size_t nc = T.classes.size();
+    if (nc > (size_t)kEncClasses48 || T.M >= kEncShells48) { err = "48-bit encoder table too small"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int m = 0; m < kEncShells48; m++)
+        for (int o = 0; o < 2; o++) { E.seg_first[m][o] = 0; E.seg_count[m][o] = 0; }
+    for (size_t i = 0; i < nc; i++) {
+        const HostClass &c = T.classes[i];
+        unsigned long long klo = 0;
+        uint32_t khi = 0;
+        for (size_t g = 0; g < c.vals.size(); g++) {
+            const int v = c.vals[g];
+            if (v > 13) { err = "48-bit class magnitude above 13"; return LLVQ_ERR_UNSUPPORTED; }
+            if (v < 12) klo += (unsigned long long)c.cnts[g] << (5 * v);
+            else khi += (uint32_t)c.cnts[g] << (5 * (v - 12));
+        }
+        E.key_lo[i] = klo;
+        E.key_hi[i] = khi;
+        E.info[i] = c.A | (uint32_t)c.B << 13 | (c.odd ? 1u : 0u) << 18 | (uint32_t)c.k << 19;
+        E.start[i] = (unsigned long long)c.start;
+        // set 1 = the codeword groups of an even class, set 0 = the rest (odd: every group)
+        const int g1 = c.odd ? 0 : c.n_side0;
+        const int first0 = c.odd ? 0 : c.n_side0, n0 = (int)c.vals.size() - first0;
+        if (n0 > 8 || g1 > 4) { err = "48-bit class with too many groups for the encoder"; return LLVQ_ERR_UNSUPPORTED; }
+        unsigned long long v0 = ~0ull, c0 = 0;
+        uint32_t v1 = ~0u, c1 = 0;
+        for (int g = 0; g < n0; g++) {
+            v0 &= ~(0xFFull << (8 * g));
+            v0 |= (unsigned long long)c.vals[first0 + g] << (8 * g);
+            c0 |= (unsigned long long)c.cnts[first0 + g] << (8 * g);
+        }
+        for (int g = 0; g < g1; g++) {
+            v1 &= ~(0xFFu << (8 * g));
+            v1 |= (uint32_t)c.vals[g] << (8 * g);
+            c1 |= (uint32_t)c.cnts[g] << (8 * g);
+        }
+        E.vals0[i] = v0;
+        E.cnt0[i] = c0;
+        E.vals1[i] = v1;
+        E.cnt1[i] = c1;
+        E.P0[i] = (unsigned long long)(c.odd ? c.P : c.P_C);
+        E.P1[i] = (unsigned long long)(c.odd ? 1 : c.P_S);
+        if (c.P > ((u128)1 << 40)) { err = "48-bit arrangement count above 2^40"; return LLVQ_ERR_UNSUPPORTED; }
+        const int o = c.odd ? 1 : 0;
+        if (E.seg_count[c.m][o] == 0) E.seg_first[c.m][o] = (uint16_t)i;
+        E.seg_count[c.m][o]++;
+        // classes of one shell and coset must ascend by key (the order the search relies on)
+        if (E.seg_count[c.m][o] > 1 &&
+            !(E.key_hi[i - 1] < khi || (E.key_hi[i - 1] == khi && E.key_lo[i - 1] < klo))) {
+            err = "48-bit class keys out of order";
+            return LLVQ_ERR_UNSUPPORTED;
+        }
+    }
     return LLVQ_OK;
 }
 
@@ -590,6 +654,7 @@ void set_kernel_attrs() {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
+        cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
         cudaFuncSetAttribute(k_decode<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem96));
@@ -715,6 +780,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::vector<Rec72> recs;
     std::vector<uint32_t> guide, tabC;
     std::vector<unsigned char> even(sizeof(SmemEven48));
+    std::vector<unsigned char> enc(sizeof(EncSmem48));
     llvq_status st;
     if (index_bits == 48) {
         image.resize(sizeof(Smem48));
@@ -722,6 +788,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
         if (st == LLVQ_OK)
             st = build_even48(T, *reinterpret_cast<Smem48 *>(image.data()), *reinterpret_cast<SmemEven48 *>(even.data()),
                               tabC, err);
+        if (st == LLVQ_OK) st = build_enc48(T, *reinterpret_cast<EncSmem48 *>(enc.data()), err);
     } else {
         image.resize(sizeof(Smem72));
         st = build_image72(T, *reinterpret_cast<Smem72 *>(image.data()), recs, guide, err);
@@ -739,7 +806,9 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
                cudaMalloc(&c->d_flags, sizeof(unsigned)) == cudaSuccess &&
                cudaMemset(c->d_flags, 0, sizeof(unsigned)) == cudaSuccess;
     if (okc && index_bits == 48) {
-        okc = cudaMalloc(&c->d_even48, even.size()) == cudaSuccess &&
+        okc = cudaMalloc(&c->d_enc48, enc.size()) == cudaSuccess &&
+              cudaMemcpy(c->d_enc48, enc.data(), enc.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_even48, even.size()) == cudaSuccess &&
               cudaMemcpy(c->d_even48, even.data(), even.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&c->d_tabC48, std::max<size_t>(tabC.size(), 1) * sizeof(uint32_t)) == cudaSuccess &&
               cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess;
@@ -769,6 +838,7 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_guide96) cudaFree(c->d_guide96);
     if (c->d_flags) cudaFree(c->d_flags);
     if (c->d_even48) cudaFree(c->d_even48);
+    if (c->d_enc48) cudaFree(c->d_enc48);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
     delete c;
 }
@@ -795,6 +865,25 @@ llvq_status llvq_decode(const llvq_codec *c, const void *d_words, int32_t word_b
                           : c->index_bits == 72 ? launch_decode<Dec72>(c, args72(c), d_words, n, d_out, st)
                                                 : launch_decode<Dec96>(c, args96(c), d_words, n, d_out, st);
     return e == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
+}
+
+llvq_status llvq_encode(const llvq_codec *c, const int8_t *d_vectors, int64_t n, void *d_words, int32_t word_bytes,
+                        void *stream) {
+    if (!c || n < 0) return LLVQ_ERR_ARG;
+    if (c->index_bits != 48) {
+        g_last_error = "llvq_encode covers the 48-bit budget";
+        return LLVQ_ERR_UNSUPPORTED;
+    }
+    if (n == 0) return LLVQ_OK;
+    if (!d_vectors || !d_words || word_bytes != 8) return LLVQ_ERR_ARG;
+    if (!aligned(d_vectors, 8) || !aligned(d_words, 8)) return LLVQ_ERR_ARG;
+    const int threads = 512;
+    const long long want = (n + threads - 1) / threads;
+    const int grid = (int)std::max(1LL, std::min(want, (long long)c->num_sms * 2));
+    k_encode48<<<grid, threads, sizeof(EncSmem48), (cudaStream_t)stream>>>(
+        (const EncSmem48 *)c->d_enc48, (unsigned long long)c->npoints, d_vectors, n,
+        (unsigned long long *)d_words, c->d_flags);
+    return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 
 llvq_status llvq_gemm_smallbatch(const llvq_codec *c, const llvq_weight *w, const void *d_X,

@@ -56,6 +56,7 @@ typedef enum {
 #define LLVQ_FLAG_INDEX_RANGE 0x1u  /* some index was >= N_M (its block decoded to zero) */
 #define LLVQ_FLAG_WAIT_TIMEOUT 0x2u /* a bounded wait for the tensor cores gave up; the output of
                                        that call is incomplete */
+#define LLVQ_FLAG_NOT_CODED 0x4u    /* llvq_encode met a vector that is not a coded lattice point */
 
 /* Opaque codec: owns the decode tables of one index budget on one device. */
 typedef struct llvq_codec llvq_codec;
@@ -101,6 +102,17 @@ llvq_status llvq_codec_info(const llvq_codec *codec, int32_t *max_shell, uint64_
  * codec), aligned to word_bytes.  d_out: device, 24*n bytes, 8-byte aligned.  n >= 0. */
 llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t word_bytes, int64_t n,
                         int8_t *d_out, void *stream);
+
+/* Encode n lattice points into packed words: the inverse of llvq_decode (the pages describe
+ * the conversion to and from bitstrings; papernotes.org notes, 关键设计 2).  d_vectors: device
+ * int8 [n][24] in the sqrt(8)-scaled coordinates llvq_decode produces, 8-byte aligned.  d_words:
+ * device, n words of word_bytes (8 for the 48-bit budget; other budgets return
+ * LLVQ_ERR_UNSUPPORTED), 8-byte aligned, written with the index in the index bits and a zero gain
+ * code.  A vector that is not a point of the coded shells (wrong coset congruences, not a Golay
+ * codeword pattern, shell outside 2..M, the zero vector) gets the index 2^48 - 1, which decodes to
+ * zero, and raises LLVQ_FLAG_NOT_CODED.  n >= 0. */
+llvq_status llvq_encode(const llvq_codec *codec, const int8_t *d_vectors, int64_t n, void *d_words,
+                        int32_t word_bytes, void *stream);
 
 /* Fused decode-and-multiply, batch 1: d_y[r] = sum_j scale(r, j) * <v(r, j), x[24 j .. 24 j + 23]>
  * with fp32 accumulation.  d_x: device fp16 [blocks_per_row * 24] (zero beyond cols), 16-byte

@@ -116,6 +116,82 @@ def test_decode_out_of_range_sets_flag(gcodec, ocodec):
     assert gcodec.get_error() == 0             # cleared by the previous read
 
 
+# ------------------------------------------------------------------ encode (48-bit) --------
+
+def gpu_encode(gcodec, vecs):
+    v = torch.from_numpy(np.ascontiguousarray(vecs, np.int8)).cuda()
+    w = torch.full((vecs.shape[0],), -1, dtype=torch.int64, device="cuda")
+    gcodec.encode(v, w)
+    torch.cuda.synchronize()
+    return w.cpu().numpy().view(np.uint64)
+
+
+def test_encode_roundtrip_uniform(gcodec, ocodec):
+    """300,000 seeded uniform indices, decoded by the oracle, encode back to themselves."""
+    lo, _ = synth.uniform_indices(synth.rng(70, 0), 300_000, ocodec.n_points, 48)
+    vecs = ocodec.decode_batch(lo)
+    assert np.array_equal(gpu_encode(gcodec, vecs), lo)
+    assert gcodec.get_error() == 0
+
+
+def test_encode_class_boundaries_and_oracle_encode(gcodec, ocodec):
+    """First, middle and last index of every class; each result also equals the oracle's encode."""
+    idx = []
+    for c in ocodec.classes():
+        idx += [c.offset, c.offset + c.size // 2, c.offset + c.size - 1]
+    idx = np.array(idx, dtype=np.uint64)
+    vecs = ocodec.decode_batch(idx)
+    got = gpu_encode(gcodec, vecs)
+    assert np.array_equal(got, idx)
+    for t in range(0, len(idx), 7):
+        assert int(got[t]) == ocodec.encode(vecs[t].astype(np.int32))
+
+
+def test_encode_not_coded(gcodec, ocodec):
+    """Vectors outside the coded set get 2^48 - 1 and raise the flag; the others in the same call
+    still encode exactly."""
+    lo, _ = synth.uniform_indices(synth.rng(71, 0), 64, ocodec.n_points, 48)
+    good = ocodec.decode_batch(lo)
+    bad = [np.zeros(24, np.int8)]                                   # zero vector
+    v = good[0].copy(); v[3] += 2; bad.append(v)                    # breaks the congruences
+    v = good[1].copy(); v[0] = -v[0] if v[0] else 4; bad.append(v)  # flips one sign / off-lattice
+    small = ocodec.decode_batch(np.array([98256], np.uint64))[0]    # shell 2, odd
+    bad.append((small * 4).astype(np.int8))                         # shell 32 > 13
+    v = good[2].copy(); v[5] ^= 1; bad.append(v)                    # mixed parity
+    bad = np.stack(bad)
+    oracle_bad = []
+    for b_ in bad:
+        try:
+            ocodec.encode(b_.astype(np.int32))
+            oracle_bad.append(False)
+        except ValueError:
+            oracle_bad.append(True)
+    vecs = np.concatenate([good[:10], bad, good[10:]])
+    got = gpu_encode(gcodec, vecs)
+    assert gcodec.get_error() == 4
+    nb = len(bad)
+    assert np.array_equal(got[:10], lo[:10]) and np.array_equal(got[10 + nb:], lo[10:])
+    for t in range(nb):
+        if oracle_bad[t]:
+            assert int(got[10 + t]) == 2**48 - 1
+        else:                                                       # a coded point after all
+            assert int(got[10 + t]) == ocodec.encode(bad[t].astype(np.int32))
+    assert all(oracle_bad[t] for t in (0, 1, 3, 4))
+
+
+@pytest.mark.parametrize("n", [0, 1, 33, 513, 4097])
+def test_encode_ragged_sizes(gcodec, ocodec, n):
+    lo, _ = synth.uniform_indices(synth.rng(72, n), max(n, 1), ocodec.n_points, 48)
+    lo = lo[:n]
+    if n == 0:
+        w = torch.full((3,), 7, dtype=torch.int64, device="cuda")
+        gcodec.encode(torch.zeros((1, 24), dtype=torch.int8, device="cuda"), w, n=0)
+        torch.cuda.synchronize()
+        assert (w.cpu() == 7).all()
+        return
+    assert np.array_equal(gpu_encode(gcodec, ocodec.decode_batch(lo)), lo)
+
+
 # ------------------------------------------------------------------ fused products ---------
 def run_gemm(gcodec, layer, batch=None):
     import codebook_free_lattice_b200 as L
