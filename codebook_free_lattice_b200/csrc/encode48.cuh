@@ -10,8 +10,11 @@
 //   2. class: the multiset of |x_i| as a count vector packed 5 bits per magnitude, the largest
 //      magnitude most significant, so that the classes of one shell and coset (ordered by their
 //      descending magnitude tuples) are in ascending key order: a binary search;
-//   3. r: the codeword's place among the codewords of its weight in ascending mask order (even)
-//      or among all codewords in ascending mask order (odd), by binary search;
+//   3. r: the codeword's place among all codewords in ascending mask order (odd) or among those
+//      of its weight (even).  Coordinates 12..23 form an information set of this code (checked
+//      when the tables are built), so the codewords' top 12 bits are distinct and ascend with the
+//      mask: the place in mask order is the top 12 bits, one lookup confirms the codeword, and a
+//      4096-entry table gives the place within the weight;
 //   4. s (even): bit j = sign of the j-th nonzero coordinate (ascending) with the highest
 //      coordinate of S skipped (its sign is the parity sign);
 //   5. I'': the lexicographic ranks p_S of the magnitudes on S (ascending positions) and p_C of
@@ -45,6 +48,7 @@ struct alignas(16) EncSmem48 {
     uint16_t seg_first[kEncShells48][2];          // classes of (shell, coset): first index
     uint16_t seg_count[kEncShells48][2];          //                            and count
     uint16_t wbase[32];                           // first by-weight slot of weight k
+    uint16_t wrank[4096];                         // codeword with top 12 bits t: place within its weight
 };
 static_assert(sizeof(EncSmem48) % 16 == 0, "16-byte table image");
 
@@ -67,16 +71,6 @@ __device__ __forceinline__ void cum_and_count8(unsigned long long c, uint32_t g,
 __device__ __forceinline__ unsigned long long exact_div_small(unsigned long long Mn, uint32_t L,
                                                               const unsigned long long *mL) {
     return L == 1u ? Mn : __umul64hi(Mn, mL[L]);
-}
-
-// first position of value w in the ascending array a[lo, lo + n), or -1
-__device__ __forceinline__ int find_sorted(const uint32_t *a, int lo, int n, uint32_t w) {
-    int l = lo, h = lo + n - 1;
-    while (l < h) {
-        const int mid = (l + h) >> 1;
-        if (a[mid] < w) l = mid + 1; else h = mid;
-    }
-    return (n > 0 && a[l] == w) ? l - lo : -1;
 }
 
 __device__ __forceinline__ bool encode48(const uint32_t xw[6], const EncSmem48 &E, unsigned long long npoints,
@@ -129,9 +123,9 @@ __device__ __forceinline__ bool encode48(const uint32_t xw[6], const EncSmem48 &
     const uint32_t info = E.info[cls];
     const uint32_t A = info & 0x1FFFu, B = (info >> 13) & 0x1Fu, k = (info >> 19) & 0x1Fu;
     // 3. r
-    const int r = odd ? find_sorted(E.golay_mask, 0, 4096, word)
-                      : find_sorted(E.golay_weight, E.wbase[k], (int)A, word);
-    if (r < 0 || (!odd && (uint32_t)__popc(word) != k)) return false;
+    const uint32_t t12 = word >> 12;
+    if (E.golay_mask[t12] != word || (!odd && (uint32_t)__popc(word) != k)) return false;
+    const uint32_t r = odd ? t12 : E.wrank[t12];
     // 4. s (even): signs of the nonzero coordinates, ascending, skipping the top of S
     uint32_t s = 0;
     if (!odd) {

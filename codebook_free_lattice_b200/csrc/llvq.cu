@@ -221,6 +221,14 @@ llvq_status build_enc48(const HostTables &T, EncSmem48 &E, std::string &err) {
     std::memcpy(E.golay_weight, T.golay_by_weight, sizeof E.golay_weight);
     for (int L = 2; L < 32; L++) E.mL[L] = (unsigned long long)((((u128)1 << 64) + L - 1) / L);
     for (int k = 0; k <= 24; k++) E.wbase[k] = (uint16_t)T.weight_base[k];
+    // the top 12 coordinates must be an information set: codeword t of the mask order has top
+    // bits t, so the encoder reads a codeword's place from its top 12 bits
+    for (int t = 0; t < 4096; t++)
+        if ((T.golay_by_mask[t] >> 12) != (uint32_t)t) { err = "Golay top 12 bits are not an information set"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int j = 0; j < 4096; j++) {
+        const uint32_t w = T.golay_by_weight[j];
+        E.wrank[w >> 12] = (uint16_t)(j - T.weight_base[__builtin_popcount(w)]);
+    }
     const size_t nc = T.classes.size();
     if (nc > (size_t)kEncClasses48 || T.M >= kEncShells48) { err = "48-bit encoder table too small"; return LLVQ_ERR_UNSUPPORTED; }
     for (int m = 0; m < kEncShells48; m++)
