@@ -7,6 +7,7 @@
 #include "codec48.cuh"
 #include "codec72.cuh"
 #include "encode48.cuh"
+#include "encode72.cuh"
 
 namespace llvq {
 
@@ -56,6 +57,30 @@ __global__ void __launch_bounds__(512, 2) k_encode48(const EncSmem48 *__restrict
         unsigned long long I;
         bad |= !encode48(xw, E, npoints, I);
         words[t] = I;
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagNotCoded);
+}
+
+// Encode n lattice points (int8 [n][24]) into 72-bit packed words (16 bytes, gain code 0).
+__global__ void __launch_bounds__(512, 2) k_encode72(const EncSmem72 *__restrict__ image,
+                                                     const Rec72 *__restrict__ recs,
+                                                     const unsigned long long *__restrict__ keys,
+                                                     unsigned long long np_lo, unsigned long long np_hi,
+                                                     const int8_t *__restrict__ vecs, long long n,
+                                                     ulonglong2 *__restrict__ words, unsigned *__restrict__ flags) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    EncSmem72 &E = *reinterpret_cast<EncSmem72 *>(smem_raw);
+    load_smem_image(&E, image, sizeof(EncSmem72));
+    __syncthreads();
+    bool bad = false;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n;
+         t += (long long)gridDim.x * blockDim.x) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(vecs + t * 24);
+        const uint2 a = __ldg(src), b = __ldg(src + 1), c = __ldg(src + 2);
+        const uint32_t xw[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
+        unsigned long long lo, hi;
+        bad |= !encode72(xw, E, recs, keys, np_lo, np_hi, lo, hi);
+        words[t] = make_ulonglong2(lo, hi);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagNotCoded);
 }

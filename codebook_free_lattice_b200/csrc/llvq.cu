@@ -23,6 +23,7 @@
 #include "kernels_tc48.cuh"
 #include "codec96.cuh"
 #include "encode48.cuh"
+#include "encode72.cuh"
 #include "tables.h"
 #include "tables96.h"
 
@@ -43,6 +44,8 @@ struct llvq_codec {
     void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
     void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
+    void *d_enc72 = nullptr;       // EncSmem72 image (72-bit encoder)
+    unsigned long long *d_keys72 = nullptr;  // 72-bit class keys (encoder)
     unsigned *d_flags = nullptr;   // sticky device flags
 };
 
@@ -279,6 +282,46 @@ llvq_status build_enc48(const HostTables &T, EncSmem48 &E, std::string &err) {
             err = "48-bit class keys out of order";
             return LLVQ_ERR_UNSUPPORTED;
         }
+    }
+    return LLVQ_OK;
+}
+
+// Encoder tables of the 72-bit budget: the unary class keys (one per class, index order), the
+// (shell, coset) ranges, and the shared-memory image (Golay masks, ranks within weight, binomials).
+llvq_status build_enc72(const HostTables &T, EncSmem72 &E, std::vector<unsigned long long> &keys, std::string &err) {
+    std::memset(&E, 0, sizeof E);
+    std::memcpy(E.golay_mask, T.golay_by_mask, sizeof E.golay_mask);
+    for (int t = 0; t < 4096; t++)
+        if ((T.golay_by_mask[t] >> 12) != (uint32_t)t) { err = "Golay top 12 bits are not an information set"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int j = 0; j < 4096; j++) {
+        const uint32_t w = T.golay_by_weight[j];
+        E.wrank[w >> 12] = (uint16_t)(j - T.weight_base[__builtin_popcount(w)]);
+    }
+    for (int L = 2; L < 32; L++) E.mL[L] = (unsigned long long)((((u128)1 << 64) + L - 1) / L);
+    for (int n = 0; n <= 24; n++)
+        for (int c = 0; c <= 24; c++) {
+            u128 b = 0;
+            if (c <= n) { b = 1; for (int i = 0; i < c; i++) b = b * (u128)(n - i) / (u128)(i + 1); }
+            E.binom[n][c] = (uint32_t)b;
+        }
+    if (T.M >= kEncShells72) { err = "72-bit encoder segment table too small"; return LLVQ_ERR_UNSUPPORTED; }
+    const size_t nc = T.classes.size();
+    keys.assign(nc, 0);
+    for (size_t i = 0; i < nc; i++) {
+        const HostClass &c = T.classes[i];
+        int cnt[15] = {0};
+        for (size_t g = 0; g < c.vals.size(); g++) {
+            if (c.vals[g] > 29) { err = "72-bit class magnitude above 29"; return LLVQ_ERR_UNSUPPORTED; }
+            cnt[c.vals[g] >> 1] += c.cnts[g];
+        }
+        unsigned long long key = 0;
+        for (int b = 14; b >= 0; b--) key = (key << (cnt[b] + 1)) | (((1ull << cnt[b]) - 1ull) << 1);
+        keys[i] = key;
+        if (c.P > ((u128)1 << 52)) { err = "72-bit arrangement count above 2^52"; return LLVQ_ERR_UNSUPPORTED; }
+        const int o = c.odd ? 1 : 0;
+        if (E.seg_count[c.m][o] == 0) E.seg_first[c.m][o] = (uint32_t)i;
+        else if (keys[i - 1] >= key) { err = "72-bit class keys out of order"; return LLVQ_ERR_UNSUPPORTED; }
+        E.seg_count[c.m][o]++;
     }
     return LLVQ_OK;
 }
@@ -663,6 +706,7 @@ void set_kernel_attrs() {
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
+        cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
         cudaFuncSetAttribute(k_decode<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem96));
@@ -789,6 +833,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::vector<uint32_t> guide, tabC;
     std::vector<unsigned char> even(sizeof(SmemEven48));
     std::vector<unsigned char> enc(sizeof(EncSmem48));
+    std::vector<unsigned char> enc72(sizeof(EncSmem72));
+    std::vector<unsigned long long> keys72;
     llvq_status st;
     if (index_bits == 48) {
         image.resize(sizeof(Smem48));
@@ -800,6 +846,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     } else {
         image.resize(sizeof(Smem72));
         st = build_image72(T, *reinterpret_cast<Smem72 *>(image.data()), recs, guide, err);
+        if (st == LLVQ_OK) st = build_enc72(T, *reinterpret_cast<EncSmem72 *>(enc72.data()), keys72, err);
     }
     if (st != LLVQ_OK) { g_last_error = err; return st; }
     llvq_codec *c = new llvq_codec;
@@ -824,6 +871,11 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     if (okc && index_bits == 72) {
         okc = cudaMalloc(&c->d_recs72, recs.size() * sizeof(Rec72)) == cudaSuccess &&
               cudaMemcpy(c->d_recs72, recs.data(), recs.size() * sizeof(Rec72), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_enc72, enc72.size()) == cudaSuccess &&
+              cudaMemcpy(c->d_enc72, enc72.data(), enc72.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_keys72, keys72.size() * sizeof(unsigned long long)) == cudaSuccess &&
+              cudaMemcpy(c->d_keys72, keys72.data(), keys72.size() * sizeof(unsigned long long),
+                         cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&c->d_guide72, guide.size() * sizeof(uint32_t)) == cudaSuccess &&
               cudaMemcpy(c->d_guide72, guide.data(), guide.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess;
     }
@@ -847,6 +899,8 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_flags) cudaFree(c->d_flags);
     if (c->d_even48) cudaFree(c->d_even48);
     if (c->d_enc48) cudaFree(c->d_enc48);
+    if (c->d_enc72) cudaFree(c->d_enc72);
+    if (c->d_keys72) cudaFree(c->d_keys72);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
     delete c;
 }
@@ -878,19 +932,24 @@ llvq_status llvq_decode(const llvq_codec *c, const void *d_words, int32_t word_b
 llvq_status llvq_encode(const llvq_codec *c, const int8_t *d_vectors, int64_t n, void *d_words, int32_t word_bytes,
                         void *stream) {
     if (!c || n < 0) return LLVQ_ERR_ARG;
-    if (c->index_bits != 48) {
-        g_last_error = "llvq_encode covers the 48-bit budget";
+    if (c->index_bits == 96) {
+        g_last_error = "llvq_encode covers the 48- and 72-bit budgets";
         return LLVQ_ERR_UNSUPPORTED;
     }
     if (n == 0) return LLVQ_OK;
-    if (!d_vectors || !d_words || word_bytes != 8) return LLVQ_ERR_ARG;
-    if (!aligned(d_vectors, 8) || !aligned(d_words, 8)) return LLVQ_ERR_ARG;
+    if (!d_vectors || !d_words || word_bytes != (c->index_bits == 48 ? 8 : 16)) return LLVQ_ERR_ARG;
+    if (!aligned(d_vectors, 8) || !aligned(d_words, (size_t)word_bytes)) return LLVQ_ERR_ARG;
     const int threads = 512;
     const long long want = (n + threads - 1) / threads;
     const int grid = (int)std::max(1LL, std::min(want, (long long)c->num_sms * 2));
-    k_encode48<<<grid, threads, sizeof(EncSmem48), (cudaStream_t)stream>>>(
-        (const EncSmem48 *)c->d_enc48, (unsigned long long)c->npoints, d_vectors, n,
-        (unsigned long long *)d_words, c->d_flags);
+    if (c->index_bits == 48)
+        k_encode48<<<grid, threads, sizeof(EncSmem48), (cudaStream_t)stream>>>(
+            (const EncSmem48 *)c->d_enc48, (unsigned long long)c->npoints, d_vectors, n,
+            (unsigned long long *)d_words, c->d_flags);
+    else
+        k_encode72<<<grid, threads, sizeof(EncSmem72), (cudaStream_t)stream>>>(
+            (const EncSmem72 *)c->d_enc72, c->d_recs72, c->d_keys72, (unsigned long long)c->npoints,
+            (unsigned long long)(c->npoints >> 64), d_vectors, n, (ulonglong2 *)d_words, c->d_flags);
     return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 

@@ -106,11 +106,11 @@ llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t wo
 /* Encode n lattice points into packed words: the inverse of llvq_decode (the pages describe
  * the conversion to and from bitstrings; papernotes.org notes, 关键设计 2).  d_vectors: device
  * int8 [n][24] in the sqrt(8)-scaled coordinates llvq_decode produces, 8-byte aligned.  d_words:
- * device, n words of word_bytes (8 for the 48-bit budget; other budgets return
- * LLVQ_ERR_UNSUPPORTED), 8-byte aligned, written with the index in the index bits and a zero gain
- * code.  A vector that is not a point of the coded shells (wrong coset congruences, not a Golay
- * codeword pattern, shell outside 2..M, the zero vector) gets the index 2^48 - 1, which decodes to
- * zero, and raises LLVQ_FLAG_NOT_CODED.  n >= 0. */
+ * device, n words of word_bytes (8 for the 48-bit budget, 16 for the 72-bit budget; the 96-bit
+ * budget returns LLVQ_ERR_UNSUPPORTED), aligned to word_bytes, written with the index in the index
+ * bits and a zero gain code.  A vector that is not a point of the coded shells (wrong coset
+ * congruences, not a Golay codeword pattern, shell outside 2..M, the zero vector) gets the index
+ * 2^index_bits - 1, which decodes to zero, and raises LLVQ_FLAG_NOT_CODED.  n >= 0. */
 llvq_status llvq_encode(const llvq_codec *codec, const int8_t *d_vectors, int64_t n, void *d_words,
                         int32_t word_bytes, void *stream);
 

@@ -408,6 +408,51 @@ def test_gemm72_full_size_sampled_rows(gcodec72, ocodec72, rows, K, batch):
     assert max_rel_err(y[:, rs], ref) < GEMV_RTOL
 
 
+def gpu_encode72(gcodec, vecs):
+    v = torch.from_numpy(np.ascontiguousarray(vecs, np.int8)).cuda()
+    w = torch.full((vecs.shape[0], 2), -1, dtype=torch.int64, device="cuda")
+    gcodec.encode(v, w)
+    torch.cuda.synchronize()
+    out = w.cpu().numpy().view(np.uint64)
+    return out[:, 0], out[:, 1]
+
+
+def test_encode72_roundtrip_uniform_and_boundaries(gcodec72, ocodec72):
+    """100,000 seeded uniform 72-bit indices and the first, middle and last index of every class,
+    decoded by the oracle, encode back to themselves (gain bits zero)."""
+    lo, hi = synth.uniform_indices(synth.rng(73, 0), 100_000, ocodec72.n_points, 72)
+    b_lo, b_hi = [], []
+    for c in ocodec72.classes():
+        for i in (c.offset, c.offset + c.size // 2, c.offset + c.size - 1):
+            b_lo.append(i & (2**64 - 1))
+            b_hi.append(i >> 64)
+    lo = np.concatenate([lo, np.array(b_lo, np.uint64)])
+    hi = np.concatenate([hi, np.array(b_hi, np.uint64)])
+    vecs = ocodec72.decode_batch(lo, hi)
+    glo, ghi = gpu_encode72(gcodec72, vecs)
+    assert np.array_equal(glo, lo) and np.array_equal(ghi, hi)
+    assert gcodec72.get_error() == 0
+    for t in range(0, 100_000, 997):
+        assert (int(ghi[t]) << 64 | int(glo[t])) == ocodec72.encode(vecs[t].astype(np.int32))
+
+
+def test_encode72_not_coded(gcodec72, ocodec72):
+    lo, hi = synth.uniform_indices(synth.rng(74, 0), 16, ocodec72.n_points, 72)
+    good = ocodec72.decode_batch(lo, hi)
+    v1 = good[0].copy(); v1[2] += 2                                   # breaks the congruences
+    v2 = good[1].copy(); v2[7] ^= 1                                   # mixed parity
+    bad = np.stack([np.zeros(24, np.int8), v1, v2])
+    for b_ in bad:
+        with pytest.raises(ValueError):
+            ocodec72.encode(b_.astype(np.int32))
+    glo, ghi = gpu_encode72(gcodec72, np.concatenate([good, bad]))
+    assert gcodec72.get_error() == 4
+    assert np.array_equal(glo[:16], lo) and np.array_equal(ghi[:16], hi)
+    assert (glo[16:] == np.uint64(2**64 - 1)).all() and (ghi[16:] == 0xFF).all()
+
+
+
+
 # ------------------------------------------------------------------ 96-bit budget ----------
 # The oracle builds the class list of a 96-bit shell on demand (up to 9.1M classes for shell
 # 214) and decodes in ascending index order, so the cases below draw their indices from a few
@@ -506,3 +551,12 @@ def test_gemm96_top_shells(gcodec96, ocodec96, batch):
                   index_base=ocodec96.shell_offset(208))
     y = run_gemm(gcodec96, layer)
     assert max_rel_err(y, oracle_gemm(ocodec96, layer)) < GEMV_RTOL
+
+
+def test_encode96_unsupported(gcodec96):
+    import codebook_free_lattice_b200 as L
+    v = torch.zeros((4, 24), dtype=torch.int8, device="cuda")
+    w = torch.zeros((4, 2), dtype=torch.int64, device="cuda")
+    with pytest.raises(L.LLVQError) as e:
+        gcodec96.encode(v, w)
+    assert e.value.status == L.LLVQ_ERR_UNSUPPORTED
