@@ -8,6 +8,7 @@
 #include "codec72.cuh"
 #include "encode48.cuh"
 #include "encode72.cuh"
+#include "encode96.cuh"
 
 namespace llvq {
 
@@ -80,6 +81,57 @@ __global__ void __launch_bounds__(512, 2) k_encode72(const EncSmem72 *__restrict
         const uint32_t xw[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
         unsigned long long lo, hi;
         bad |= !encode72(xw, E, recs, keys, np_lo, np_hi, lo, hi);
+        words[t] = make_ulonglong2(lo, hi);
+    }
+    if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagNotCoded);
+}
+
+// The 96-bit class keys: the unary code of the class's magnitude counts from the coset's
+// largest magnitude down, from the class records (one thread per class).
+__global__ void k_keys96(const Rec96 *__restrict__ recs, long long ncls, unsigned long long *__restrict__ keys) {
+    const long long c = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= ncls) return;
+    const ulonglong2 *rp = reinterpret_cast<const ulonglong2 *>(recs + c);
+    const uint32_t meta = (uint32_t)(__ldg(rp).y >> 32);
+    const uint4 cumv = __ldg(reinterpret_cast<const uint4 *>(rp + 2));
+    const uint4 valv = __ldg(reinterpret_cast<const uint4 *>(rp + 3));
+    const bool odd = meta & kMeta96Odd;
+    const uint32_t cw[4] = {cumv.x, cumv.y, cumv.z, cumv.w}, vw[4] = {valv.x, valv.y, valv.z, valv.w};
+    unsigned long long key = 0;
+    for (int b = 29; b >= 0; b--) {
+        if (odd && b == 29) continue;
+        const uint32_t v = 2u * (uint32_t)b + (odd ? 1u : 0u);
+        uint32_t cnt = 0, prev = 0;
+        for (int g = 0; g < 16; g++) {
+            const uint32_t cg = ((cw[g >> 2] >> (8 * (g & 3))) & 0xFFu) - 0x7Fu;
+            const uint32_t vg = (vw[g >> 2] >> (8 * (g & 3))) & 0xFFu;
+            if (cg > prev && vg == v) cnt = cg - prev;
+            prev = cg;
+        }
+        key = (key << (cnt + 1u)) | (((1ull << cnt) - 1ull) << 1);
+    }
+    keys[c] = key;
+}
+
+// Encode n lattice points (int8 [n][24]) into 96-bit packed words (16 bytes, gain code 0).
+__global__ void __launch_bounds__(256, 2) k_encode96(const EncSmem96 *__restrict__ image,
+                                                     const Rec96 *__restrict__ recs,
+                                                     const unsigned long long *__restrict__ keys,
+                                                     unsigned long long np_lo, unsigned long long np_hi,
+                                                     const int8_t *__restrict__ vecs, long long n,
+                                                     ulonglong2 *__restrict__ words, unsigned *__restrict__ flags) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    EncSmem96 &E = *reinterpret_cast<EncSmem96 *>(smem_raw);
+    load_smem_image(&E, image, sizeof(EncSmem96));
+    __syncthreads();
+    bool bad = false;
+    for (long long t = (long long)blockIdx.x * blockDim.x + threadIdx.x; t < n;
+         t += (long long)gridDim.x * blockDim.x) {
+        const uint2 *src = reinterpret_cast<const uint2 *>(vecs + t * 24);
+        const uint2 a = __ldg(src), b = __ldg(src + 1), c = __ldg(src + 2);
+        const uint32_t xw[6] = {a.x, a.y, b.x, b.y, c.x, c.y};
+        unsigned long long lo, hi;
+        bad |= !encode96(xw, E, recs, keys, np_lo, np_hi, lo, hi);
         words[t] = make_ulonglong2(lo, hi);
     }
     if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0) atomicOr(flags, kFlagNotCoded);

@@ -24,6 +24,7 @@
 #include "codec96.cuh"
 #include "encode48.cuh"
 #include "encode72.cuh"
+#include "encode96.cuh"
 #include "tables.h"
 #include "tables96.h"
 
@@ -46,6 +47,8 @@ struct llvq_codec {
     void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
     void *d_enc72 = nullptr;       // EncSmem72 image (72-bit encoder)
     unsigned long long *d_keys72 = nullptr;  // 72-bit class keys (encoder)
+    void *d_enc96 = nullptr;       // EncSmem96 image (96-bit encoder)
+    unsigned long long *d_keys96 = nullptr;  // 96-bit class keys (encoder, built on the device)
     unsigned *d_flags = nullptr;   // sticky device flags
 };
 
@@ -485,6 +488,47 @@ llvq_status create96(llvq_codec *c, std::vector<unsigned char> &image, std::stri
         err = "96-bit guide construction failed";
         return LLVQ_ERR_CUDA;
     }
+    // encoder: class keys on the device, (shell, coset) ranges and small tables in an image
+    if (cudaMalloc(&c->d_keys96, (size_t)T.n_classes * sizeof(unsigned long long)) != cudaSuccess) {
+        err = "device memory for the 96-bit class keys not available";
+        cudaGetLastError();
+        return LLVQ_ERR_CUDA;
+    }
+    k_keys96<<<(unsigned)((T.n_classes + 255) / 256), 256>>>(c->d_recs96, T.n_classes, c->d_keys96);
+    if (cudaGetLastError() != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+        err = "96-bit class keys failed";
+        return LLVQ_ERR_CUDA;
+    }
+    std::vector<unsigned char> eimg(sizeof(EncSmem96), 0);
+    EncSmem96 &E = *reinterpret_cast<EncSmem96 *>(eimg.data());
+    std::memcpy(E.golay_mask, T.golay_by_mask, sizeof E.golay_mask);
+    for (int t = 0; t < 4096; t++)
+        if ((T.golay_by_mask[t] >> 12) != (uint32_t)t) { err = "Golay top 12 bits are not an information set"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int j = 0; j < 4096; j++) {
+        const uint32_t w = T.golay_by_weight[j];
+        E.wrank[w >> 12] = (uint16_t)(j - T.weight_base[__builtin_popcount(w)]);
+    }
+    for (int L = 2; L < 32; L++) E.mL[L] = (unsigned long long)((((u128)1 << 64) + L - 1) / L);
+    for (int n = 0; n <= 24; n++)
+        for (int k = 0; k <= 24; k++) {
+            u128 b = 0;
+            if (k <= n) { b = 1; for (int i = 0; i < k; i++) b = b * (u128)(n - i) / (u128)(i + 1); }
+            E.binom[n][k] = (uint32_t)b;
+        }
+    for (int k = 0; k <= 24; k++) E.nwords[k] = (uint16_t)T.words_of_weight[k];
+    if (T.M >= kEncShells96) { err = "96-bit encoder segment table too small"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int m = 2; m <= T.M; m++) {
+        E.seg_first[m][0] = (uint32_t)T.class_base[m];
+        E.seg_count[m][0] = (uint32_t)T.shell_even[m];
+        E.seg_first[m][1] = (uint32_t)(T.class_base[m] + T.shell_even[m]);
+        E.seg_count[m][1] = (uint32_t)(T.shell_classes[m] - T.shell_even[m]);
+    }
+    if (cudaMalloc(&c->d_enc96, eimg.size()) != cudaSuccess ||
+        cudaMemcpy(c->d_enc96, eimg.data(), eimg.size(), cudaMemcpyHostToDevice) != cudaSuccess) {
+        err = "device allocation for the 96-bit encoder failed";
+        cudaGetLastError();
+        return LLVQ_ERR_CUDA;
+    }
     return LLVQ_OK;
 }
 
@@ -707,6 +751,7 @@ void set_kernel_attrs() {
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
         cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
+        cudaFuncSetAttribute(k_encode96, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem96));
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
         set_gemm_attrs<Dec72>(std::make_integer_sequence<int, kTensorCoreMinBatch - 1>{});
         cudaFuncSetAttribute(k_decode<Dec96>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem96));
@@ -901,6 +946,8 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_enc48) cudaFree(c->d_enc48);
     if (c->d_enc72) cudaFree(c->d_enc72);
     if (c->d_keys72) cudaFree(c->d_keys72);
+    if (c->d_enc96) cudaFree(c->d_enc96);
+    if (c->d_keys96) cudaFree(c->d_keys96);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
     delete c;
 }
@@ -932,10 +979,6 @@ llvq_status llvq_decode(const llvq_codec *c, const void *d_words, int32_t word_b
 llvq_status llvq_encode(const llvq_codec *c, const int8_t *d_vectors, int64_t n, void *d_words, int32_t word_bytes,
                         void *stream) {
     if (!c || n < 0) return LLVQ_ERR_ARG;
-    if (c->index_bits == 96) {
-        g_last_error = "llvq_encode covers the 48- and 72-bit budgets";
-        return LLVQ_ERR_UNSUPPORTED;
-    }
     if (n == 0) return LLVQ_OK;
     if (!d_vectors || !d_words || word_bytes != (c->index_bits == 48 ? 8 : 16)) return LLVQ_ERR_ARG;
     if (!aligned(d_vectors, 8) || !aligned(d_words, (size_t)word_bytes)) return LLVQ_ERR_ARG;
@@ -946,10 +989,17 @@ llvq_status llvq_encode(const llvq_codec *c, const int8_t *d_vectors, int64_t n,
         k_encode48<<<grid, threads, sizeof(EncSmem48), (cudaStream_t)stream>>>(
             (const EncSmem48 *)c->d_enc48, (unsigned long long)c->npoints, d_vectors, n,
             (unsigned long long *)d_words, c->d_flags);
-    else
+    else if (c->index_bits == 72)
         k_encode72<<<grid, threads, sizeof(EncSmem72), (cudaStream_t)stream>>>(
             (const EncSmem72 *)c->d_enc72, c->d_recs72, c->d_keys72, (unsigned long long)c->npoints,
             (unsigned long long)(c->npoints >> 64), d_vectors, n, (ulonglong2 *)d_words, c->d_flags);
+    else {
+        const long long want96 = (n + 255) / 256;
+        const int grid96 = (int)std::max(1LL, std::min(want96, (long long)c->num_sms * 4));
+        k_encode96<<<grid96, 256, sizeof(EncSmem96), (cudaStream_t)stream>>>(
+            (const EncSmem96 *)c->d_enc96, c->d_recs96, c->d_keys96, (unsigned long long)c->npoints,
+            (unsigned long long)(c->npoints >> 64), d_vectors, n, (ulonglong2 *)d_words, c->d_flags);
+    }
     return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 

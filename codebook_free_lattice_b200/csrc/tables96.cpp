@@ -103,6 +103,7 @@ struct ShellEnum {
     int64_t n = 0;             // valid classes so far
     u128 offset = 0;           // index offset inside the shell (fill mode)
     bool bad = false;
+    int64_t n_even = 0;        // classes of the even coset (enumerated first)
     int gv[kDim], gc[kDim], ng = 0;   // groups chosen so far, descending magnitude
 
     void run() {
@@ -112,6 +113,7 @@ struct ShellEnum {
             while (top * top > norm) top--;
             if ((top & 1) != parity) top--;
             if (top >= parity) dfs(kDim, norm, top, parity);
+            if (parity == 0) n_even = n;
         }
     }
 
@@ -246,6 +248,7 @@ bool build_tables96(Tables96 &T, int threads, std::string &err) {
 
     // classes per shell, counted in parallel (largest shells first)
     T.shell_classes.assign(T.M + 1, 0);
+    T.shell_even.assign(T.M + 1, 0);
     std::atomic<int> next(0);
     std::vector<std::thread> pool;
     const int nthreads = std::max(1, threads);
@@ -260,6 +263,7 @@ bool build_tables96(Tables96 &T, int threads, std::string &err) {
                 e.m = m;
                 e.run();
                 T.shell_classes[m] = e.n;
+                T.shell_even[m] = e.n_even;
             }
         });
     for (auto &t : pool) t.join();

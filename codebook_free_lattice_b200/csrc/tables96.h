@@ -47,6 +47,7 @@ struct Tables96 {
     u128 n_points = 0;                     // N_M
     std::vector<u128> shell_start;         // [m], m = 0..M+1 (first global index of shell m)
     std::vector<int64_t> shell_classes;    // [m]: classes in shell m
+    std::vector<int64_t> shell_even;       // [m]: even-coset classes in shell m (they come first)
     std::vector<int64_t> class_base;       // [m]: global index of the first class of shell m
     int64_t n_classes = 0;
     uint32_t golay_by_mask[4096];          // codewords, ascending mask

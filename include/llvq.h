@@ -86,9 +86,10 @@ typedef struct {
  * llvq_codec_destroy.  Thread-safe to use from several streams afterwards (the codec is
  * read-only except for its sticky flag word).
  * 48 and 72 bits: tables of 76 KB / 11 MB, built in well under a second.  96 bits: 304,649,365
- * class records of 64 bytes plus a 1 GB guide (about 20.5 GB of device memory), built on all host
- * cores (several seconds; a few GB of host memory while it runs); LLVQ_ERR_CUDA when the device
- * memory is not available, with the reason in llvq_last_error_message. */
+ * class records of 64 bytes, a 1 GB guide and 2.4 GB of encoder class keys (about 23 GB of device
+ * memory), built on all host cores and the device (several seconds; a few GB of host memory while
+ * it runs); LLVQ_ERR_CUDA when the device memory is not available, with the reason in
+ * llvq_last_error_message. */
 llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out);
 void llvq_codec_destroy(llvq_codec *codec);
 
@@ -106,9 +107,8 @@ llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t wo
 /* Encode n lattice points into packed words: the inverse of llvq_decode (the pages describe
  * the conversion to and from bitstrings; papernotes.org notes, 关键设计 2).  d_vectors: device
  * int8 [n][24] in the sqrt(8)-scaled coordinates llvq_decode produces, 8-byte aligned.  d_words:
- * device, n words of word_bytes (8 for the 48-bit budget, 16 for the 72-bit budget; the 96-bit
- * budget returns LLVQ_ERR_UNSUPPORTED), aligned to word_bytes, written with the index in the index
- * bits and a zero gain code.  A vector that is not a point of the coded shells (wrong coset
+ * device, n words of word_bytes (8 for the 48-bit budget, 16 for the 72- and 96-bit budgets),
+ * aligned to word_bytes, written with the index in the index bits and a zero gain code.  A vector that is not a point of the coded shells (wrong coset
  * congruences, not a Golay codeword pattern, shell outside 2..M, the zero vector) gets the index
  * 2^index_bits - 1, which decodes to zero, and raises LLVQ_FLAG_NOT_CODED.  n >= 0. */
 llvq_status llvq_encode(const llvq_codec *codec, const int8_t *d_vectors, int64_t n, void *d_words,

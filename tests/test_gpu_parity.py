@@ -553,10 +553,45 @@ def test_gemm96_top_shells(gcodec96, ocodec96, batch):
     assert max_rel_err(y, oracle_gemm(ocodec96, layer)) < GEMV_RTOL
 
 
-def test_encode96_unsupported(gcodec96):
-    import codebook_free_lattice_b200 as L
-    v = torch.zeros((4, 24), dtype=torch.int8, device="cuda")
-    w = torch.zeros((4, 2), dtype=torch.int64, device="cuda")
-    with pytest.raises(L.LLVQError) as e:
-        gcodec96.encode(v, w)
-    assert e.value.status == L.LLVQ_ERR_UNSUPPORTED
+def test_encode96_roundtrip(gcodec96, ocodec96):
+    """Every class boundary of shells 2..6, sampled classes of shells 120 and 214, seeded uniform
+    indices inside shells 3, 50 and 214 and over shells 205..214, and the last coded index:
+    decoded by the oracle, they encode back to themselves; a sample also equals the oracle's
+    encode."""
+    idx = []
+    for m in range(2, 7):
+        for j in range(ocodec96.shell_nclasses(m)):
+            c = ocodec96.shell_class(m, j)
+            idx += [c.offset, c.offset + c.size // 2, c.offset + c.size - 1]
+    for m in (120, 214):
+        n = ocodec96.shell_nclasses(m)
+        for j in list(range(0, n, max(1, n // 60))) + [n - 1]:
+            c = ocodec96.shell_class(m, j)
+            idx += [c.offset, c.offset + c.size - 1]
+    for seed, m in enumerate((3, 50, 214)):
+        idx += uniform_in_shells(ocodec96, m, m, 300, 80 + seed)
+    idx += uniform_in_shells(ocodec96, 205, 214, 2000, 84)
+    idx.append(ocodec96.n_points - 1)
+    lo, hi = split96(idx)
+    vecs = ocodec96.decode_batch(lo, hi)
+    glo, ghi = gpu_encode72(gcodec96, vecs)
+    assert np.array_equal(glo, lo) and np.array_equal(ghi, hi)
+    assert gcodec96.get_error() == 0
+    for t in range(0, len(idx), 97):
+        assert (int(ghi[t]) << 64 | int(glo[t])) == ocodec96.encode(vecs[t].astype(np.int32))
+
+
+def test_encode96_not_coded(gcodec96, ocodec96):
+    lo, hi = split96(uniform_in_shells(ocodec96, 2, 40, 16, 85))
+    good = ocodec96.decode_batch(lo, hi)
+    v1 = good[0].copy(); v1[2] += 2                                   # breaks the congruences
+    v2 = good[1].copy(); v2[7] ^= 1                                   # mixed parity
+    big = (ocodec96.decode_batch(np.array([98256], np.uint64))[0] * 12).astype(np.int8)   # shell 288 > 214
+    bad = np.stack([np.zeros(24, np.int8), v1, v2, big])
+    for b_ in bad:
+        with pytest.raises(ValueError):
+            ocodec96.encode(b_.astype(np.int32))
+    glo, ghi = gpu_encode72(gcodec96, np.concatenate([good, bad]))
+    assert gcodec96.get_error() == 4
+    assert np.array_equal(glo[:16], lo) and np.array_equal(ghi[:16], hi)
+    assert (glo[16:] == np.uint64(2**64 - 1)).all() and (ghi[16:] == 0xFFFFFFFF).all()
