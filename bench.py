@@ -43,13 +43,20 @@ def algorithmic_bytes(rows=ROWS, nb=NB, batch=1) -> int:
 
 
 def kernel_sources_hash() -> str:
+    """Hash of the library sources with comments and blank lines removed, so that the committed
+    ncu record stays tied to the code it was measured on and not to its comments."""
     import glob
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in sorted(glob.glob(os.path.join(ROOT, "codebook_free_lattice_b200", "csrc", "*"))):
         h.update(os.path.basename(f).encode())
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f, encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        lines = [" ".join(line.split()) for line in src.splitlines()]
+        h.update("\n".join(line for line in lines if line).encode())
     return h.hexdigest()
 
 
