@@ -1,8 +1,9 @@
-// kernels.cuh -- decode and fused decode-and-multiply kernels, generic over the index budget's
-// decoder (Dec48 / Dec72).  "Leech Lattice Vector Quantization for Efficient LLM Compression",
-// papernotes.org notes, 方法详解 / 关键设计 4: each block is decoded to its 24-dim integer
-// vector in registers and multiplied with the activations; dequantized weights never reach
-// global memory.
+// kernels.cuh -- decode and fused decode-and-multiply kernels generic over the index budget's
+// decoder (Dec48 for the allocation-free decode; Dec72, Dec96 for every product and decode at 3
+// and 4 bits), and the encoder kernels.  "Leech Lattice Vector Quantization for Efficient LLM
+// Compression", papernotes.org notes, 方法详解 / 关键设计 4: each block is decoded to its 24-dim
+// integer vector in registers and multiplied with the activations; dequantized weights never
+// reach global memory.
 #pragma once
 #include "codec48.cuh"
 #include "codec72.cuh"

@@ -1,7 +1,7 @@
 // llvq.cu -- host side of libllvq: decode-table images for the 48-, 72- and 96-bit index
-// budgets, kernel launches, and the C ABI declared in include/llvq.h.  Kernels: kernels.cuh;
-// decoders: codec48.cuh, codec72.cuh, codec96.cuh; host table construction: tables.cpp,
-// tables96.cpp.
+// budgets, kernel launches, and the C ABI declared in include/llvq.h.  Kernels: kernels.cuh,
+// kernels_bin48.cuh, kernels_tc48.cuh; decoders: codec48.cuh, codec72.cuh, codec96.cuh; encoders:
+// encode48.cuh, encode72.cuh, encode96.cuh; host table construction: tables.cpp, tables96.cpp.
 #include <algorithm>
 #include <atomic>
 #include <cmath>
