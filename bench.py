@@ -42,6 +42,21 @@ def algorithmic_bytes(rows=ROWS, nb=NB, batch=1) -> int:
     return rows * nb * 8 + rows * 512 + batch * nb * 24 * 2 + batch * rows * 4
 
 
+def max_over_ranks(dist, values, device):
+    """Each timing's maximum over all ranks (every rank runs the same steps; the slowest one
+    bounds the whole job)."""
+    import torch
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_gbps(bytes_per_launch, launches_per_rank, secs, world):
+    """Whole-job throughput: every rank streams the same number of launches, the time is the
+    max over ranks, so the job moves world times the per-rank bytes in that time."""
+    return bytes_per_launch * launches_per_rank * world / secs / 1e9
+
+
 def kernel_sources_hash() -> str:
     """Hash of the library sources with comments and blank lines removed, so that the committed
     ncu record stays tied to the code it was measured on and not to its comments."""
@@ -498,19 +513,17 @@ def main():
         secs_e2e = time_steps(args.steps, e2e_step)
 
     if world > 1:
-        t = torch.tensor([secs, secs_e2e], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        secs, secs_e2e = t.tolist()
+        secs, secs_e2e = max_over_ranks(dist, [secs, secs_e2e], dev)
 
     launches = args.steps * R
     bytes_launch = algorithmic_bytes(batch=B)
     per_launch_s = secs / launches
-    gbs = bytes_launch / per_launch_s / 1e9
-    value = gbs * world
+    gbs = bytes_launch / per_launch_s / 1e9                            # one GPU's kernel, for the roofline
+    value = whole_job_gbps(bytes_launch, launches, secs, world)
     peak, peak_kind = measured_peaks()
     h2d = R * B * NB * 24 * 2
     d2h = R * B * ROWS * 4
-    e2e_gbs = bytes_launch * launches / secs_e2e / 1e9 * world
+    e2e_gbs = whole_job_gbps(bytes_launch, launches, secs_e2e, world)
 
     if rank == 0:
         line = {
