@@ -104,3 +104,18 @@ def test_shell_range_and_errors():
     assert L.lib().llvq_class_table96(214, None, 0, C.byref(n)) == L.LLVQ_OK and n.value == 9124194
     small = (L.llvq_class96 * 2)()
     assert L.lib().llvq_class_table96(4, C.cast(small, C.c_void_p), 2, C.byref(n)) == L.LLVQ_ERR_ARG
+
+
+def test_shell_starts_match_theta_series():
+    """Shell m's class records span exactly N_m indices, N_m from the theta series computed here
+    independently (tests/theta.py, Python integers), for m = 2..40."""
+    from tests.theta import leech_shell_sizes
+    N = leech_shell_sizes(41)
+    starts = {}
+    for m in range(2, 42):
+        r0 = L.class_table96(m)[0]
+        starts[m] = int(r0["start_lo"]) | int(r0["start_hi"]) << 64
+    assert starts[2] == 0
+    for m in range(2, 41):
+        assert starts[m + 1] - starts[m] == N[m], m
+
