@@ -58,6 +58,35 @@ def test_host_argument_checks_without_device(lib):
     assert lib.llvq_gemv(None, None, None, None, None) == L.LLVQ_ERR_ARG
     flags = C.c_uint32()
     assert lib.llvq_get_error(None, None, C.byref(flags)) == L.LLVQ_ERR_ARG
+    assert lib.llvq_encode(None, None, 1, None, 8, None) == L.LLVQ_ERR_ARG
+    assert lib.llvq_gemm_smallbatch(None, None, None, 1, None, None) == L.LLVQ_ERR_ARG
+    assert lib.llvq_decode_noalloc(72, None, 16, 1, None, None) == L.LLVQ_ERR_UNSUPPORTED
+    assert "48-bit" in L.lib().llvq_last_error_message().decode()
+
+
+def test_flag_values_match_the_header():
+    import codebook_free_lattice_b200 as L
+    src = open(os.path.join(ROOT, "include", "llvq.h")).read()
+    for name in ("LLVQ_FLAG_INDEX_RANGE", "LLVQ_FLAG_WAIT_TIMEOUT", "LLVQ_FLAG_NOT_CODED"):
+        val = int(re.search(r"#define\s+" + name + r"\s+(0x[0-9a-fA-F]+)u", src).group(1), 16)
+        assert getattr(L, name) == val
+
+
+def test_ncu_record_hash_ignores_comments(tmp_path, monkeypatch):
+    """The bench ties its committed ncu record to the kernel code, not to comments or spacing."""
+    import shutil
+
+    import bench
+    src = os.path.join(ROOT, "codebook_free_lattice_b200", "csrc")
+    dst = tmp_path / "codebook_free_lattice_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_sources_hash()
+    f = dst / "kernels.cuh"
+    f.write_text("// a new comment line\n" + f.read_text().replace("#pragma once", "#pragma once   /* note */"))
+    assert bench.kernel_sources_hash() == h0
+    f.write_text(f.read_text() + "\nconstexpr int kExtra = 1;\n")
+    assert bench.kernel_sources_hash() != h0
 
 
 def test_no_device_is_a_status_not_a_crash(lib):
