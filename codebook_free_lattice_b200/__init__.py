@@ -123,7 +123,8 @@ def _stream(stream) -> C.c_void_p:
 
 
 class Codec:
-    """Decode tables of one index budget (48, 72 or 96 bits) on the current CUDA device."""
+    """Decode and encode tables of one index budget (48, 72 or 96 bits) on the current CUDA device.
+    close() (or leaving a `with` block) releases them at once; the 96-bit tables hold 23.6 GB."""
 
     def __init__(self, index_bits: int = 48):
         h = C.c_void_p()
@@ -151,6 +152,13 @@ class Codec:
             self.close()
         except Exception:
             pass
+
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *exc):
+        self.close()
+        return False
 
     def weight(self, words, gains, rows: int, cols: int, gain_mode: int,
                row_pitch_words: int | None = None) -> llvq_weight:
