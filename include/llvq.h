@@ -1,6 +1,7 @@
 /*
- * llvq.h -- C ABI of libllvq: Leech lattice vector quantization (LLVQ) decode and fused
- * decode-and-multiply on one NVIDIA B200 (sm_100a).
+ * llvq.h -- C ABI of libllvq: Leech lattice vector quantization (LLVQ) decode, encode and
+ * fused decode-and-multiply on one NVIDIA B200 (sm_100a), for 48-, 72- and 96-bit block indices
+ * (2, 3 and 4 bits per weight).
  *
  * What the calls compute ("Leech Lattice Vector Quantization for Efficient LLM Compression",
  * arXiv 2603.11021):
@@ -25,8 +26,9 @@
  *   - Calls validate their arguments on the host and return LLVQ_ERR_ARG without launching
  *     anything when a check fails.  Launch failures return LLVQ_ERR_CUDA.  No call allocates
  *     device memory or synchronises, except llvq_codec_create/destroy and llvq_get_error.
- *   - Device-side faults in the data (an index >= N_M) do not trap: the block decodes to the
- *     zero vector and a sticky flag is set, read back by llvq_get_error.
+ *   - Device-side faults in the data (an index >= N_M; for llvq_encode, a vector outside the
+ *     coded set) do not trap: the block decodes to the zero vector (the vector encodes to an
+ *     invalid index) and a sticky flag is set, read back by llvq_get_error.
  *   - Kernels are written for sm_100a only; there is no CPU fallback.
  */
 #ifndef LLVQ_H
