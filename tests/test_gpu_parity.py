@@ -351,6 +351,14 @@ def split128(vals):
     return lo, hi
 
 
+@pytest.mark.parametrize("batch", [8, 11])
+def test_gemm72_cuda_core_batches(gcodec72, ocodec72, batch):
+    """Batch 8 (its own instantiation) and batch 11 (the 16-wide kernel with a runtime batch) on
+    the CUDA cores, ragged rows and blocks, against the oracle."""
+    layer = Layer(72, 150, 24 * 21 + 5, batch, 90 + batch, ocodec72.n_points, 1)
+    assert max_rel_err(run_gemm(gcodec72, layer), oracle_gemm(ocodec72, layer)) < GEMV_RTOL
+
+
 def test_codec72_info_matches_oracle(gcodec72, ocodec72):
     assert gcodec72.max_shell == ocodec72.max_shell == 53
     assert gcodec72.n_points == ocodec72.n_points
@@ -542,6 +550,14 @@ def test_gemm96_low_shells(gcodec96, ocodec96, batch, rows, K, gain_mode):
                   norms_fn=norms)
     y = run_gemm(gcodec96, layer)
     assert max_rel_err(y, oracle_gemm(ocodec96, layer)) < GEMV_RTOL
+
+
+@pytest.mark.parametrize("batch", [8, 13])
+def test_gemm96_cuda_core_batches(gcodec96, ocodec96, batch):
+    """Batch 8 and batch 13 (runtime batch in the 16-wide kernel), indices over shells 2..60."""
+    layer = Layer(96, 90, 24 * 17 + 3, batch, 95 + batch, ocodec96.n_points, 1,
+                  index_limit=ocodec96.shell_offset(61))
+    assert max_rel_err(run_gemm(gcodec96, layer), oracle_gemm(ocodec96, layer)) < GEMV_RTOL
 
 
 @pytest.mark.parametrize("batch", [1, 16])
