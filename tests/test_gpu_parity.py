@@ -292,8 +292,9 @@ def test_gemm_batch_equals_gemv_columns(gcodec, ocodec):
 
 @pytest.mark.parametrize("bits,rows,K", [(48, 300, 24 * 45 + 5), (72, 130, 24 * 9)])
 def test_tensor_core_batch_equals_column_gemvs(gcodec, gcodec72, ocodec, ocodec72, bits, rows, K):
-    """Batch 16 (tensor-core path, ragged 128-row tile and ragged 4-block chunk) against 16
-    separate batch-1 products (CUDA-core path)."""
+    """Batch 16 against 16 separate batch-1 products: at 48 bits the tensor-core path (ragged
+    128-row tile and ragged 8-block round) against the coset-sorted GEMV, at 72 bits the 16-wide
+    CUDA-core kernel against the batch-1 one."""
     g, o = (gcodec, ocodec) if bits == 48 else (gcodec72, ocodec72)
     layer = Layer(bits, rows, K, 16, 60 + bits, o.n_points, 1)
     Y = run_gemm(g, layer)
