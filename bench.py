@@ -228,9 +228,23 @@ def encode_throughput(torch, codec, dev, n, steps, warmup):
     return {"n": n, "us_per_launch": t * 1e6, "encoded_vectors_per_s": n / t, "GBps": n * 32 / t / 1e9}
 
 
-def cpu_baseline(steps_seconds=12.0):
+def cpu_model() -> str:
+    """The host CPU's model name (first /proc/cpuinfo entry)."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
+def cpu_baseline(steps_seconds=12.0, one_core_seconds=3.0):
     """The oracle (fp64, plain C) on a bounded sample of the same workload: whole rows of the
-    layer, decoded and multiplied on every host core, timed until ~steps_seconds of work."""
+    layer, decoded and multiplied on every host core, timed until ~steps_seconds of work; then,
+    when one_core_seconds > 0, the same on one core for ~one_core_seconds."""
     import oracle
     from codebook_free_lattice_b200 import synth
     oc = oracle.Codec(48)
@@ -251,10 +265,23 @@ def cpu_baseline(steps_seconds=12.0):
             break
     bytes_per_row = NB * 8 + 512
     gbs = done_rows * bytes_per_row / el / 1e9
-    return {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done_rows} rows of the 4096x4104 layer ({rows} rows per pass, all cores), "
-                      f"{el:.1f} s; GB/s of packed words + gain tables processed",
-            "vectors_per_s": done_rows * NB / el}
+    out = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle",
+           "sample": f"{done_rows} rows of the 4096x4104 layer ({rows} rows per pass, all cores), "
+                     f"{el:.1f} s; GB/s of packed words + gain tables processed",
+           "vectors_per_s": done_rows * NB / el, "cpu_model": cpu_model()}
+    if one_core_seconds > 0:
+        r1 = min(8, rows)
+        done1, t1 = 0, time.perf_counter()
+        while True:
+            oc.gemm(words[:r1], NB, 1, gains[:r1], x, 1, threads=1)
+            done1 += r1
+            el1 = time.perf_counter() - t1
+            if el1 > one_core_seconds:
+                break
+        out["one_core"] = {"value": done1 * bytes_per_row / el1 / 1e9, "unit": "GB/s",
+                           "vectors_per_s": done1 * NB / el1,
+                           "sample": f"{done1} rows, {el1:.1f} s on one core"}
+    return out
 
 
 # ------------------------------------------------------------------ secondary measurements
@@ -385,8 +412,8 @@ def run_reference(args, rank, world):
     t0 = time.perf_counter()
     per_step = max(2.0, min(20.0, 150.0 / max(args.steps + args.warmup, 1)))
     for _ in range(args.warmup):
-        cpu_baseline(per_step / 4)
-    vals = [cpu_baseline(per_step) for _ in range(args.steps)]
+        cpu_baseline(per_step / 4, one_core_seconds=0)
+    vals = [cpu_baseline(per_step, one_core_seconds=0) for _ in range(args.steps)]
     v = statistics.median(x["value"] for x in vals)
     ms = statistics.median(algorithmic_bytes() / (x["value"] * 1e9) * 1e3 for x in vals)
     cb = dict(vals[0])
