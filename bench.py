@@ -404,6 +404,33 @@ def sweep(torch, dev):
         print(json.dumps({"sweep": "llama-2-7b stack (224 GEMVs)", "index_bits": bits, "batch": 1,
                           "ms": t * 1e3, "GBps": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / peak,
                           "cublas_fp16_ms": tc * 1e3, "speedup_vs_fp16": tc / t}), flush=True)
+    print(json.dumps(oracle_stack(48)), flush=True)
+
+
+def oracle_stack(bits=48):
+    """The oracle (fp64, all host cores) on one Llama-2-7B-shaped decoder layer (q, k, v, o, gate,
+    up, down GEMVs, u8 gain tables), times 32 for the stack: the whole stack would take minutes."""
+    import oracle
+    from codebook_free_lattice_b200 import synth
+    oc = oracle.Codec(bits)
+    cores = os.cpu_count() or 1
+    secs, nbytes, blocks = 0.0, 0, 0
+    for i, (_, rows, k) in enumerate(LLAMA7B_LAYER):
+        nb = -(-k // 24)
+        lo, hi = synth.uniform_indices(synth.rng(950 + i, 0), rows * nb, oc.n_points, bits)
+        codes = synth.gain_codes(synth.rng(950 + i, 1), rows * nb)
+        w = synth.pack_words(lo, hi, codes, bits)
+        w = w.reshape((rows, nb) + w.shape[1:])
+        gains = synth.chi24_tables(synth.rng(950 + i, 2), rows)
+        x = synth.activations(synth.rng(950 + i, 3), 1, k)
+        t0 = time.perf_counter()
+        oc.gemm(w, nb, 1, gains, x, 1, threads=cores)
+        secs += time.perf_counter() - t0
+        nbytes += rows * nb * (8 if bits == 48 else 16) + rows * 512 + nb * 48 + rows * 4
+        blocks += rows * nb
+    return {"sweep": "llama-2-7b stack, oracle (one decoder layer x 32)", "index_bits": bits, "batch": 1,
+            "ms": 32 * secs * 1e3, "GBps": nbytes / secs / 1e9, "decoded_vectors_per_s": blocks / secs,
+            "cores": cores, "cpu_model": cpu_model()}
 
 
 def run_reference(args, rank, world):
