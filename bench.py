@@ -383,6 +383,7 @@ def sweep(torch, dev):
         del Ws
         print(json.dumps({"sweep": name, "index_bits": bits, "batch": batch, "us": t * 1e6,
                           "GBps": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / peak,
+                          "fp16_equivalent_GBps": 2 * rows * K / t / 1e9,
                           "decoded_vectors_per_s": rows * nb / t, "cublas_fp16_us": tc * 1e6,
                           "speedup_vs_fp16": tc / t, "layer_copies": copies}), flush=True)
         torch.cuda.empty_cache()
@@ -591,6 +592,7 @@ def main():
                                     f"({R * layer_bytes / 2**20:.0f} MiB of words) per step",
                        "parallelism": f"replicas x{world}"},
             "us_per_layer": per_launch_s * 1e6,
+            "fp16_equivalent_GBps": 2 * ROWS * K / per_launch_s / 1e9 * world,
             "decoded_vectors_per_s": ROWS * NB / per_launch_s * world,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
                          "frac": gbs / peak, "traffic": measured_traffic() if B == 1 else None,
