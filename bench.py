@@ -601,6 +601,7 @@ def main():
                     "d2h_bytes_per_step": d2h},
             "gpu_launches": launches,
             "clocks": clk,
+            "gpu_name": torch.cuda.get_device_name(dev),
         }
         if B == 1:
             line["issue_roofline"] = issue_roofline(per_launch_s, clk.get("sm_mhz") if clk else None)
