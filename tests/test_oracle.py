@@ -300,3 +300,16 @@ def test_gemm_batch_equals_repeated_gemv(c48):
         assert (yb == y[b]).all()
     ymt = c48.gemm(words, nb, 1, gains, x, batch, threads=3)
     assert (ymt == y).all()
+
+
+def test_budgets_share_the_index_format():
+    """Shell and class offsets do not depend on the budget: an index below N_13 decodes to the
+    same vector at 48, 72 and 96 bits (the larger budgets only add shells above)."""
+    from codebook_free_lattice_b200 import synth
+    c48, c72, c96 = oracle.Codec(48), oracle.Codec(72), oracle.Codec(96)
+    assert c72.shell_offset(14) == c96.shell_offset(14) == c48.n_points
+    lo, _ = synth.uniform_indices(synth.rng(97, 0), 3000, c48.n_points, 48)
+    lo = np.concatenate([lo, np.array([0, 196559, 196560, c48.n_points - 1], np.uint64)])
+    v48 = c48.decode_batch(lo)
+    assert np.array_equal(c72.decode_batch(lo, np.zeros_like(lo)), v48)
+    assert np.array_equal(c96.decode_batch(lo, np.zeros_like(lo)), v48)
