@@ -93,14 +93,13 @@ def measured_traffic():
     return int(rec["traffic_bytes_per_launch"]) if rec else None
 
 
-def issue_roofline(per_launch_s, sm_mhz):
+def issue_roofline(per_launch_s, sm_mhz, sms):
     """Instruction-issue roofline of the metric's kernel: thread-instructions per second (ncu count
-    of one launch / the measured launch time) against 148 SMs x 4 schedulers x 32 lanes x the SM
+    of one launch / the measured launch time) against sms SMs x 4 schedulers x 32 lanes x the SM
     clock measured during the timed region (one warp-instruction per scheduler and cycle)."""
     rec = profile_record()
     if not rec or "warp_instructions_per_launch" not in rec or not sm_mhz:
         return None
-    sms = torch.cuda.get_device_properties(0).multi_processor_count
     achieved = rec["warp_instructions_per_launch"] * 32 / per_launch_s
     peak = sms * 4 * 32 * sm_mhz * 1e6
     return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "thread-instructions/s",
@@ -434,6 +433,47 @@ def oracle_stack(bits=48):
             "cores": cores, "cpu_model": cpu_model()}
 
 
+def build_line(steps, warmup, R, B, world, secs, secs_e2e, clk, sms, gpu_name):
+    """The bench's JSON record from the timings of one run: secs and secs_e2e are the device
+    times (max over ranks) of `steps` graph replays of R layer launches each, without and with
+    the host copies; clk is the clock summary sampled during the timed region."""
+    launches = steps * R
+    bytes_launch = algorithmic_bytes(batch=B)
+    per_launch_s = secs / launches
+    gbs = bytes_launch / per_launch_s / 1e9                            # one GPU's kernel, for the roofline
+    value = whole_job_gbps(bytes_launch, launches, secs, world)
+    peak, peak_kind = measured_peaks()
+    h2d = R * B * NB * 24 * 2
+    d2h = R * B * ROWS * 4
+    e2e_gbs = whole_job_gbps(bytes_launch, launches, secs_e2e, world)
+    layer_bytes = ROWS * NB * 8
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
+        "warmup": warmup, "ms_per_step": secs / steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD if B == 1 else WORKLOAD.replace("batch 1", f"batch {B}"),
+                   "rows": ROWS, "cols": K, "blocks_per_row": NB,
+                   "batch": B, "index_bits": 48, "layer_copies_per_step": R,
+                   "l2_policy": f"inputs larger than L2: {R} distinct layer copies "
+                                f"({R * layer_bytes / 2**20:.0f} MiB of words) per step",
+                   "parallelism": f"replicas x{world}"},
+        "us_per_layer": per_launch_s * 1e6,
+        "fp16_equivalent_GBps": 2 * ROWS * K / per_launch_s / 1e9 * world,
+        "decoded_vectors_per_s": ROWS * NB / per_launch_s * world,
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                     "frac": gbs / peak, "traffic": measured_traffic() if B == 1 else None,
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
+        "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "gpu_name": gpu_name,
+    }
+    if B == 1:
+        line["issue_roofline"] = issue_roofline(per_launch_s, clk.get("sm_mhz") if clk else None, sms)
+    return line
+
+
 def run_reference(args, rank, world):
     if rank != 0:
         return 0
@@ -570,41 +610,10 @@ def main():
     if world > 1:
         secs, secs_e2e = max_over_ranks(dist, [secs, secs_e2e], dev)
 
-    launches = args.steps * R
-    bytes_launch = algorithmic_bytes(batch=B)
-    per_launch_s = secs / launches
-    gbs = bytes_launch / per_launch_s / 1e9                            # one GPU's kernel, for the roofline
-    value = whole_job_gbps(bytes_launch, launches, secs, world)
-    peak, peak_kind = measured_peaks()
-    h2d = R * B * NB * 24 * 2
-    d2h = R * B * ROWS * 4
-    e2e_gbs = whole_job_gbps(bytes_launch, launches, secs_e2e, world)
-
     if rank == 0:
-        line = {
-            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": WORKLOAD if B == 1 else WORKLOAD.replace("batch 1", f"batch {B}"),
-                       "rows": ROWS, "cols": K, "blocks_per_row": NB,
-                       "batch": B, "index_bits": 48, "layer_copies_per_step": R,
-                       "l2_policy": f"inputs larger than L2: {R} distinct layer copies "
-                                    f"({R * layer_bytes / 2**20:.0f} MiB of words) per step",
-                       "parallelism": f"replicas x{world}"},
-            "us_per_layer": per_launch_s * 1e6,
-            "fp16_equivalent_GBps": 2 * ROWS * K / per_launch_s / 1e9 * world,
-            "decoded_vectors_per_s": ROWS * NB / per_launch_s * world,
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": measured_traffic() if B == 1 else None,
-                         "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)"},
-            "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                    "d2h_bytes_per_step": d2h},
-            "gpu_launches": launches,
-            "clocks": clk,
-            "gpu_name": torch.cuda.get_device_name(dev),
-        }
-        if B == 1:
-            line["issue_roofline"] = issue_roofline(per_launch_s, clk.get("sm_mhz") if clk else None)
+        props = torch.cuda.get_device_properties(dev)
+        line = build_line(args.steps, args.warmup, R, B, world, secs, secs_e2e, clk,
+                          props.multi_processor_count, torch.cuda.get_device_name(dev))
         line["decode"] = decode_throughput(torch, codec, dev, args.decode_n, 5, 2)
         line["encode"] = encode_throughput(torch, codec, dev, args.decode_n, 5, 2)
         if not args.no_cpu_baseline:
