@@ -96,7 +96,8 @@ struct Cls48 {
     bool ok;                   // index < N_M (otherwise the digits describe index 0)
 };
 
-__device__ __forceinline__ Cls48 classify48(unsigned long long w, const Smem48 &S, unsigned long long npoints) {
+template <class Img>
+__device__ __forceinline__ Cls48 classify48(unsigned long long w, const Img &S, unsigned long long npoints) {
     Cls48 c;
     unsigned long long idx = w & 0xFFFFFFFFFFFFull;
     c.ok = idx < npoints;
@@ -140,7 +141,8 @@ __device__ __forceinline__ Cls48 classify48(unsigned long long w, const Smem48 &
 
 // Step 5 after the arrangement: magnitudes and sign flags from the class's group tables by the
 // recorded group nibbles, then the signs.
-__device__ __forceinline__ void finish48(const Smem48 &S, int cls, uint32_t info, bool odd, uint32_t word,
+template <class Img>
+__device__ __forceinline__ void finish48(const Img &S, int cls, uint32_t info, bool odd, uint32_t word,
                                          uint32_t s, bool ok, const uint32_t sel[6], uint32_t v[6]) {
     const uint32_t vals = S.c_vals[cls], gflag = S.c_gflag[cls];
     const uint32_t val4 = info_val4(info), flag4 = info_flag4(info);
@@ -153,14 +155,14 @@ __device__ __forceinline__ void finish48(const Smem48 &S, int cls, uint32_t info
     apply_signs(odd, word, s, F, (info & kInfoParity) ? 1u : 0u, mag, ok, S.pdep_off, S.pdep, v);
 }
 
-// Steps 3-5 for any class: codeword, the arrangement of both coordinate sets, signs.
-__device__ __forceinline__ void arrange48(const Smem48 &S, int cls, uint32_t info, unsigned long long p,
-                                          uint32_t r, uint32_t s, bool ok, uint32_t v[6]) {
+// Steps 4-5 for any class, given its codeword (step 3): the arrangement of both coordinate sets,
+// signs.
+template <class Img>
+__device__ __forceinline__ void arrange48_word(const Img &S, int cls, uint32_t info, uint32_t word,
+                                               unsigned long long p, uint32_t s, bool ok, uint32_t v[6]) {
     const uint32_t info2 = S.c_info2[cls];
     const int nS = (int)((info2 >> 12) & 0x1Fu);
-    // 3. codeword
     const bool odd = info & kInfoOdd;
-    const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
     const uint32_t side0 = odd ? 0xFFFFFFu : word;
     // 4. arrangement.  Byte b of cumB is 0x7F + C_<=b (remaining items of groups 0..b),
     //    biased one below the guard bit so the byte-wise subtraction of the slot never borrows.
@@ -194,6 +196,15 @@ __device__ __forceinline__ void arrange48(const Smem48 &S, int cls, uint32_t inf
         sel[i >> 2] += ssel << (4 * (i & 3));                    // nibble = grp (bias -0x3333)
     }
     finish48(S, cls, info, odd, word, s, ok, sel, v);
+}
+
+// Steps 3-5 for any class: codeword from the shared-memory Golay tables, then the arrangement.
+__device__ __forceinline__ void arrange48(const Smem48 &S, int cls, uint32_t info, unsigned long long p,
+                                          uint32_t r, uint32_t s, bool ok, uint32_t v[6]) {
+    const uint32_t info2 = S.c_info2[cls];
+    const bool odd = info & kInfoOdd;
+    const uint32_t word = odd ? S.golay_mask[r & 4095u] : S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
+    arrange48_word(S, cls, info, word, p, s, ok, v);
 }
 
 // One coordinate of the odd-class loop: at coordinate i the set has 24 - i places left and the
@@ -249,7 +260,8 @@ __device__ __forceinline__ void arrange_odd48(const Smem48 &S, int cls, uint32_t
 struct Even48Idx {
     uint32_t pC, pS;
 };
-__device__ __forceinline__ Even48Idx even48_indices(const Smem48 &S, int cls, unsigned long long p) {
+template <class Img>
+__device__ __forceinline__ Even48Idx even48_indices(const Img &S, int cls, unsigned long long p) {
     Even48Idx x;
     const double fC = __dmul_ru(small_to_double((uint32_t)p), S.c_invP[cls]);   // (p_C + p_S/P_S) / P_C
     const double g0 = __dmul_ru(fC, S.c_PC[cls]);                               // p_C + p_S/P_S
@@ -261,11 +273,11 @@ __device__ __forceinline__ Even48Idx even48_indices(const Smem48 &S, int cls, un
     return x;
 }
 
-// Steps 3 and 5 for an even class on the table path, given the two sets' code sequences: the
-// codeword S, the sequences merged nibble by nibble along S, then the signs.
-__device__ __forceinline__ void even48_merge(const Smem48 &S, const SmemEven48 &E, uint32_t info, uint32_t info2,
-                                             uint32_t r, uint32_t s, uint32_t sS, uint32_t cS, uint32_t v[6]) {
-    const uint32_t word = S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
+// Step 5 for an even class on the table path, given its codeword and the two sets' code sequences:
+// the sequences merged nibble by nibble along the codeword, then the signs.
+template <class Img>
+__device__ __forceinline__ void even48_merge_word(const Img &S, const uint32_t *merge, uint32_t info, uint32_t word,
+                                                  uint32_t s, uint32_t sS, uint32_t cS, uint32_t v[6]) {
     uint32_t mag[6], F = 0, Sw = word;
 #pragma unroll
     for (int q = 0; q < 6; q++) {
@@ -273,13 +285,21 @@ __device__ __forceinline__ void even48_merge(const Smem48 &S, const SmemEven48 &
         Sw >>= 4;
         const uint32_t n2 = 2u * (uint32_t)__popc(mq);
         const uint32_t bits = ((sS & ((1u << n2) - 1u)) | (cS << n2)) & 0xFFu;
-        const uint32_t e = E.merge[(mq << 8) | bits];
+        const uint32_t e = merge[(mq << 8) | bits];
         mag[q] = e & 0x0F0F0F0Fu;
         F |= (e >> 28) << (4 * q);
         sS >>= n2;
         cS >>= 8u - n2;
     }
     apply_signs(false, word, s, F, (info & kInfoParity) ? 1u : 0u, mag, true, S.pdep_off, S.pdep, v);
+}
+
+// Steps 3 and 5 for an even class on the table path: the codeword S from the shared-memory table,
+// then the merge.
+__device__ __forceinline__ void even48_merge(const Smem48 &S, const SmemEven48 &E, uint32_t info, uint32_t info2,
+                                             uint32_t r, uint32_t s, uint32_t sS, uint32_t cS, uint32_t v[6]) {
+    const uint32_t word = S.golay_weight[min((info2 & 0xFFFu) + r, 4095u)];
+    even48_merge_word(S, E.merge, info, word, s, sS, cS, v);
 }
 
 // Steps 3-5 for an even class on the table path.
@@ -315,5 +335,136 @@ struct Dec48 {
         return c.ok;
     }
 };
+
+}  // namespace llvq
+
+namespace llvq {
+
+// ---- odd-coset decode producing fp16 weights (fused products) --------------------------------
+//
+// The odd class's arrangement rank is unranked by the same exact arithmetic decoding as above,
+// restated for the product path so that each coordinate costs fewer instructions:
+//   * the group search yields, by one byte permutation, the biased bytes (31 + C_<a, 31 + C_<=a)
+//     of the chosen group a; the start and the count c follow by two byte dot products;
+//   * each coordinate emits a byte-permutation selector (nibbles 2a, 2a + 1) that later picks
+//     the group's fp16 value from an 8-byte table;
+//   * the last 8 coordinates come from one table: the 4^8 arrangements of every multiset of 8
+//     items over 4 groups, lexicographic per multiset, indexed by the multiset (its cumulative
+//     counts) and floor(f * arrangements).
+// Only classes with at most 4 magnitude groups take this path.
+
+constexpr int kOddTail48 = 8;                                  // coordinates taken from the tail table
+constexpr int kOddBias48 = 31;                                 // byte bias of the cumulative counts
+
+// Shared-memory image of the fused product kernel (k_gemv48): what classification, the odd-coset
+// fp16 path, the even-coset table path and the rare generic path read per block.  The Golay
+// codewords by weight and the S-side arrangement tables are read from global memory (once per
+// even-coset block); an odd codeword is computed from r.
+struct alignas(16) SmemGv48 {
+    unsigned long long starts[400];               // class starts, [nclasses] = N_M
+    double c_invA[kClasses48];                    // 1/A rounded up
+    double c_invP[kClasses48];                    // 1/P rounded up
+    double c_PC[kClasses48];                      // arrangements off S (even; exact), 1 for odd
+    double invc[32];                              // 1/c rounded up, c = 1..24
+    uint32_t c_info[kClasses48];
+    uint32_t c_info2[kClasses48];
+    uint32_t c_offs[kClasses48];
+    uint32_t c_cum[kClasses48];                   // bytes: cumulative counts C_<=g, g = 0..3 (sat. 24)
+    uint32_t c_vals[kClasses48];                  // bytes: magnitudes of groups 0..3
+    uint32_t c_gflag[kClasses48];                 // bytes: per-group sign flag
+    uint32_t c_cumodd[kClasses48];                // odd, <= 4 groups: bytes 31 + C_<=g, g = 0..3
+    uint32_t c_vt[kClasses48][2];                 // odd, <= 4 groups: fp16 value of groups 0..3 on T
+    float invnorm[16];                            // 1 / (4 sqrt(m))
+    uint32_t merge[4096];                         // even table path: merge[mq << 8 | bits] (see SmemEven48)
+    uint4 tsign[256];                             // for a byte of T: the four coordinate-pair masks 0x8000 off T
+    uint2 tailc[732];                             // [C<=0 + 9 C<=1 + 81 C<=2] of an 8-item multiset: (first entry, count)
+    uint16_t guide[(1 << kGuideBits48) + 8];
+    uint16_t tlow[128];                           // low 12 bits of the codeword whose top 12 bits are r: [r & 63] ^ [64 + (r >> 6)]
+    uint16_t pdep_off[256];
+    uint8_t pdep[kPdepEntries + 15];
+};
+static_assert(sizeof(SmemGv48) % 16 == 0, "16-byte table image");
+
+// The codeword T of an odd class: the codeword whose top 12 bits are r (coordinates 12..23 are an
+// information set of this Golay code, and codewords in mask order ascend by their top bits).
+__device__ __forceinline__ uint32_t odd_codeword48(const SmemGv48 &S, uint32_t r) {
+    return r << 12 | (uint32_t)(S.tlow[r & 63u] ^ S.tlow[64u + (r >> 6)]);
+}
+
+// PTX prmt in its generic mode: a selector nibble with bit 3 set replicates the sign of the byte.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// One coordinate of the odd-class decode.  cum bytes: 31 + C_<=b of the remaining items.  One
+// byte permutation of (31 << 24, cum) gives (31 + C_<a, 31 + C_<=a) of the chosen group a
+// (C_<0 = 0 comes from the constant's top byte); then f <- (f L - C_<a) / c rounded upward.
+// sel[i / 4] byte i % 4 receives 0x10 + 0x22 a (fp16 selector of group a).
+template <int I>
+__device__ __forceinline__ void odd_step_f16(double &f, uint32_t &cum, uint32_t sel[6], const double *invc) {
+    constexpr double L = (double)(24 - I);
+    const double g = __dmul_ru(f, L);
+    const uint32_t slot = (uint32_t)__double2loint(__dadd_rz(g, 0x1p52));
+    const uint32_t u = cum - slot * 0x01010101u;                 // bit 5 of byte b: C_<=b > slot
+    const uint32_t dm = (u >> 5) & 0x01010101u;                  // one per group b >= a
+    const uint32_t osel = (uint32_t)__dp4a((int)dm, (int)0xDEDEDEDE, 0x98);     // 0x10 + 0x22 a
+    const uint32_t psel = (uint32_t)__dp4a((int)dm, (int)0xEFEFEFEF, 0x8887);   // 3 + a, 4 + a, zero, zero
+    const uint32_t r = prmt(0x1F000000u, cum, psel);             // (31 + C_<a) | (31 + C_<=a) << 8
+    const uint32_t c = (uint32_t)__dp4a((int)r, 0x000001FF, 0);  // C_<=a - C_<a
+    const int st = __dp4a((int)r, 1, -kOddBias48);               // C_<a
+    const double d = __dadd_ru(g, -(__hiloint2double(0x43300000, st) - 0x1p52));
+    f = __dmul_ru(d, invc[c]);
+    cum -= dm;
+    sel[I >> 2] += osel << (8 * (I & 3));
+}
+
+// Steps 3-5 of an odd class on the fp16 path: the 24 coordinates as fp16 pairs v[q] (coordinates
+// 2q, 2q + 1), signs included.
+__device__ __forceinline__ void arrange_odd48_f16(const SmemGv48 &S,
+                                                  const unsigned long long *__restrict__ tail, int cls,
+                                                  unsigned long long p, uint32_t r, uint32_t v[12]) {
+    double f = __dmul_ru(__hiloint2double(0x43300000 | (int)(uint32_t)(p >> 32), (int)(uint32_t)p) - 0x1p52,
+                         S.c_invP[cls]);
+    uint32_t cum = S.c_cumodd[cls];
+    uint32_t sel[6] = {0u, 0u, 0u, 0u, 0u, 0u};
+    odd_step_f16<0>(f, cum, sel, S.invc);
+    odd_step_f16<1>(f, cum, sel, S.invc);
+    odd_step_f16<2>(f, cum, sel, S.invc);
+    odd_step_f16<3>(f, cum, sel, S.invc);
+    odd_step_f16<4>(f, cum, sel, S.invc);
+    odd_step_f16<5>(f, cum, sel, S.invc);
+    odd_step_f16<6>(f, cum, sel, S.invc);
+    odd_step_f16<7>(f, cum, sel, S.invc);
+    odd_step_f16<8>(f, cum, sel, S.invc);
+    odd_step_f16<9>(f, cum, sel, S.invc);
+    odd_step_f16<10>(f, cum, sel, S.invc);
+    odd_step_f16<11>(f, cum, sel, S.invc);
+    odd_step_f16<12>(f, cum, sel, S.invc);
+    odd_step_f16<13>(f, cum, sel, S.invc);
+    odd_step_f16<14>(f, cum, sel, S.invc);
+    odd_step_f16<15>(f, cum, sel, S.invc);
+    // the last 8 coordinates: multiset by its cumulative counts, rank floor(f * count)
+    const uint32_t cid = (uint32_t)__dp4a((int)cum, 0x00510901, -kOddBias48 * 91);
+    const uint2 tc = S.tailc[cid];
+    const double cnt = __hiloint2double(0x43300000, (int)tc.y) - 0x1p52;
+    const uint32_t rank = (uint32_t)__double2loint(__dadd_rz(__dmul_ru(f, cnt), 0x1p52));
+    const unsigned long long t = __ldg(tail + tc.x + rank);
+    sel[4] = (uint32_t)t;
+    sel[5] = (uint32_t)(t >> 32);
+    // values: the group's fp16 value on T, negated off T
+    const uint32_t T = odd_codeword48(S, r);
+    const uint32_t vt0 = S.c_vt[cls][0], vt1 = S.c_vt[cls][1];
+#pragma unroll
+    for (int b = 0; b < 3; b++) {
+        const uint4 m = S.tsign[(T >> (8 * b)) & 0xFFu];
+        const uint32_t s0 = sel[2 * b], s1 = sel[2 * b + 1];
+        v[4 * b + 0] = prmt(vt0, vt1, s0) ^ m.x;
+        v[4 * b + 1] = prmt(vt0, vt1, s0 >> 16) ^ m.y;
+        v[4 * b + 2] = prmt(vt0, vt1, s1) ^ m.z;
+        v[4 * b + 3] = prmt(vt0, vt1, s1 >> 16) ^ m.w;
+    }
+}
 
 }  // namespace llvq

@@ -33,12 +33,15 @@ __device__ __forceinline__ bool mbar_try_wait_parity(uint32_t bar, uint32_t pari
 // Table images into shared memory with the bulk-copy engine: thread 0 initialises the mbarrier
 // `bar`, announces the bytes of all regions and starts one bulk copy per region (sizes multiples
 // of 16 bytes, both addresses 16-byte aligned); every thread then waits for the bytes to land,
-// for at most kBulkWaitTries polls.  Returns false in every thread if any wait gave up (the
-// caller then skips its work and raises a flag).  Ends with a CTA barrier.
-constexpr int kBulkWaitTries = 1 << 22;
+// for at most first_tries polls.  Returns false in every thread if any wait gave up (the caller
+// then skips its work, raises a flag and returns); in that case every thread first waits again,
+// for at most kBulkWaitTries polls, so that no copy is still writing the shared memory the CTA
+// is about to release.  Ends with a CTA barrier.
+constexpr uint32_t kBulkWaitTries = 1u << 22;
 template <int N>
 __device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void *const (&src)[N],
-                                               const uint32_t (&bytes)[N], unsigned long long *bar) {
+                                               const uint32_t (&bytes)[N], unsigned long long *bar,
+                                               uint32_t first_tries = kBulkWaitTries) {
     const uint32_t b = smem_u32(bar);
     if (threadIdx.x == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
@@ -54,8 +57,11 @@ __device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void
     }
     __syncthreads();                               // barrier initialised before anyone polls it
     bool done = false;
-    for (int it = 0; it < kBulkWaitTries && !done; it++) done = mbar_try_wait_parity(b, 0);
-    return __syncthreads_and(done) != 0;
+    for (uint32_t it = 0; it < first_tries && !done; it++) done = mbar_try_wait_parity(b, 0);
+    if (__syncthreads_and(done) != 0) return true;
+    for (uint32_t it = 0; it < kBulkWaitTries && !done; it++) done = mbar_try_wait_parity(b, 0);
+    __syncthreads();
+    return false;
 }
 
 // int8 x4 -> two half2 (exact): (b ^ 0x80) + 1024 is the fp16 with bits 0x64XX; minus 1152 = b

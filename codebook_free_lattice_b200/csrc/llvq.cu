@@ -19,6 +19,7 @@
 #include "../../include/llvq.h"
 #include "kernels.cuh"
 #include "kernels_bin48.cuh"
+#include "kernels_gemv48.cuh"
 #include "kernels_tc.cuh"
 #include "kernels_tc48.cuh"
 #include "codec96.cuh"
@@ -44,6 +45,10 @@ struct llvq_codec {
     uint32_t *d_guide96 = nullptr; // 96-bit guide table (top 28 index bits)
     void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
+    void *d_gv48 = nullptr;        // SmemGv48 image (48-bit fused products, k_gemv48)
+    unsigned long long *d_tail48 = nullptr;  // 8-coordinate arrangement table (odd-coset fp16 path)
+    uint32_t *d_gweight48 = nullptr;  // Golay codewords by (weight, mask), global copy for k_gemv48
+    uint32_t *d_tabS48 = nullptr;  // S-side arrangement table, global copy for k_gemv48
     void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
     void *d_enc72 = nullptr;       // EncSmem72 image (72-bit encoder)
     unsigned long long *d_keys72 = nullptr;  // 72-bit class keys (encoder)
@@ -55,6 +60,7 @@ struct llvq_codec {
 namespace {
 
 thread_local std::string g_last_error;
+std::atomic<uint32_t> g_first_wait_tries{kBulkWaitTries};   // polls of a kernel's first table-copy wait
 
 // 48-bit batches from this size up run on the tensor cores (k_gemm_tc48); smaller ones, and every
 // 72/96-bit batch, on the CUDA cores
@@ -66,6 +72,7 @@ double round_up_ratio(double n, double d) {
     while (std::fma(r, d, -n) < 0.0) r = std::nextafter(r, INFINITY);
     return r;
 }
+
 
 void fill_pdep(uint16_t off_tab[256], uint8_t tab[kPdepEntries]) {
     int off = 0;
@@ -216,6 +223,88 @@ llvq_status build_even48(const HostTables &T, Smem48 &S, SmemEven48 &E, std::vec
             }
             E.merge[mq << 8 | bits] = e;
         }
+    return LLVQ_OK;
+}
+
+// The image of the fused product kernel (SmemGv48), assembled from the decode image and the
+// even-coset tables, plus the tables of the odd-coset fp16 path: the tail table of every multiset
+// of 8 items over 4 groups, per-class cumulative counts and fp16 values on T, the pair sign masks
+// of a byte of T, and the low codeword bits as a linear function of the top 12 (checked against
+// the whole code).
+uint16_t fp16_bits(int v) {
+    // exact for |v| <= 2048: sign, exponent, 10-bit mantissa
+    if (v == 0) return 0;
+    const uint16_t sign = v < 0 ? 0x8000 : 0;
+    int a = v < 0 ? -v : v, e = 0;
+    while ((a >> e) > 1) e++;
+    const uint32_t mant = (uint32_t)((a << 10) >> e) & 0x3FFu;
+    return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)mant);
+}
+
+llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E, SmemGv48 &G,
+                       std::vector<unsigned long long> &tail, std::string &err) {
+    std::memset(&G, 0, sizeof G);
+    std::memcpy(G.starts, S.starts, sizeof G.starts);
+    std::memcpy(G.c_invA, S.c_invA, sizeof G.c_invA);
+    std::memcpy(G.c_invP, S.c_invP, sizeof G.c_invP);
+    std::memcpy(G.c_PC, S.c_PC, sizeof G.c_PC);
+    std::memcpy(G.invc, S.invc, sizeof G.invc);
+    std::memcpy(G.c_info, S.c_info, sizeof G.c_info);
+    std::memcpy(G.c_info2, S.c_info2, sizeof G.c_info2);
+    std::memcpy(G.c_offs, S.c_offs, sizeof G.c_offs);
+    std::memcpy(G.c_cum, S.c_cum, sizeof G.c_cum);
+    std::memcpy(G.c_vals, S.c_vals, sizeof G.c_vals);
+    std::memcpy(G.c_gflag, S.c_gflag, sizeof G.c_gflag);
+    std::memcpy(G.invnorm, S.invnorm, sizeof G.invnorm);
+    std::memcpy(G.merge, E.merge, sizeof G.merge);
+    std::memcpy(G.guide, S.guide, sizeof S.guide);
+    std::memcpy(G.pdep_off, S.pdep_off, sizeof G.pdep_off);
+    std::memcpy(G.pdep, S.pdep, sizeof S.pdep);
+    // tail: multisets (n0, n1, n2, n3) of 8 items, arrangements lexicographic over groups 0 < 1 < 2 < 3
+    tail.clear();
+    for (int c0 = 0; c0 <= kOddTail48; c0++)
+        for (int c1 = c0; c1 <= kOddTail48; c1++)
+            for (int c2 = c1; c2 <= kOddTail48; c2++) {
+                const int n[4] = {c0, c1 - c0, c2 - c1, kOddTail48 - c2};
+                std::vector<int> seq;
+                for (int g = 0; g < 4; g++)
+                    for (int t = 0; t < n[g]; t++) seq.push_back(g);
+                const uint32_t off = (uint32_t)tail.size();
+                do {
+                    unsigned long long e = 0;
+                    for (int k = 0; k < kOddTail48; k++) e |= (unsigned long long)(0x10 + 0x22 * seq[k]) << (8 * k);
+                    tail.push_back(e);
+                } while (std::next_permutation(seq.begin(), seq.end()));
+                G.tailc[c0 + 9 * c1 + 81 * c2] = make_uint2(off, (uint32_t)(tail.size() - off));
+            }
+    if (tail.size() != 65536) { err = "odd tail table size"; return LLVQ_ERR_UNSUPPORTED; }
+    for (size_t i = 0; i < T.classes.size(); i++) {
+        const HostClass &c = T.classes[i];
+        if (!c.odd || c.vals.size() > 4) continue;
+        G.c_cumodd[i] = (uint32_t)cum_bytes(c, 4) + 0x01010101u * (uint32_t)kOddBias48;
+        uint32_t vt[2] = {0, 0};
+        for (size_t g = 0; g < c.vals.size(); g++) {
+            const int a = c.vals[g];
+            const int on = a % 4 == 1 ? a : -a;        // x_i = a_i exactly when (i in T) == (a_i = 1 mod 4)
+            vt[g / 2] |= (uint32_t)fp16_bits(on) << (16 * (g % 2));
+        }
+        G.c_vt[i][0] = vt[0];
+        G.c_vt[i][1] = vt[1];
+    }
+    for (int tb = 0; tb < 256; tb++) {
+        uint32_t m[4];
+        for (int j = 0; j < 4; j++)
+            m[j] = ((tb >> (2 * j) & 1) ? 0u : 0x8000u) | ((tb >> (2 * j + 1) & 1) ? 0u : 0x80000000u);
+        G.tsign[tb] = make_uint4(m[0], m[1], m[2], m[3]);
+    }
+    for (int j = 0; j < 64; j++) {
+        G.tlow[j] = (uint16_t)(T.golay_by_mask[j] & 0xFFFu);
+        G.tlow[64 + j] = (uint16_t)(T.golay_by_mask[j << 6] & 0xFFFu);
+    }
+    for (uint32_t r = 0; r < 4096; r++) {
+        const uint32_t w = r << 12 | (uint32_t)(G.tlow[r & 63u] ^ G.tlow[64u + (r >> 6)]);
+        if (w != T.golay_by_mask[r]) { err = "Golay low bits are not linear in the top 12"; return LLVQ_ERR_UNSUPPORTED; }
+    }
     return LLVQ_OK;
 }
 
@@ -586,48 +675,50 @@ void set_gemm_attrs(std::integer_sequence<int, Bs...>) {
 
 constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per block on sm_100
 
-template <int... Bs>
-void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
-    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                          (int)kBinSmemLimit), ...);
-    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                          (int)kBinSmemLimit), ...);
+void set_bin48_attrs() {
     cudaFuncSetAttribute(k_bin48<DecodeSink, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kBinSmemLimit);
 }
 
-// Tensor-core path: 128-row tiles x K chunks of 4 blocks; enough K splits to give every SM its
-// CTAs; the output is zeroed here because the splits add into it.
+// 48-bit products of batch 1..7 (k_gemv48): one CTA per SM over a row range; the row range
+// shrinks (more CTAs than SMs) when the row accumulators would not fit next to the tables.
 template <int B>
-cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, float *Y,
-                              cudaStream_t st) {
+cudaError_t launch_gemv48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, float *Y,
+                          cudaStream_t st) {
     const int nb = w->blocks_per_row;
     if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
-    // one CTA per SM over a row range; 5 blocks per thread and chunk when the row accumulators
-    // leave room, else 4, else the row range shrinks (more CTAs than SMs)
     int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
-    int per = bin48_smem_bytes(B, rpc, 5) <= kBinSmemLimit ? 5 : 4;
-    while (rpc > 1 && bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) rpc = (rpc + 1) / 2;
-    if (bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) return cudaErrorInvalidValue;
+    while (rpc > 1 && gv48_smem_bytes(B, rpc) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (gv48_smem_bytes(B, rpc) > kBinSmemLimit) return cudaErrorInvalidValue;
+    if (rpc > 0xFFFF) return cudaErrorInvalidValue;                 // row field of a record
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
     const int grid = (w->rows + rpc - 1) / rpc;
-    const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
-    GemvSink<B> sink{};
-    sink.words = (const unsigned long long *)w->words;
-    sink.pitch = w->row_pitch_words;
-    sink.rows = w->rows;
-    sink.nb = nb;
-    sink.nb_recip = recip;
-    sink.gain_mode = w->gain_mode;
-    sink.gains = (const __half *)w->gains;
-    sink.X = (const __half *)X;
-    sink.Y = Y;
-    sink.rows_per_cta = rpc;
-    auto kern = per == 5 ? k_bin48<GemvSink<B>, 5> : k_bin48<GemvSink<B>, 4>;
-    kern<<<grid, kBinThreads, bin48_smem_bytes(B, rpc, per), st>>>(a, (const SmemEven48 *)c->d_even48,
-                                                                  c->d_tabC48, sink, c->d_flags);
+    GvArgs g{};
+    g.image = (const SmemGv48 *)c->d_gv48;
+    g.npoints = a.npoints;
+    g.gweight = c->d_gweight48;
+    g.tabS = c->d_tabS48;
+    g.tabC = c->d_tabC48;
+    g.tail = c->d_tail48;
+    g.words = (const unsigned long long *)w->words;
+    g.pitch = w->row_pitch_words;
+    g.rows = w->rows;
+    g.nb = nb;
+    g.nb_recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
+    g.gain_mode = w->gain_mode;
+    g.gains = (const __half *)w->gains;
+    g.X = (const __half *)X;
+    g.Y = Y;
+    g.rows_per_cta = rpc;
+    g.wait_tries = g_first_wait_tries.load();
+    k_gemv48<B><<<grid, kGvThreads, gv48_smem_bytes(B, rpc), st>>>(g, c->d_flags);
     return cudaGetLastError();
+}
+
+template <int... Bs>
+void set_gemv48_attrs(std::integer_sequence<int, Bs...>) {
+    (cudaFuncSetAttribute(k_gemv48<Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
 }
 
 // 48-bit tensor-core path: 128-row tiles x K splits of 8-block rounds.  The split is chosen to
@@ -667,13 +758,13 @@ cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_we
     }
     if constexpr (std::is_same<D, Dec48>::value) {
         switch (batch) {
-            case 1: return launch_gemm_bin48<1>(c, a, w, X, Y, s);
-            case 2: return launch_gemm_bin48<2>(c, a, w, X, Y, s);
-            case 3: return launch_gemm_bin48<3>(c, a, w, X, Y, s);
-            case 4: return launch_gemm_bin48<4>(c, a, w, X, Y, s);
-            case 5: return launch_gemm_bin48<5>(c, a, w, X, Y, s);
-            case 6: return launch_gemm_bin48<6>(c, a, w, X, Y, s);
-            default: return launch_gemm_bin48<7>(c, a, w, X, Y, s);
+            case 1: return launch_gemv48<1>(c, a, w, X, Y, s);
+            case 2: return launch_gemv48<2>(c, a, w, X, Y, s);
+            case 3: return launch_gemv48<3>(c, a, w, X, Y, s);
+            case 4: return launch_gemv48<4>(c, a, w, X, Y, s);
+            case 5: return launch_gemv48<5>(c, a, w, X, Y, s);
+            case 6: return launch_gemv48<6>(c, a, w, X, Y, s);
+            default: return launch_gemv48<7>(c, a, w, X, Y, s);
         }
     } else {
         switch (batch) {
@@ -703,14 +794,16 @@ llvq_status check_weight(const llvq_codec *c, const llvq_weight *w) {
 }  // namespace
 
 // ---- decode without any device allocation -----------------------------------------------
-// A caller that cannot allocate device memory (inside a CUDA-graph capture, under a framework's
-// memory pool that owns every byte, in a plug-in with a fixed device budget) cannot create a
-// codec, because llvq_codec_create allocates its tables with cudaMalloc.  llvq_decode_noalloc
-// keeps the decode kernel's non-input, non-output global memory -- the 48-bit table image and
-// the sticky flag word -- in this file-scope device array instead.  Every GPU that loads the
-// library holds it (kNoAllocScratchBytes) until the process exits.
+// A caller that cannot allocate device memory (under a framework's memory pool that owns every
+// byte, in a plug-in with a fixed device budget, on a path where cudaMalloc's device-wide
+// synchronisation is not allowed) cannot create a codec, because llvq_codec_create allocates its
+// tables with cudaMalloc.  llvq_decode_noalloc keeps the decode kernel's non-input, non-output
+// global memory -- the 48-bit table image and the status word -- in this file-scope device array
+// instead.  Every GPU that loads the library holds it (kNoAllocScratchBytes) until the process
+// exits.
 constexpr size_t kNoAllocFlagOffset = (sizeof(Smem48) + 255) / 256 * 256;
-constexpr size_t kNoAllocScratchBytes = kNoAllocFlagOffset + 256;     // 66,304 B
+constexpr size_t kNoAllocScratchBytes = kNoAllocFlagOffset + 256;     // 76,544 B
+static_assert(kNoAllocScratchBytes == 76544, "the documented size of the allocation-free decode's array");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
@@ -748,7 +841,8 @@ void set_kernel_attrs() {
     std::call_once(once, [] {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
-        set_bin48_attrs(std::make_integer_sequence<int, 7>{});
+        set_bin48_attrs();
+        set_gemv48_attrs(std::make_integer_sequence<int, 7>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
         cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
         cudaFuncSetAttribute(k_encode96, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem96));
@@ -797,7 +891,7 @@ extern "C" {
 llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t word_bytes, int64_t n,
                                 int8_t *d_out, void *stream) {
     if (index_bits != 48) {
-        g_last_error = "llvq_decode_noalloc holds only the 48-bit table image (64.4 KiB); larger budgets need a codec";
+        g_last_error = "llvq_decode_noalloc holds only the 48-bit table image (76,544 bytes); larger budgets need a codec";
         return LLVQ_ERR_UNSUPPORTED;
     }
     if (n < 0 || word_bytes != 8) return LLVQ_ERR_ARG;
@@ -877,6 +971,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::vector<Rec72> recs;
     std::vector<uint32_t> guide, tabC;
     std::vector<unsigned char> even(sizeof(SmemEven48));
+    std::vector<unsigned char> gv(sizeof(SmemGv48));
+    std::vector<unsigned long long> tail48;
     std::vector<unsigned char> enc(sizeof(EncSmem48));
     std::vector<unsigned char> enc72(sizeof(EncSmem72));
     std::vector<unsigned long long> keys72;
@@ -887,6 +983,9 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
         if (st == LLVQ_OK)
             st = build_even48(T, *reinterpret_cast<Smem48 *>(image.data()), *reinterpret_cast<SmemEven48 *>(even.data()),
                               tabC, err);
+        if (st == LLVQ_OK)
+            st = build_gv48(T, *reinterpret_cast<const Smem48 *>(image.data()), *reinterpret_cast<const SmemEven48 *>(even.data()),
+                            *reinterpret_cast<SmemGv48 *>(gv.data()), tail48, err);
         if (st == LLVQ_OK) st = build_enc48(T, *reinterpret_cast<EncSmem48 *>(enc.data()), err);
     } else {
         image.resize(sizeof(Smem72));
@@ -911,7 +1010,18 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
               cudaMalloc(&c->d_even48, even.size()) == cudaSuccess &&
               cudaMemcpy(c->d_even48, even.data(), even.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&c->d_tabC48, std::max<size_t>(tabC.size(), 1) * sizeof(uint32_t)) == cudaSuccess &&
-              cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess;
+              cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_gv48, gv.size()) == cudaSuccess &&
+              cudaMemcpy(c->d_gv48, gv.data(), gv.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_gweight48, 4096 * sizeof(uint32_t)) == cudaSuccess &&
+              cudaMemcpy(c->d_gweight48, reinterpret_cast<const Smem48 *>(image.data())->golay_weight, 4096 * sizeof(uint32_t),
+                         cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_tabS48, kTabS48 * sizeof(uint32_t)) == cudaSuccess &&
+              cudaMemcpy(c->d_tabS48, reinterpret_cast<const SmemEven48 *>(even.data())->tabS, kTabS48 * sizeof(uint32_t),
+                         cudaMemcpyHostToDevice) == cudaSuccess &&
+              cudaMalloc(&c->d_tail48, tail48.size() * sizeof(unsigned long long)) == cudaSuccess &&
+              cudaMemcpy(c->d_tail48, tail48.data(), tail48.size() * sizeof(unsigned long long),
+                         cudaMemcpyHostToDevice) == cudaSuccess;
     }
     if (okc && index_bits == 72) {
         okc = cudaMalloc(&c->d_recs72, recs.size() * sizeof(Rec72)) == cudaSuccess &&
@@ -949,6 +1059,10 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_enc96) cudaFree(c->d_enc96);
     if (c->d_keys96) cudaFree(c->d_keys96);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
+    if (c->d_gv48) cudaFree(c->d_gv48);
+    if (c->d_gweight48) cudaFree(c->d_gweight48);
+    if (c->d_tabS48) cudaFree(c->d_tabS48);
+    if (c->d_tail48) cudaFree(c->d_tail48);
     delete c;
 }
 

@@ -132,17 +132,22 @@ llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void 
 llvq_status llvq_gemm_smallbatch(const llvq_codec *codec, const llvq_weight *w, const void *d_X,
                                  int32_t batch, float *d_Y, void *stream);
 
-/* Decode without any device allocation, for callers that cannot call cudaMalloc -- for
- * example code running inside a CUDA-graph capture, or a plug-in whose device memory is owned by
- * a framework allocator.  The paper has no counterpart; this is a packaging variant of
+/* Decode without any device allocation.  Some callers cannot call cudaMalloc: a plug-in whose
+ * device memory is all owned by a framework's caching allocator, or a latency-critical path
+ * where cudaMalloc's implicit device synchronisation is not allowed.  They cannot create a codec
+ * (llvq_codec_create allocates its tables), so this entry point keeps what the decode kernel
+ * needs besides its input and output -- the 48-bit table image and a status word -- in one
+ * static device array inside the library: 76,544 bytes on every device that loads the library,
+ * held until the process exits.  The paper has no counterpart; this is a packaging variant of
  * llvq_decode for the 48-bit budget only (index_bits must be 48, word_bytes 8; anything else is
- * LLVQ_ERR_UNSUPPORTED / LLVQ_ERR_ARG).  The decode tables and the status word live in one
- * static device array inside the library (76,544 bytes on every device that loads it, held until
- * the process exits) instead of a codec.  The first call on a device builds the tables on the
- * host and copies them in synchronously, so make that first call before any stream capture.
- * Calls share the array: indices >= N_M still decode to the zero vector (a coded point is never
- * zero), and the shared status word is cleared by every call, so calls that overlap on the GPU
- * race on it.  Arguments as for llvq_decode. */
+ * LLVQ_ERR_UNSUPPORTED / LLVQ_ERR_ARG).  It calls no cudaMalloc, cudaFree or allocating library
+ * routine.  The first call on a device builds the tables on the host and copies them into the
+ * array synchronously (set-up, once per device).  Do not reset the device after that call: the
+ * library keeps the array's address and would not copy the tables again.  Calls share the
+ * array, and calls that overlap on the GPU race on its status word.  An index >= N_M decodes to
+ * the zero vector (a coded point is never zero); no call reports it -- llvq_get_error reads a
+ * codec's flags, not this array -- so zero rows are the only sign of such an index.  Arguments
+ * as for llvq_decode. */
 llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t word_bytes, int64_t n,
                                 int8_t *d_out, void *stream);
 
