@@ -67,6 +67,8 @@ def lib() -> C.CDLL:
         L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
         L.llvq_decode_noalloc.argtypes = [C.c_int32, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
         L.llvq_encode.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_int32, C.c_void_p]
+        L.llvq_set_wait_polls.argtypes = [C.c_uint32, C.c_uint32]
+        L.llvq_set_wait_polls.restype = None
         L.llvq_last_error_message.argtypes = []
         L.llvq_last_error_message.restype = C.c_char_p
         L.llvq_class_table96.argtypes = [C.c_int32, C.c_void_p, C.c_int64, C.POINTER(C.c_int64)]
@@ -80,7 +82,13 @@ def lib() -> C.CDLL:
 
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
             "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
-            "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message", "llvq_encode")
+            "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message", "llvq_encode",
+            "llvq_set_wait_polls")
+
+
+def llvq_set_wait_polls(table_polls: int = 0xFFFFFFFF, mma_polls: int = 0xFFFFFFFF) -> None:
+    """Limits of the kernels' first bounded waits (tests of the timeout paths); defaults restore."""
+    lib().llvq_set_wait_polls(table_polls, mma_polls)
 
 
 def llvq_status_string(status: int) -> str:

@@ -348,18 +348,25 @@ namespace llvq {
 //     of the chosen group a; the start and the count c follow by two byte dot products;
 //   * each coordinate emits a byte-permutation selector (nibbles 2a, 2a + 1) that later picks
 //     the group's fp16 value from an 8-byte table;
-//   * the last 8 coordinates come from one table: the 4^8 arrangements of every multiset of 8
-//     items over 4 groups, lexicographic per multiset, indexed by the multiset (its cumulative
-//     counts) and floor(f * arrangements).
+//   * the last 6 coordinates come from one shared-memory table: the 4^6 arrangements of every
+//     multiset of 6 items over 4 groups, lexicographic per multiset (2-bit group codes), indexed by
+//     the multiset (its cumulative counts) and floor(f * arrangements).
 // Only classes with at most 4 magnitude groups take this path.
 
-constexpr int kOddTail48 = 8;                                  // coordinates taken from the tail table
+constexpr int kOddTail48 = 6;                                  // coordinates taken from the tail table
+constexpr int kOddSteps48 = 24 - kOddTail48;                   // coordinates decoded step by step
 constexpr int kOddBias48 = 31;                                 // byte bias of the cumulative counts
 
 // Shared-memory image of the fused product kernel (k_gemv48): what classification, the odd-coset
-// fp16 path, the even-coset table path and the rare generic path read per block.  The Golay
-// codewords by weight and the S-side arrangement tables are read from global memory (once per
-// even-coset block); an odd codeword is computed from r.
+// fp16 path, the even-coset table path and the rare generic path read per block.  An odd codeword
+// is computed from r; the complement arrangement table (1.6 MB) is read from global memory.
+//
+// merge16[mq << 8 | bits] serves the even-coset fp16 path: for the four coordinates of one nibble
+// whose codeword positions are mq, bits holds the popcount(mq) S-side codes and then the
+// complement codes (2 bits each, in position order); the entry is the byte-permutation selectors
+// of the coordinates' fp16 values as two pairs, (z0, i0, z1, i1) and (z2, i2, z3, i3), where i is
+// |x| / 2, an index into the 8-byte table of the fp16 high bytes of 0, 2, ..., 14, and z is the
+// nibble 0 or 8 (both give the zero low byte), bit 3 of z_k being the coordinate's nonzero flag.
 struct alignas(16) SmemGv48 {
     unsigned long long starts[400];               // class starts, [nclasses] = N_M
     double c_invA[kClasses48];                    // 1/A rounded up
@@ -374,10 +381,14 @@ struct alignas(16) SmemGv48 {
     uint32_t c_gflag[kClasses48];                 // bytes: per-group sign flag
     uint32_t c_cumodd[kClasses48];                // odd, <= 4 groups: bytes 31 + C_<=g, g = 0..3
     uint32_t c_vt[kClasses48][2];                 // odd, <= 4 groups: fp16 value of groups 0..3 on T
+    uint32_t c_magS[kClasses48];                  // even table path: ceil(2^32 / P_S), 0 for P_S = 1
     float invnorm[16];                            // 1 / (4 sqrt(m))
-    uint32_t merge[4096];                         // even table path: merge[mq << 8 | bits] (see SmemEven48)
-    uint4 tsign[256];                             // for a byte of T: the four coordinate-pair masks 0x8000 off T
-    uint2 tailc[732];                             // [C<=0 + 9 C<=1 + 81 C<=2] of an 8-item multiset: (first entry, count)
+    uint32_t merge16[4096];                       // even table path (see above)
+    uint32_t tabS[kTabS48];                       // even table path: S-side code sequences (see SmemEven48)
+    uint32_t gweight[4096];                       // Golay codewords in (weight, mask) order
+    uint2 nsign[16];                              // for a nibble of negative flags: the two coordinate-pair masks
+    uint2 tailc[344];                             // [C<=0 + 7 C<=1 + 49 C<=2] of a 6-item multiset: (first entry, count)
+    uint16_t tail[4096];                          // the 6-item arrangements, 2-bit group codes, first coordinate lowest
     uint16_t guide[(1 << kGuideBits48) + 8];
     uint16_t tlow[128];                           // low 12 bits of the codeword whose top 12 bits are r: [r & 63] ^ [64 + (r >> 6)]
     uint16_t pdep_off[256];
@@ -420,51 +431,101 @@ __device__ __forceinline__ void odd_step_f16(double &f, uint32_t &cum, uint32_t 
     sel[I >> 2] += osel << (8 * (I & 3));
 }
 
-// Steps 3-5 of an odd class on the fp16 path: the 24 coordinates as fp16 pairs v[q] (coordinates
-// 2q, 2q + 1), signs included.
-__device__ __forceinline__ void arrange_odd48_f16(const SmemGv48 &S,
-                                                  const unsigned long long *__restrict__ tail, int cls,
-                                                  unsigned long long p, uint32_t r, uint32_t v[12]) {
-    double f = __dmul_ru(__hiloint2double(0x43300000 | (int)(uint32_t)(p >> 32), (int)(uint32_t)p) - 0x1p52,
-                         S.c_invP[cls]);
-    uint32_t cum = S.c_cumodd[cls];
-    uint32_t sel[6] = {0u, 0u, 0u, 0u, 0u, 0u};
-    odd_step_f16<0>(f, cum, sel, S.invc);
-    odd_step_f16<1>(f, cum, sel, S.invc);
-    odd_step_f16<2>(f, cum, sel, S.invc);
-    odd_step_f16<3>(f, cum, sel, S.invc);
-    odd_step_f16<4>(f, cum, sel, S.invc);
-    odd_step_f16<5>(f, cum, sel, S.invc);
-    odd_step_f16<6>(f, cum, sel, S.invc);
-    odd_step_f16<7>(f, cum, sel, S.invc);
-    odd_step_f16<8>(f, cum, sel, S.invc);
-    odd_step_f16<9>(f, cum, sel, S.invc);
-    odd_step_f16<10>(f, cum, sel, S.invc);
-    odd_step_f16<11>(f, cum, sel, S.invc);
-    odd_step_f16<12>(f, cum, sel, S.invc);
-    odd_step_f16<13>(f, cum, sel, S.invc);
-    odd_step_f16<14>(f, cum, sel, S.invc);
-    odd_step_f16<15>(f, cum, sel, S.invc);
-    // the last 8 coordinates: multiset by its cumulative counts, rank floor(f * count)
-    const uint32_t cid = (uint32_t)__dp4a((int)cum, 0x00510901, -kOddBias48 * 91);
-    const uint2 tc = S.tailc[cid];
-    const double cnt = __hiloint2double(0x43300000, (int)tc.y) - 0x1p52;
-    const uint32_t rank = (uint32_t)__double2loint(__dadd_rz(__dmul_ru(f, cnt), 0x1p52));
-    const unsigned long long t = __ldg(tail + tc.x + rank);
-    sel[4] = (uint32_t)t;
-    sel[5] = (uint32_t)(t >> 32);
-    // values: the group's fp16 value on T, negated off T
-    const uint32_t T = odd_codeword48(S, r);
-    const uint32_t vt0 = S.c_vt[cls][0], vt1 = S.c_vt[cls][1];
+// Steps 3-5 of an even class on the table path, as fp16 pairs v[q] (coordinates 2q, 2q + 1):
+// p = p_S + P_S p_C by one multiply-high and a correction; the complement's code sequence from
+// the global table cS (its entry fetched by the caller), the S side from shared memory; the two
+// sequences merged nibble by nibble into fp16 selectors (merge16), with the nonzero flags F; the
+// sign bits s deposited on the nonzero coordinates skipping the highest of S, whose sign makes the
+// number of negatives on S match the class parity; signs applied to the fp16 pairs.
+__device__ __forceinline__ uint32_t even48_pC(const SmemGv48 &S, int cls, uint32_t p, uint32_t &pS) {
+    const uint32_t PS = S.c_info2[cls] >> 17, m = S.c_magS[cls];
+    uint32_t q = m ? __umulhi(p, m) : p;                  // q or q + 1
+    int rem = (int)(p - q * PS);
+    if (rem < 0) {
+        rem += (int)PS;
+        q -= 1u;
+    }
+    pS = (uint32_t)rem;
+    return q;
+}
+__device__ __forceinline__ void arrange_even48_f16(const SmemGv48 &S, int cls, uint32_t info, uint32_t pS,
+                                                   uint32_t r, uint32_t s, uint32_t cS, uint32_t v[12]) {
+    const uint32_t offs = S.c_offs[cls];
+    const uint32_t info2 = S.c_info2[cls];
+    uint32_t sS = S.tabS[(offs >> 19) + pS];
+    const uint32_t word = S.gweight[min((info2 & 0xFFFu) + r, 4095u)];
+    constexpr uint32_t kVlo = 0x46444000u, kVhi = 0x4B4A4948u;   // fp16 high bytes of 0, 2, ..., 14
+    uint32_t Sw = word, F = 0;
 #pragma unroll
-    for (int b = 0; b < 3; b++) {
-        const uint4 m = S.tsign[(T >> (8 * b)) & 0xFFu];
-        const uint32_t s0 = sel[2 * b], s1 = sel[2 * b + 1];
-        v[4 * b + 0] = prmt(vt0, vt1, s0) ^ m.x;
-        v[4 * b + 1] = prmt(vt0, vt1, s0 >> 16) ^ m.y;
-        v[4 * b + 2] = prmt(vt0, vt1, s1) ^ m.z;
-        v[4 * b + 3] = prmt(vt0, vt1, s1 >> 16) ^ m.w;
+    for (int q = 0; q < 6; q++) {
+        const uint32_t mq = Sw & 0xFu;
+        Sw >>= 4;
+        const uint32_t n2 = 2u * (uint32_t)__popc(mq);
+        const uint32_t bits = ((sS & ((1u << n2) - 1u)) | (cS << n2)) & 0xFFu;
+        const uint32_t e = S.merge16[(mq << 8) | bits];
+        sS >>= n2;
+        cS >>= 8u - n2;
+        v[2 * q] = prmt(kVlo, kVhi, e);
+        v[2 * q + 1] = prmt(kVlo, kVhi, e >> 16);
+        F |= (((e & 0x08080808u) * 0x01020408u) >> 27) << (4 * q);
+    }
+    const uint32_t topbit = word ? (0x80000000u >> __clz(word)) : 0u;
+    uint32_t neg = pdep24(s, F & ~topbit, S.pdep_off, S.pdep);
+    neg |= ((__popc(neg & word) ^ ((info & kInfoParity) ? 1u : 0u)) & 1u) ? topbit : 0u;
+#pragma unroll
+    for (int q = 0; q < 6; q++) {
+        const uint2 m = S.nsign[(neg >> (4 * q)) & 0xFu];
+        v[2 * q] ^= m.x;
+        v[2 * q + 1] ^= m.y;
     }
 }
 
+// Steps 3-5 of an odd class on the fp16 path: the 24 coordinates as fp16 pairs v[q] (coordinates
+// 2q, 2q + 1), signs included.
+__device__ __forceinline__ void odd48_setup(const SmemGv48 &S, int cls, unsigned long long p, double &f,
+                                            uint32_t &cum, uint32_t sel[6]) {
+    f = __dmul_ru(__hiloint2double(0x43300000 | (int)(uint32_t)(p >> 32), (int)(uint32_t)p) - 0x1p52, S.c_invP[cls]);
+    cum = S.c_cumodd[cls];
+#pragma unroll
+    for (int q = 0; q < 6; q++) sel[q] = 0u;
+}
+// the last 6 coordinates from the tail table: multiset by its cumulative counts, rank
+// floor(f * count); the 2-bit group codes spread to nibbles, then to fp16 selectors (0x10 + 0x22 a
+// by a byte permutation); then the values (the group's fp16 value on T, negated off T)
+__device__ __forceinline__ void odd48_finish(const SmemGv48 &S, int cls, uint32_t r, double f, uint32_t cum,
+                                             uint32_t sel[6], uint32_t v[12]) {
+    const uint32_t cid = (uint32_t)__dp4a((int)cum, 0x00310701, -kOddBias48 * 57);
+    const uint2 tc = S.tailc[cid];
+    const double cnt = __hiloint2double(0x43300000, (int)tc.y) - 0x1p52;
+    const uint32_t rank = (uint32_t)__double2loint(__dadd_rz(__dmul_ru(f, cnt), 0x1p52));
+    uint32_t x = S.tail[tc.x + rank];                       // codes of coordinates 18..23
+    x = (x | x << 8) & 0x00FF00FFu;
+    x = (x | x << 4) & 0x0F0F0F0Fu;
+    x = (x | x << 2) & 0x33333333u;                         // nibble k: code of coordinate 18 + k
+    sel[4] |= prmt(0x76543210u, 0u, x) << 16;               // coordinates 18, 19 into bytes 2, 3
+    sel[5] = prmt(0x76543210u, 0u, x >> 8);                 // coordinates 20..23
+    const uint32_t offT = ~odd_codeword48(S, r);
+    const uint32_t vt0 = S.c_vt[cls][0], vt1 = S.c_vt[cls][1];
+#pragma unroll
+    for (int b = 0; b < 3; b++) {
+        const uint2 m0 = S.nsign[(offT >> (8 * b)) & 0xFu], m1 = S.nsign[(offT >> (8 * b + 4)) & 0xFu];
+        const uint32_t s0 = sel[2 * b], s1 = sel[2 * b + 1];
+        v[4 * b + 0] = prmt(vt0, vt1, s0) ^ m0.x;
+        v[4 * b + 1] = prmt(vt0, vt1, s0 >> 16) ^ m0.y;
+        v[4 * b + 2] = prmt(vt0, vt1, s1) ^ m1.x;
+        v[4 * b + 3] = prmt(vt0, vt1, s1 >> 16) ^ m1.y;
+    }
+}
+#define LLVQ_ODD_STEPS(X)                                                                         \
+    X(0) X(1) X(2) X(3) X(4) X(5) X(6) X(7) X(8) X(9) X(10) X(11) X(12) X(13) X(14) X(15) X(16) X(17)
+__device__ __forceinline__ void arrange_odd48_f16(const SmemGv48 &S, int cls, unsigned long long p, uint32_t r,
+                                                  uint32_t v[12]) {
+    double f;
+    uint32_t cum, sel[6];
+    odd48_setup(S, cls, p, f, cum, sel);
+#define LLVQ_STEP1(I) odd_step_f16<I>(f, cum, sel, S.invc);
+    LLVQ_ODD_STEPS(LLVQ_STEP1)
+#undef LLVQ_STEP1
+    odd48_finish(S, cls, r, f, cum, sel, v);
+}
 }  // namespace llvq

@@ -30,18 +30,16 @@ __device__ __forceinline__ bool mbar_try_wait_parity(uint32_t bar, uint32_t pari
     return ok != 0;
 }
 
-// Table images into shared memory with the bulk-copy engine: thread 0 initialises the mbarrier
-// `bar`, announces the bytes of all regions and starts one bulk copy per region (sizes multiples
-// of 16 bytes, both addresses 16-byte aligned); every thread then waits for the bytes to land,
-// for at most first_tries polls.  Returns false in every thread if any wait gave up (the caller
-// then skips its work, raises a flag and returns); in that case every thread first waits again,
-// for at most kBulkWaitTries polls, so that no copy is still writing the shared memory the CTA
-// is about to release.  Ends with a CTA barrier.
+// Table images into shared memory with the bulk-copy engine: one bulk copy per region (sizes
+// multiples of 16 bytes, both addresses 16-byte aligned) tracked by the mbarrier `bar`, then a
+// bounded wait; a false return (in every thread) means a wait gave up, and the caller skips its
+// work, raises a flag and returns.
 constexpr uint32_t kBulkWaitTries = 1u << 22;
+// The first half: thread 0 initialises the mbarrier, announces the bytes and starts the copies;
+// ends with a CTA barrier (the mbarrier is initialised before anyone polls it).
 template <int N>
-__device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void *const (&src)[N],
-                                               const uint32_t (&bytes)[N], unsigned long long *bar,
-                                               uint32_t first_tries = kBulkWaitTries) {
+__device__ __forceinline__ void bulk_load_issue(void *const (&dst)[N], const void *const (&src)[N],
+                                                const uint32_t (&bytes)[N], unsigned long long *bar) {
     const uint32_t b = smem_u32(bar);
     if (threadIdx.x == 0) {
         asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(b) : "memory");
@@ -55,13 +53,27 @@ __device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void
             asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                          ::"r"(smem_u32(dst[i])), "l"(src[i]), "r"(bytes[i]), "r"(b) : "memory");
     }
-    __syncthreads();                               // barrier initialised before anyone polls it
+    __syncthreads();
+}
+// The second half: every thread waits for the bytes, for at most first_tries polls; false in every
+// thread if any wait gave up, after a second wait (at most kBulkWaitTries polls) so that no copy is
+// still writing the shared memory the CTA is about to release.  Ends with a CTA barrier.
+__device__ __forceinline__ bool bulk_load_wait(unsigned long long *bar, uint32_t first_tries) {
+    const uint32_t b = smem_u32(bar);
     bool done = false;
     for (uint32_t it = 0; it < first_tries && !done; it++) done = mbar_try_wait_parity(b, 0);
     if (__syncthreads_and(done) != 0) return true;
     for (uint32_t it = 0; it < kBulkWaitTries && !done; it++) done = mbar_try_wait_parity(b, 0);
     __syncthreads();
     return false;
+}
+// Both halves.
+template <int N>
+__device__ __forceinline__ bool bulk_load_smem(void *const (&dst)[N], const void *const (&src)[N],
+                                               const uint32_t (&bytes)[N], unsigned long long *bar,
+                                               uint32_t first_tries = kBulkWaitTries) {
+    bulk_load_issue(dst, src, bytes, bar);
+    return bulk_load_wait(bar, first_tries);
 }
 
 // int8 x4 -> two half2 (exact): (b ^ 0x80) + 1024 is the fp16 with bits 0x64XX; minus 1152 = b

@@ -10,8 +10,9 @@
 // p) and writes a 16-byte record per block into a shared-memory list, odd-coset records from the
 // front and even-coset records from the back; in phase 2 every warp takes 32 records of one list
 // at a time, so each warp runs one decode path.  The next chunk's packed words load during
-// phase 2.  The sink (DecodeSink) stores the int8 vectors; the fused products of batch 1..7 run in
-// kernels_gemv48.cuh.
+// phase 2.  One kernel body serves two outputs (sinks): the fused product (GemvSink; short row
+// ranges, see kernels_gemv48.cuh for the long ones) and the plain decode to int8 vectors
+// (DecodeSink).
 #pragma once
 #include "kernels.cuh"
 
@@ -28,10 +29,92 @@ constexpr int kBinPer = 5;                        // blocks per thread and chunk
 // code sequence (fetched while classifying), y bits 21..31 = p_S.
 using BinRec = uint4;
 
-// shared memory of the binned kernel: tables, records, counters and mbarrier
+// shared memory of a binned kernel: tables, records, counters and mbarrier, then the sink's own
 __host__ __device__ constexpr size_t bin48_base_smem(int per) {
     return sizeof(Smem48) + sizeof(SmemEven48) + sizeof(BinRec) * kBinThreads * per + 8 * sizeof(int) + 8;
 }
+__host__ __device__ constexpr size_t bin48_smem_bytes(int batch, int rows_per_cta, int per) {
+    return bin48_base_smem(per) + sizeof(float) * (size_t)batch * rows_per_cta * 32;
+}
+
+// y contribution of one decoded block: scale * <v, x_b> for every batch row b, added to the
+// CTA's shared accumulators (slot per lane; warps of the CTA may meet on a slot).
+template <int BATCH>
+__device__ __forceinline__ void accumulate_block(const uint32_t v[6], float scale, const __half *__restrict__ X,
+                                                 long long K, int j, float *acc, int rl, int rows_per_cta,
+                                                 int lane) {
+    uint32_t wh[12];                                           // exact fp16 coordinates, in pairs
+#pragma unroll
+    for (int q = 0; q < 6; q++) i8x4_to_h2x2(v[q], wh[2 * q], wh[2 * q + 1]);
+#pragma unroll
+    for (int bb = 0; bb < BATCH; bb++) {
+        const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
+        float d0 = 0.f, d1 = 0.f;                              // two chains for latency
+#pragma unroll
+        for (int c = 0; c < 3; c++) {
+            const uint4 raw = __ldg(xp + c);
+            d0 = fma2_f16_f32(wh[4 * c + 0], raw.x, d0);
+            d1 = fma2_f16_f32(wh[4 * c + 1], raw.y, d1);
+            d0 = fma2_f16_f32(wh[4 * c + 2], raw.z, d0);
+            d1 = fma2_f16_f32(wh[4 * c + 3], raw.w, d1);
+        }
+        atomicAdd(&acc[(bb * rows_per_cta + rl) * 32 + lane], scale * (d0 + d1));
+    }
+}
+
+// Fused product: a CTA owns rows [row0, row0 + rows_per_cta); block t of the CTA is row t / nb
+// (multiply-high with ceil(2^32 / nb)), column t mod nb; record position = row | column << 16.
+template <int BATCH>
+struct GemvSink {
+    const unsigned long long *words;
+    long long pitch;
+    int rows, nb;
+    uint32_t nb_recip;
+    int gain_mode;
+    const __half *gains, *X;
+    float *Y;
+    int rows_per_cta;
+    // per CTA
+    int row0, nrows;
+    float *acc;
+
+    __device__ void init(unsigned char *extra) {
+        acc = reinterpret_cast<float *>(extra);                 // [BATCH][rows_per_cta][32]
+        for (int i = threadIdx.x; i < BATCH * rows_per_cta * 32; i += kBinThreads) acc[i] = 0.f;
+        row0 = blockIdx.x * rows_per_cta;
+        nrows = max(0, min(rows_per_cta, rows - row0));
+    }
+    __device__ int total() const { return nrows * nb; }
+    __device__ int row_of(int t) const { return nb == 1 ? t : (int)__umulhi((uint32_t)t, nb_recip); }
+    __device__ unsigned long long load(int t) const {
+        const int rl = row_of(t);
+        return __ldg(words + (long long)(row0 + rl) * pitch + (t - rl * nb));
+    }
+    __device__ uint32_t where(int t) const {
+        const int rl = row_of(t);
+        return (uint32_t)rl | (uint32_t)(t - rl * nb) << 16;
+    }
+    __device__ void invalid(int) const {}                       // a bad index contributes nothing
+    __device__ void consume(const uint32_t v[6], uint32_t info, uint32_t z, uint32_t w, const Smem48 &S,
+                            int lane) const {
+        const int rl = (int)(w & 0xFFFFu), j = (int)(w >> 16);
+        const long long row = (long long)row0 + rl;
+        const float scale = gain_mode == 0 ? __half2float(__ldg(gains + row * nb + j))
+                                           : __half2float(__ldg(gains + row * 256 + (z >> 24))) *
+                                                 S.invnorm[info_m(info)];
+        accumulate_block<BATCH>(v, scale, X, (long long)nb * 24, j, acc, rl, rows_per_cta, lane);
+    }
+    __device__ void finish(int lane) const {
+        const int warp = threadIdx.x >> 5;
+        for (int i = warp; i < BATCH * nrows; i += kBinThreads >> 5) {
+            const int bb = i / nrows, rl = i - bb * nrows;
+            float sum = acc[(bb * rows_per_cta + rl) * 32 + lane];
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+            if (lane == 0) Y[(long long)bb * rows + row0 + rl] = sum;
+        }
+    }
+};
 
 // Plain decode: a CTA owns words [base, base + per_cta); record position = t; output int8 [n][24].
 struct DecodeSink {
@@ -93,7 +176,7 @@ __device__ __forceinline__ void bin48_process(const BinRec e, const Smem48 &S, c
 template <class Sink, int PER>
 __global__ void __launch_bounds__(kBinThreads, 1) k_bin48(Dec48::Args args, const SmemEven48 *even,
                                                           const uint32_t *__restrict__ tabC, Sink sink,
-                                                          unsigned *__restrict__ flags) {
+                                                          unsigned *__restrict__ flags, uint32_t wait_tries) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     Smem48 &S = *reinterpret_cast<Smem48 *>(smem_raw);
     SmemEven48 &E = *reinterpret_cast<SmemEven48 *>(smem_raw + sizeof(Smem48));
@@ -122,7 +205,7 @@ __global__ void __launch_bounds__(kBinThreads, 1) k_bin48(Dec48::Args args, cons
         void *const dst[2] = {&S, &E};
         const void *const src[2] = {args.image, even};
         const uint32_t bytes[2] = {(uint32_t)sizeof(Smem48), (uint32_t)sizeof(SmemEven48)};
-        if (!bulk_load_smem(dst, src, bytes, bar)) {
+        if (!bulk_load_smem(dst, src, bytes, bar, wait_tries)) {
             if (threadIdx.x == 0) atomicOr(flags, kFlagWaitTimeout);
             return;
         }

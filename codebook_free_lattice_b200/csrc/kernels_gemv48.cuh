@@ -11,7 +11,12 @@
 // (odd with five magnitude groups, even off the table path) are decoded where they are met.  Each
 // block's product is added to y in global memory by a reduction (no return value), so no warp
 // waits for another: the CTA zeroes its rows of y before its warps start, and a warp that runs out
-// of slices decodes what is left in its rings and exits.
+// of slices decodes what is left in its rings and exits.  An even-coset block's complement code
+// sequence (a global table) is requested when the block is classified and its record is written
+// to the ring one slice later, so the load overlaps the warp's other work.  The table image is
+// copied to shared memory before the kernel waits for the kernels it depends on (programmatic
+// dependent launch), so that copy overlaps the end of the previous kernel on the stream; the
+// activations are staged in shared memory when they fit.
 #pragma once
 #include "kernels_bin48.cuh"
 
@@ -21,21 +26,19 @@ constexpr int kGvThreads = 1024;
 constexpr int kGvWarps = kGvThreads / 32;
 constexpr int kGvRing = 64;                   // records per ring (a warp drains a ring at 32)
 
-// table image, the rings [warp][odd, even][kGvRing], the slice counter and the table mbarrier
+// table image, the rings [warp][odd, even][kGvRing], the slice counter and the table mbarrier,
+// then (when staged) the activations [batch][nb * 24] fp16
 __host__ __device__ constexpr size_t gv48_fixed_smem() {
     return sizeof(SmemGv48) + sizeof(BinRec) * (kGvWarps * 2 * kGvRing) + 16;
 }
-__host__ __device__ constexpr size_t gv48_smem_bytes(int batch, int rows_per_cta) {
-    return gv48_fixed_smem() + 0 * (size_t)batch * rows_per_cta;
+__host__ __device__ constexpr size_t gv48_smem_bytes(int batch, int nb, bool stage_x) {
+    return gv48_fixed_smem() + (stage_x ? (size_t)batch * nb * 48 : 0);
 }
 
 struct GvArgs {
     const SmemGv48 *image;
     unsigned long long npoints;
-    const uint32_t *gweight;                  // Golay codewords by (weight, mask)
-    const uint32_t *tabS;                     // S-side arrangement table (even table path)
     const uint32_t *tabC;                     // complement arrangement table (even table path)
-    const unsigned long long *tail;           // 8-coordinate arrangement table (odd fp16 path)
     const unsigned long long *words;
     long long pitch;
     int rows, nb;
@@ -47,17 +50,18 @@ struct GvArgs {
     uint32_t wait_tries;                      // polls of the table copy's first wait
 };
 
-// The decoded block (12 fp16 pairs, exact small integers) times the activations, scaled.
-template <int BATCH>
+// The decoded block (12 fp16 pairs, exact small integers) times the activations, scaled; the
+// activations from shared memory (XS) or global memory.
+template <int BATCH, bool XS>
 __device__ __forceinline__ void gv_dot(const uint32_t wh[12], float scale, const __half *__restrict__ X,
-                                       long long K, int j, float d[BATCH]) {
+                                       const __half *xs, long long K, int j, float d[BATCH]) {
 #pragma unroll
     for (int bb = 0; bb < BATCH; bb++) {
-        const uint4 *xp = reinterpret_cast<const uint4 *>(X + bb * K + (long long)j * 24);
+        const uint4 *xp = reinterpret_cast<const uint4 *>((XS ? xs : X) + bb * K + (long long)j * 24);
         float d0 = 0.f, d1 = 0.f;
 #pragma unroll
         for (int c = 0; c < 3; c++) {
-            const uint4 raw = __ldg(xp + c);
+            const uint4 raw = XS ? xp[c] : __ldg(xp + c);
             d0 = fma2_f16_f32(wh[4 * c + 0], raw.x, d0);
             d1 = fma2_f16_f32(wh[4 * c + 1], raw.y, d1);
             d0 = fma2_f16_f32(wh[4 * c + 2], raw.z, d0);
@@ -74,53 +78,48 @@ __device__ __forceinline__ void gv_decode(const GvArgs &a, const SmemGv48 &S, co
                                           uint32_t info, uint32_t wh[12]) {
     const unsigned long long p = (unsigned long long)((e.y >> 21) & 1u) << 32 | e.x;
     if constexpr (KIND == 0) {
-        arrange_odd48_f16(S, a.tail, cls, p, r, wh);
+        arrange_odd48_f16(S, cls, p, r, wh);
+    } else if constexpr (KIND == 1) {
+        // x: the complement's code sequence (fetched at classification), y bits 21..31: p_S
+        arrange_even48_f16(S, cls, info, e.y >> 21, r, e.z & 0xFFFFFFu, e.x, wh);
     } else {
-        const uint32_t s = e.z & 0xFFFFFFu;
+        const uint32_t word = (info & kInfoOdd) ? odd_codeword48(S, r)
+                                                : S.gweight[min((S.c_info2[cls] & 0xFFFu) + r, 4095u)];
         uint32_t v[6];
-        if constexpr (KIND == 1) {
-            const Even48Idx ix = even48_indices(S, cls, p);
-            const uint32_t offs = S.c_offs[cls];
-            const uint32_t cS = __ldg(a.tabC + (offs & 0x7FFFFu) + ix.pC);
-            const uint32_t sS = __ldg(a.tabS + (offs >> 19) + ix.pS);
-            const uint32_t word = __ldg(a.gweight + min((S.c_info2[cls] & 0xFFFu) + r, 4095u));
-            even48_merge_word(S, S.merge, info, word, s, sS, cS, v);
-        } else {
-            const uint32_t word = (info & kInfoOdd) ? odd_codeword48(S, r)
-                                                    : __ldg(a.gweight + min((S.c_info2[cls] & 0xFFFu) + r, 4095u));
-            arrange48_word(S, cls, info, word, p, s, true, v);
-        }
+        arrange48_word(S, cls, info, word, p, e.z & 0xFFFFFFu, true, v);
 #pragma unroll
         for (int q = 0; q < 6; q++) i8x4_to_h2x2(v[q], wh[2 * q], wh[2 * q + 1]);
     }
 }
 
-// Decode a record and add its product to y (a reduction in global memory).
-template <int KIND, int BATCH>
-__device__ __forceinline__ void gv_consume(const GvArgs &a, const SmemGv48 &S, const BinRec e, int row0) {
+// Decode a record and add its product to y (a reduction in global memory).  GAIN: 0 direct fp16
+// gain per block, 1 per-row table indexed by the word's gain code.
+template <int KIND, int BATCH, int GAIN, bool XS>
+__device__ __forceinline__ void gv_consume(const GvArgs &a, const SmemGv48 &S, const __half *xs, const BinRec e,
+                                           int row0) {
     const int cls = (int)(e.y & 0x1FFu);
     const uint32_t r = (e.y >> 9) & 0xFFFu;
     const uint32_t info = S.c_info[cls];
     const int rl = (int)(e.w & 0xFFFFu), j = (int)(e.w >> 16);
     const long long row = (long long)row0 + rl;
-    const float scale = a.gain_mode == 0 ? __half2float(__ldg(a.gains + row * a.nb + j))
-                                         : __half2float(__ldg(a.gains + row * 256 + (e.z >> 24))) *
-                                               S.invnorm[info_m(info)];
+    const float scale = GAIN == 0 ? __half2float(__ldg(a.gains + row * a.nb + j))
+                                  : __half2float(__ldg(a.gains + row * 256 + (e.z >> 24))) * S.invnorm[info_m(info)];
     uint32_t wh[12];
     gv_decode<KIND>(a, S, e, cls, r, info, wh);
     float d[BATCH];
-    gv_dot<BATCH>(wh, scale, a.X, (long long)a.nb * 24, j, d);
+    gv_dot<BATCH, XS>(wh, scale, a.X, xs, (long long)a.nb * 24, j, d);
 #pragma unroll
     for (int bb = 0; bb < BATCH; bb++) atomicAdd(a.Y + (long long)bb * a.rows + row, d[bb]);
 }
 
-template <int BATCH>
+template <int BATCH, int GAIN, bool XS>
 __global__ void __launch_bounds__(kGvThreads, 1) k_gemv48(GvArgs a, unsigned *__restrict__ flags) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SmemGv48 &S = *reinterpret_cast<SmemGv48 *>(smem_raw);
     BinRec *rings = reinterpret_cast<BinRec *>(smem_raw + sizeof(SmemGv48));
     int *slice_next = reinterpret_cast<int *>(rings + kGvWarps * 2 * kGvRing);
     unsigned long long *bar = reinterpret_cast<unsigned long long *>(slice_next + 2);
+    __half *xs = reinterpret_cast<__half *>(bar + 1);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const unsigned lanes_below = (1u << lane) - 1u;
@@ -133,21 +132,32 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gemv48(GvArgs a, unsigned *__
     BinRec *ring_odd = rings + warp * 2 * kGvRing;
     BinRec *ring_even = ring_odd + kGvRing;
 
-    for (int i = tid; i < BATCH * nrows; i += kGvThreads) {
-        const int bb = i / nrows, rr = i - bb * nrows;
-        a.Y[(long long)bb * a.rows + row0 + rr] = 0.f;
-    }
+    // the next kernel on the stream may start its own table copy now; it waits (as this one does
+    // below) for the kernels before it to finish before it touches their results
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (tid == 0) *slice_next = kGvWarps;      // slices 0..31 go to warps 0..31 directly
-    // the table image by one bulk copy; the call ends with a CTA barrier, which also orders the
-    // zeroed rows of y before any reduction into them
     {
         void *const dst[1] = {&S};
         const void *const src[1] = {a.image};
         const uint32_t bytes[1] = {(uint32_t)sizeof(SmemGv48)};
-        if (!bulk_load_smem(dst, src, bytes, bar, a.wait_tries)) {
-            if (tid == 0) atomicOr(flags, kFlagWaitTimeout);
-            return;
-        }
+        bulk_load_issue(dst, src, bytes, bar);
+    }
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    for (int i = tid; i < BATCH * nrows; i += kGvThreads) {
+        const int bb = i / nrows, rr = i - bb * nrows;
+        a.Y[(long long)bb * a.rows + row0 + rr] = 0.f;
+    }
+    if constexpr (XS) {
+        const int n16 = BATCH * nb * 3;                             // 16-byte units
+        const uint4 *src = reinterpret_cast<const uint4 *>(a.X);
+        uint4 *dst = reinterpret_cast<uint4 *>(xs);
+        for (int i = tid; i < n16; i += kGvThreads) dst[i] = __ldg(src + i);
+    }
+    // the table copy's wait ends with a CTA barrier, which also orders the zeroed rows of y before
+    // any reduction into them and the staged activations before their use
+    if (!bulk_load_wait(bar, a.wait_tries)) {
+        if (tid == 0) atomicOr(flags, kFlagWaitTimeout);
+        return;
     }
 
     const bool dense = a.pitch == (long long)nb;
@@ -161,6 +171,28 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gemv48(GvArgs a, unsigned *__
 
     bool bad = false;
     int oh = 0, ot = 0, eh = 0, et = 0;       // ring heads and tails (warp-uniform)
+    // the previous slice's record, written to its ring one slice late (pk: 0 odd, 1 even, 3 none)
+    BinRec prec;
+    int pk = 3;
+    prec.x = prec.y = prec.z = prec.w = 0u;
+    auto append = [&](const BinRec &rec, int k) {
+        const unsigned mo = __ballot_sync(0xFFFFFFFFu, k == 0);
+        const unsigned me = __ballot_sync(0xFFFFFFFFu, k == 1);
+        if (k == 0) ring_odd[(ot + __popc(mo & lanes_below)) & (kGvRing - 1)] = rec;
+        if (k == 1) ring_even[(et + __popc(me & lanes_below)) & (kGvRing - 1)] = rec;
+        ot += __popc(mo);
+        et += __popc(me);
+        __syncwarp();
+        if (ot - oh >= 32) {
+            gv_consume<0, BATCH, GAIN, XS>(a, S, xs, ring_odd[(oh + lane) & (kGvRing - 1)], row0);
+            oh += 32;
+        }
+        if (et - eh >= 32) {
+            gv_consume<1, BATCH, GAIN, XS>(a, S, xs, ring_even[(eh + lane) & (kGvRing - 1)], row0);
+            eh += 32;
+        }
+        __syncwarp();
+    };
     int sl = warp;                             // current slice (warp-uniform)
     unsigned long long w = sl < nslices ? word_at(sl * 32 + lane) : 0ull;
     while (sl < nslices) {
@@ -169,42 +201,38 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gemv48(GvArgs a, unsigned *__
         sn = __shfl_sync(0xFFFFFFFFu, sn, 0);
         const unsigned long long wn = sn < nslices ? word_at(sn * 32 + lane) : 0ull;
         const int t = sl * 32 + lane;
-        // classify this slice and append the records
+        // classify this slice; an even block on the table path requests its complement sequence
         const bool valid = t < total;
         const Cls48 cl = classify48(w, S, a.npoints);
         bad |= valid && !cl.ok;
         const bool enq = valid && cl.ok;
         const bool odd = cl.info & kInfoOdd;
-        const int kind = odd ? (info_val4(cl.info) == 0u ? 0 : 2) : ((cl.info & kInfoTable) ? 1 : 2);
+        int kind = odd ? (info_val4(cl.info) == 0u ? 0 : 2) : ((cl.info & kInfoTable) ? 1 : 2);
+        if (!enq) kind = 3;
         const int rl = valid ? (nb == 1 ? t : (int)__umulhi((uint32_t)t, a.nb_recip)) : 0;
         BinRec rec;
         rec.x = (uint32_t)cl.p;
         rec.y = (uint32_t)cl.cls | cl.r << 9 | (uint32_t)(cl.p >> 32) << 21;
         rec.z = cl.s | (uint32_t)((w >> 48) & 0xFFu) << 24;
         rec.w = (uint32_t)rl | (uint32_t)(t - rl * nb) << 16;
-        const unsigned mo = __ballot_sync(0xFFFFFFFFu, enq && kind == 0);
-        const unsigned me = __ballot_sync(0xFFFFFFFFu, enq && kind == 1);
-        if (enq && kind == 0) ring_odd[(ot + __popc(mo & lanes_below)) & (kGvRing - 1)] = rec;
-        if (enq && kind == 1) ring_even[(et + __popc(me & lanes_below)) & (kGvRing - 1)] = rec;
-        if (enq && kind == 2) gv_consume<2, BATCH>(a, S, rec, row0);
-        ot += __popc(mo);
-        et += __popc(me);
-        __syncwarp();
-        if (ot - oh >= 32) {
-            gv_consume<0, BATCH>(a, S, ring_odd[(oh + lane) & (kGvRing - 1)], row0);
-            oh += 32;
+        if (kind == 1) {
+            uint32_t pS;
+            const uint32_t pC = even48_pC(S, cl.cls, (uint32_t)cl.p, pS);
+            rec.x = __ldg(a.tabC + (S.c_offs[cl.cls] & 0x7FFFFu) + pC);
+            rec.y = (uint32_t)cl.cls | cl.r << 9 | pS << 21;
         }
-        if (et - eh >= 32) {
-            gv_consume<1, BATCH>(a, S, ring_even[(eh + lane) & (kGvRing - 1)], row0);
-            eh += 32;
-        }
-        __syncwarp();
+        if (kind == 2) gv_consume<2, BATCH, GAIN, XS>(a, S, xs, rec, row0);
+        // the previous slice's records into the rings, full batches decoded
+        append(prec, pk);
+        prec = rec;
+        pk = kind;
         w = wn;
         sl = sn;
     }
+    append(prec, pk);
     // what is left in the rings
-    if (lane < ot - oh) gv_consume<0, BATCH>(a, S, ring_odd[(oh + lane) & (kGvRing - 1)], row0);
-    if (lane < et - eh) gv_consume<1, BATCH>(a, S, ring_even[(eh + lane) & (kGvRing - 1)], row0);
+    if (lane < ot - oh) gv_consume<0, BATCH, GAIN, XS>(a, S, xs, ring_odd[(oh + lane) & (kGvRing - 1)], row0);
+    if (lane < et - eh) gv_consume<1, BATCH, GAIN, XS>(a, S, xs, ring_even[(eh + lane) & (kGvRing - 1)], row0);
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(flags, kFlagIndexRange);
 }
 

@@ -66,11 +66,12 @@ __device__ __forceinline__ void tc48_store_a(Tc48Smem &T, int dr, int jj, const 
             make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
 }
 
-// bounded wait for the round's MMAs; the result is the same in every lane of the warp, so the
-// warp-collective TMEM load that follows is taken by all lanes or by none
-__device__ __forceinline__ bool tc48_wait_mma(Tc48Smem &T, uint32_t phase) {
+// bounded wait for the round's MMAs (at most `tries` polls); the result is the same in every lane
+// of the warp, so the warp-collective TMEM load that follows is taken by all lanes or by none
+constexpr uint32_t kMmaWaitTries = 1u << 20;
+__device__ __forceinline__ bool tc48_wait_mma(Tc48Smem &T, uint32_t phase, uint32_t tries) {
     bool done = false;
-    for (int it = 0; it < (1 << 20) && !done; it++) done = mbar_try_wait_parity(smem_u32(&T.mbar_mma), phase);
+    for (uint32_t it = 0; it < tries && !done; it++) done = mbar_try_wait_parity(smem_u32(&T.mbar_mma), phase);
     return __all_sync(0xFFFFFFFFu, done);
 }
 
@@ -91,7 +92,7 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
     Dec48::Args args, const SmemEven48 *even, const uint32_t *__restrict__ tabC,
     const unsigned long long *__restrict__ words, long long pitch, int rows, int nb, int batch, int gain_mode,
     const __half *__restrict__ gains, const __half *__restrict__ X, float *__restrict__ Y, int rounds_per_split,
-    unsigned *__restrict__ flags) {
+    unsigned *__restrict__ flags, uint32_t table_tries, uint32_t mma_tries) {
     extern __shared__ __align__(128) unsigned char smem_tc48[];
     Smem48 &S = *reinterpret_cast<Smem48 *>(smem_tc48);
     SmemEven48 &E = *reinterpret_cast<SmemEven48 *>(smem_tc48 + sizeof(Smem48));
@@ -149,7 +150,7 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
         void *const dst[2] = {&S, &E};
         const void *const src[2] = {args.image, even};
         const uint32_t bytes[2] = {(uint32_t)sizeof(Smem48), (uint32_t)sizeof(SmemEven48)};
-        if (!bulk_load_smem(dst, src, bytes, &T.mbar_load)) {
+        if (!bulk_load_smem(dst, src, bytes, &T.mbar_load, table_tries)) {
             if (tid == 0) atomicOr(flags, kFlagWaitTimeout);
             return;                                           // no TMEM allocated yet
         }
@@ -172,6 +173,9 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
     for (int b = 0; b < 16; b++) yacc[b] = 0.f;
     bool bad = false;
     uint32_t phase = 0;
+    // committed MMAs not yet waited for by this warp, and their phase parity
+    bool pending = false;
+    uint32_t pphase = 0;
 
     for (int ch = c0; ch < c1; ch++) {
         const int j0 = ch * kTc48Slots;
@@ -222,7 +226,8 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
         const uint4 xnow = load_x(ch);                          // L2-resident; lands during the wait
         // ---- 2. the previous round's products: bounded wait, then the epilogue
         if (ch > c0) {
-            if (tc48_wait_mma(T, phase)) {
+            if (tc48_wait_mma(T, phase, mma_tries)) {
+                pending = false;
                 tc_fence_after();
                 tc48_epilogue(etaddr, gep, yacc);
             } else if (lane == 0) {
@@ -291,12 +296,15 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
             asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
                          ::"r"(smem_u32(&T.mbar_mma)) : "memory");
         }
+        pending = true;
+        pphase = phase;
     }
     // ---- the last round's products (T.status is uniform here: nothing wrote it since the
     // last barrier)
     if (c0 < c1 && !T.status) {
         const float gep = T.gain[eslot][em];
-        if (tc48_wait_mma(T, phase)) {
+        if (tc48_wait_mma(T, phase, mma_tries)) {
+            pending = false;
             tc_fence_after();
             tc48_epilogue(etaddr, gep, yacc);
         } else if (lane == 0) {
@@ -319,7 +327,15 @@ __global__ void __launch_bounds__(kTc48Threads, 1) k_gemm_tc48(
     }
     if (tid == 0 && T.status) atomicOr(flags, kFlagWaitTimeout);
     if (__any_sync(0xFFFFFFFFu, bad) && lane == 0) atomicOr(flags, kFlagIndexRange);
-    // ---- free the accumulator columns (all TMEM reads have completed above)
+    // ---- free the accumulator columns.  After a wait gave up, the committed MMAs may still be
+    // writing them: every thread waits again (at most kMmaWaitTries polls) for the last commit,
+    // and the columns are released only if it arrived; otherwise they are left allocated (the
+    // flag is raised) rather than freed under the running MMAs.
+    if (__syncthreads_or(pending)) {
+        bool done = false;
+        for (uint32_t it = 0; it < kMmaWaitTries && !done; it++) done = mbar_try_wait_parity(smem_u32(&T.mbar_mma), pphase);
+        if (!__syncthreads_and(done)) return;
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();

@@ -46,9 +46,6 @@ struct llvq_codec {
     void *d_even48 = nullptr;      // SmemEven48 image (48-bit table path)
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
     void *d_gv48 = nullptr;        // SmemGv48 image (48-bit fused products, k_gemv48)
-    unsigned long long *d_tail48 = nullptr;  // 8-coordinate arrangement table (odd-coset fp16 path)
-    uint32_t *d_gweight48 = nullptr;  // Golay codewords by (weight, mask), global copy for k_gemv48
-    uint32_t *d_tabS48 = nullptr;  // S-side arrangement table, global copy for k_gemv48
     void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
     void *d_enc72 = nullptr;       // EncSmem72 image (72-bit encoder)
     unsigned long long *d_keys72 = nullptr;  // 72-bit class keys (encoder)
@@ -60,11 +57,18 @@ struct llvq_codec {
 namespace {
 
 thread_local std::string g_last_error;
-std::atomic<uint32_t> g_first_wait_tries{kBulkWaitTries};   // polls of a kernel's first table-copy wait
+// polls of a kernel's first bounded wait on its table copy and on its tensor-core products
+// (llvq_set_wait_polls; tests set them to 0 to take the timeout paths)
+std::atomic<uint32_t> g_first_wait_tries{kBulkWaitTries};
+std::atomic<uint32_t> g_mma_wait_tries{kMmaWaitTries};
 
 // 48-bit batches from this size up run on the tensor cores (k_gemm_tc48); smaller ones, and every
 // 72/96-bit batch, on the CUDA cores
 constexpr int kTensorCoreMinBatch = 8;
+// 48-bit batch 1-2 products with at least this many blocks per SM run the warp-binned kernel
+// (k_gemv48): 4-9% faster than the coset-sorted kernel on B200 from 11008x4104 up, slower on
+// 4096x4104 (4.7k blocks per SM) and at batch 4
+constexpr long long kWarpBinnedMinBlocks = 10000;
 
 // smallest double >= n / d for small positive integers (directed rounding of the host division)
 double round_up_ratio(double n, double d) {
@@ -228,9 +232,9 @@ llvq_status build_even48(const HostTables &T, Smem48 &S, SmemEven48 &E, std::vec
 
 // The image of the fused product kernel (SmemGv48), assembled from the decode image and the
 // even-coset tables, plus the tables of the odd-coset fp16 path: the tail table of every multiset
-// of 8 items over 4 groups, per-class cumulative counts and fp16 values on T, the pair sign masks
-// of a byte of T, and the low codeword bits as a linear function of the top 12 (checked against
-// the whole code).
+// of 6 items over 4 groups, per-class cumulative counts and fp16 values on T, the pair sign masks
+// of a nibble of negative flags, and the low codeword bits as a linear function of the top 12
+// (checked against the whole code).
 uint16_t fp16_bits(int v) {
     // exact for |v| <= 2048: sign, exponent, 10-bit mantissa
     if (v == 0) return 0;
@@ -241,8 +245,7 @@ uint16_t fp16_bits(int v) {
     return (uint16_t)(sign | (uint16_t)((e + 15) << 10) | (uint16_t)mant);
 }
 
-llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E, SmemGv48 &G,
-                       std::vector<unsigned long long> &tail, std::string &err) {
+llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E, SmemGv48 &G, std::string &err) {
     std::memset(&G, 0, sizeof G);
     std::memcpy(G.starts, S.starts, sizeof G.starts);
     std::memcpy(G.c_invA, S.c_invA, sizeof G.c_invA);
@@ -256,12 +259,32 @@ llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E
     std::memcpy(G.c_vals, S.c_vals, sizeof G.c_vals);
     std::memcpy(G.c_gflag, S.c_gflag, sizeof G.c_gflag);
     std::memcpy(G.invnorm, S.invnorm, sizeof G.invnorm);
-    std::memcpy(G.merge, E.merge, sizeof G.merge);
+    std::memcpy(G.tabS, E.tabS, sizeof G.tabS);
+    std::memcpy(G.gweight, S.golay_weight, sizeof G.gweight);
+    // even-coset fp16 merge: selectors (z, |x|/2) per coordinate, z = 8 on a nonzero coordinate
+    for (uint32_t mq = 0; mq < 16; mq++)
+        for (uint32_t bits = 0; bits < 256; bits++) {
+            const int n2 = 2 * __builtin_popcount(mq);
+            uint32_t sb = bits & ((1u << n2) - 1u), cb = bits >> n2, e = 0;
+            for (int pos = 0; pos < 4; pos++) {
+                uint32_t mag;
+                if (mq >> pos & 1u) { mag = 2 + 4 * (sb & 3u); sb >>= 2; }
+                else { mag = 4 * (cb & 3u); cb >>= 2; }
+                const uint32_t sel = (mag != 0 ? 8u : 0u) | (mag / 2) << 4;   // nibbles z, |x|/2
+                e |= sel << (8 * pos);
+            }
+            G.merge16[mq << 8 | bits] = e;
+        }
+    for (size_t i = 0; i < T.classes.size(); i++) {
+        const HostClass &c = T.classes[i];
+        if (c.odd || !(S.c_info[i] & kInfoTable)) continue;
+        G.c_magS[i] = c.P_S == 1 ? 0u : (uint32_t)((((u128)1 << 32) + c.P_S - 1) / c.P_S);
+    }
     std::memcpy(G.guide, S.guide, sizeof S.guide);
     std::memcpy(G.pdep_off, S.pdep_off, sizeof G.pdep_off);
     std::memcpy(G.pdep, S.pdep, sizeof S.pdep);
-    // tail: multisets (n0, n1, n2, n3) of 8 items, arrangements lexicographic over groups 0 < 1 < 2 < 3
-    tail.clear();
+    // tail: multisets (n0, n1, n2, n3) of 6 items, arrangements lexicographic over groups 0 < 1 < 2 < 3
+    uint32_t ntail = 0;
     for (int c0 = 0; c0 <= kOddTail48; c0++)
         for (int c1 = c0; c1 <= kOddTail48; c1++)
             for (int c2 = c1; c2 <= kOddTail48; c2++) {
@@ -269,15 +292,16 @@ llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E
                 std::vector<int> seq;
                 for (int g = 0; g < 4; g++)
                     for (int t = 0; t < n[g]; t++) seq.push_back(g);
-                const uint32_t off = (uint32_t)tail.size();
+                const uint32_t off = ntail;
                 do {
-                    unsigned long long e = 0;
-                    for (int k = 0; k < kOddTail48; k++) e |= (unsigned long long)(0x10 + 0x22 * seq[k]) << (8 * k);
-                    tail.push_back(e);
+                    uint32_t e = 0;
+                    for (int k = 0; k < kOddTail48; k++) e |= (uint32_t)seq[k] << (2 * k);
+                    if (ntail >= 4096) { err = "odd tail table overflow"; return LLVQ_ERR_UNSUPPORTED; }
+                    G.tail[ntail++] = (uint16_t)e;
                 } while (std::next_permutation(seq.begin(), seq.end()));
-                G.tailc[c0 + 9 * c1 + 81 * c2] = make_uint2(off, (uint32_t)(tail.size() - off));
+                G.tailc[c0 + 7 * c1 + 49 * c2] = make_uint2(off, ntail - off);
             }
-    if (tail.size() != 65536) { err = "odd tail table size"; return LLVQ_ERR_UNSUPPORTED; }
+    if (ntail != 4096) { err = "odd tail table size"; return LLVQ_ERR_UNSUPPORTED; }
     for (size_t i = 0; i < T.classes.size(); i++) {
         const HostClass &c = T.classes[i];
         if (!c.odd || c.vals.size() > 4) continue;
@@ -291,12 +315,9 @@ llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E
         G.c_vt[i][0] = vt[0];
         G.c_vt[i][1] = vt[1];
     }
-    for (int tb = 0; tb < 256; tb++) {
-        uint32_t m[4];
-        for (int j = 0; j < 4; j++)
-            m[j] = ((tb >> (2 * j) & 1) ? 0u : 0x8000u) | ((tb >> (2 * j + 1) & 1) ? 0u : 0x80000000u);
-        G.tsign[tb] = make_uint4(m[0], m[1], m[2], m[3]);
-    }
+    for (int nb = 0; nb < 16; nb++)                        // bit k: coordinate k of the nibble negative
+        G.nsign[nb] = make_uint2(((nb & 1) ? 0x8000u : 0u) | ((nb & 2) ? 0x80000000u : 0u),
+                                 ((nb & 4) ? 0x8000u : 0u) | ((nb & 8) ? 0x80000000u : 0u));
     for (int j = 0; j < 64; j++) {
         G.tlow[j] = (uint16_t)(T.golay_by_mask[j] & 0xFFFu);
         G.tlow[64 + j] = (uint16_t)(T.golay_by_mask[j << 6] & 0xFFFu);
@@ -636,7 +657,7 @@ cudaError_t launch_decode(const llvq_codec *c, typename D::Args a, const void *w
         sink.out = out;
         sink.per_cta = per;
         k_bin48<DecodeSink, kBinPer><<<grid, kBinThreads, bin48_base_smem(kBinPer), st>>>(
-            a, (const SmemEven48 *)c->d_even48, c->d_tabC48, sink, c->d_flags);
+            a, (const SmemEven48 *)c->d_even48, c->d_tabC48, sink, c->d_flags, g_first_wait_tries.load());
         return cudaGetLastError();
     }
     const int threads = 512;
@@ -675,9 +696,49 @@ void set_gemm_attrs(std::integer_sequence<int, Bs...>) {
 
 constexpr size_t kBinSmemLimit = 232448;          // opt-in shared memory per block on sm_100
 
-void set_bin48_attrs() {
+template <int... Bs>
+void set_bin48_attrs(std::integer_sequence<int, Bs...>) {
+    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_bin48<GemvSink<Bs + 1>, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                          (int)kBinSmemLimit), ...);
     cudaFuncSetAttribute(k_bin48<DecodeSink, kBinPer>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)kBinSmemLimit);
+}
+
+// The coset-sorted product (k_bin48 with GemvSink): one CTA per SM over a row range, the whole
+// range classified in chunks of up to 5 blocks per thread.
+template <int B>
+cudaError_t launch_gemm_bin48(const llvq_codec *c, Dec48::Args a, const llvq_weight *w, const void *X, float *Y,
+                              cudaStream_t st) {
+    const int nb = w->blocks_per_row;
+    if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
+    // one CTA per SM over a row range; 5 blocks per thread and chunk when the row accumulators
+    // leave room, else 4, else the row range shrinks (more CTAs than SMs)
+    int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
+    int per = bin48_smem_bytes(B, rpc, 5) <= kBinSmemLimit ? 5 : 4;
+    while (rpc > 1 && bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) rpc = (rpc + 1) / 2;
+    if (bin48_smem_bytes(B, rpc, per) > kBinSmemLimit) return cudaErrorInvalidValue;
+    // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
+    if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
+    const int grid = (w->rows + rpc - 1) / rpc;
+    const uint32_t recip = nb > 1 ? (uint32_t)(((1ull << 32) + nb - 1) / nb) : 0u;
+    GemvSink<B> sink{};
+    sink.words = (const unsigned long long *)w->words;
+    sink.pitch = w->row_pitch_words;
+    sink.rows = w->rows;
+    sink.nb = nb;
+    sink.nb_recip = recip;
+    sink.gain_mode = w->gain_mode;
+    sink.gains = (const __half *)w->gains;
+    sink.X = (const __half *)X;
+    sink.Y = Y;
+    sink.rows_per_cta = rpc;
+    auto kern = per == 5 ? k_bin48<GemvSink<B>, 5> : k_bin48<GemvSink<B>, 4>;
+    kern<<<grid, kBinThreads, bin48_smem_bytes(B, rpc, per), st>>>(a, (const SmemEven48 *)c->d_even48,
+                                                                  c->d_tabC48, sink, c->d_flags,
+                                                                  g_first_wait_tries.load());
+    return cudaGetLastError();
 }
 
 // 48-bit products of batch 1..7 (k_gemv48): one CTA per SM over a row range; the row range
@@ -687,20 +748,15 @@ cudaError_t launch_gemv48(const llvq_codec *c, Dec48::Args a, const llvq_weight 
                           cudaStream_t st) {
     const int nb = w->blocks_per_row;
     if (nb > 0xFFFF) return cudaErrorInvalidValue;                  // column field of a record
-    int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
-    while (rpc > 1 && gv48_smem_bytes(B, rpc) > kBinSmemLimit) rpc = (rpc + 1) / 2;
-    if (gv48_smem_bytes(B, rpc) > kBinSmemLimit) return cudaErrorInvalidValue;
+    const int rpc = std::max(1, (w->rows + c->num_sms - 1) / c->num_sms);
     if (rpc > 0xFFFF) return cudaErrorInvalidValue;                 // row field of a record
     // block index -> row by a multiply-high: exact while rpc * nb < 2^32 / nb
     if ((unsigned long long)rpc * nb * nb >= (1ull << 32)) return cudaErrorInvalidValue;
-    const int grid = (w->rows + rpc - 1) / rpc;
+    const size_t smem = gv48_smem_bytes(B, nb, false);   // activations read through L1
     GvArgs g{};
     g.image = (const SmemGv48 *)c->d_gv48;
     g.npoints = a.npoints;
-    g.gweight = c->d_gweight48;
-    g.tabS = c->d_tabS48;
     g.tabC = c->d_tabC48;
-    g.tail = c->d_tail48;
     g.words = (const unsigned long long *)w->words;
     g.pitch = w->row_pitch_words;
     g.rows = w->rows;
@@ -712,13 +768,31 @@ cudaError_t launch_gemv48(const llvq_codec *c, Dec48::Args a, const llvq_weight 
     g.Y = Y;
     g.rows_per_cta = rpc;
     g.wait_tries = g_first_wait_tries.load();
-    k_gemv48<B><<<grid, kGvThreads, gv48_smem_bytes(B, rpc), st>>>(g, c->d_flags);
-    return cudaGetLastError();
+    // programmatic dependent launch: this kernel's table copy may overlap the end of the previous
+    // kernel on the stream (the kernel waits for it before touching any data)
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((w->rows + rpc - 1) / rpc));
+    cfg.blockDim = dim3(kGvThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    unsigned *flags = c->d_flags;
+    const bool direct = w->gain_mode == LLVQ_GAIN_FP16_DIRECT;
+    if (direct) return cudaLaunchKernelEx(&cfg, k_gemv48<B, 0, false>, g, flags);
+    return cudaLaunchKernelEx(&cfg, k_gemv48<B, 1, false>, g, flags);
 }
 
 template <int... Bs>
 void set_gemv48_attrs(std::integer_sequence<int, Bs...>) {
-    (cudaFuncSetAttribute(k_gemv48<Bs + 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+
+
+    (cudaFuncSetAttribute(k_gemv48<Bs + 1, 0, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+    (cudaFuncSetAttribute(k_gemv48<Bs + 1, 1, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBinSmemLimit), ...);
+
 }
 
 // 48-bit tensor-core path: 128-row tiles x K splits of 8-block rounds.  The split is chosen to
@@ -742,7 +816,7 @@ cudaError_t launch_gemm_tc48(const llvq_codec *c, Dec48::Args a, const llvq_weig
     k_gemm_tc48<<<dim3(mt, splits), kTc48Threads, tc48_smem_bytes(), st>>>(
         a, (const SmemEven48 *)c->d_even48, c->d_tabC48, (const unsigned long long *)w->words, w->row_pitch_words,
         w->rows, w->blocks_per_row, batch, w->gain_mode, (const __half *)w->gains, (const __half *)X, Y, best_rps,
-        c->d_flags);
+        c->d_flags, g_first_wait_tries.load(), g_mma_wait_tries.load());
     return cudaGetLastError();
 }
 
@@ -757,14 +831,19 @@ cudaError_t gemm_dispatch(const llvq_codec *c, typename D::Args a, const llvq_we
         else return launch_gemm<D, 16>(c, a, w, X, Y, s, batch);
     }
     if constexpr (std::is_same<D, Dec48>::value) {
+        // long row ranges (>= kWarpBinnedMinBlocks blocks per SM) at batch 1 and 2: the warp-binned
+        // kernel; shorter ranges and larger batches: the coset-sorted kernel (measured on B200)
+        const long long per_sm = (long long)((w->rows + c->num_sms - 1) / c->num_sms) * w->blocks_per_row;
+        if (per_sm >= kWarpBinnedMinBlocks && batch <= 2)
+            return batch == 1 ? launch_gemv48<1>(c, a, w, X, Y, s) : launch_gemv48<2>(c, a, w, X, Y, s);
         switch (batch) {
-            case 1: return launch_gemv48<1>(c, a, w, X, Y, s);
-            case 2: return launch_gemv48<2>(c, a, w, X, Y, s);
-            case 3: return launch_gemv48<3>(c, a, w, X, Y, s);
-            case 4: return launch_gemv48<4>(c, a, w, X, Y, s);
-            case 5: return launch_gemv48<5>(c, a, w, X, Y, s);
-            case 6: return launch_gemv48<6>(c, a, w, X, Y, s);
-            default: return launch_gemv48<7>(c, a, w, X, Y, s);
+            case 1: return launch_gemm_bin48<1>(c, a, w, X, Y, s);
+            case 2: return launch_gemm_bin48<2>(c, a, w, X, Y, s);
+            case 3: return launch_gemm_bin48<3>(c, a, w, X, Y, s);
+            case 4: return launch_gemm_bin48<4>(c, a, w, X, Y, s);
+            case 5: return launch_gemm_bin48<5>(c, a, w, X, Y, s);
+            case 6: return launch_gemm_bin48<6>(c, a, w, X, Y, s);
+            default: return launch_gemm_bin48<7>(c, a, w, X, Y, s);
         }
     } else {
         switch (batch) {
@@ -841,8 +920,8 @@ void set_kernel_attrs() {
     std::call_once(once, [] {
         cudaFuncSetAttribute(k_decode<Dec48>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem48));
         cudaFuncSetAttribute(k_decode<Dec72>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(Smem72));
-        set_bin48_attrs();
-        set_gemv48_attrs(std::make_integer_sequence<int, 7>{});
+        set_bin48_attrs(std::make_integer_sequence<int, 7>{});
+        set_gemv48_attrs(std::make_integer_sequence<int, 2>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
         cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
         cudaFuncSetAttribute(k_encode96, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem96));
@@ -919,6 +998,11 @@ llvq_status llvq_decode_noalloc(int32_t index_bits, const void *d_words, int32_t
 
 const char *llvq_last_error_message(void) { return g_last_error.c_str(); }
 
+void llvq_set_wait_polls(uint32_t table_polls, uint32_t mma_polls) {
+    g_first_wait_tries.store(table_polls == 0xFFFFFFFFu ? kBulkWaitTries : table_polls);
+    g_mma_wait_tries.store(mma_polls == 0xFFFFFFFFu ? kMmaWaitTries : mma_polls);
+}
+
 llvq_status llvq_class_table96(int32_t m, llvq_class96 *out, int64_t capacity, int64_t *n_classes) {
     static_assert(sizeof(llvq_class96) == sizeof(Rec96), "llvq_class96 mirrors Rec96");
     static std::mutex mu;
@@ -972,7 +1056,6 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::vector<uint32_t> guide, tabC;
     std::vector<unsigned char> even(sizeof(SmemEven48));
     std::vector<unsigned char> gv(sizeof(SmemGv48));
-    std::vector<unsigned long long> tail48;
     std::vector<unsigned char> enc(sizeof(EncSmem48));
     std::vector<unsigned char> enc72(sizeof(EncSmem72));
     std::vector<unsigned long long> keys72;
@@ -985,7 +1068,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
                               tabC, err);
         if (st == LLVQ_OK)
             st = build_gv48(T, *reinterpret_cast<const Smem48 *>(image.data()), *reinterpret_cast<const SmemEven48 *>(even.data()),
-                            *reinterpret_cast<SmemGv48 *>(gv.data()), tail48, err);
+                            *reinterpret_cast<SmemGv48 *>(gv.data()), err);
         if (st == LLVQ_OK) st = build_enc48(T, *reinterpret_cast<EncSmem48 *>(enc.data()), err);
     } else {
         image.resize(sizeof(Smem72));
@@ -1013,15 +1096,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
               cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&c->d_gv48, gv.size()) == cudaSuccess &&
               cudaMemcpy(c->d_gv48, gv.data(), gv.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
-              cudaMalloc(&c->d_gweight48, 4096 * sizeof(uint32_t)) == cudaSuccess &&
-              cudaMemcpy(c->d_gweight48, reinterpret_cast<const Smem48 *>(image.data())->golay_weight, 4096 * sizeof(uint32_t),
-                         cudaMemcpyHostToDevice) == cudaSuccess &&
-              cudaMalloc(&c->d_tabS48, kTabS48 * sizeof(uint32_t)) == cudaSuccess &&
-              cudaMemcpy(c->d_tabS48, reinterpret_cast<const SmemEven48 *>(even.data())->tabS, kTabS48 * sizeof(uint32_t),
-                         cudaMemcpyHostToDevice) == cudaSuccess &&
-              cudaMalloc(&c->d_tail48, tail48.size() * sizeof(unsigned long long)) == cudaSuccess &&
-              cudaMemcpy(c->d_tail48, tail48.data(), tail48.size() * sizeof(unsigned long long),
-                         cudaMemcpyHostToDevice) == cudaSuccess;
+
+              true;
     }
     if (okc && index_bits == 72) {
         okc = cudaMalloc(&c->d_recs72, recs.size() * sizeof(Rec72)) == cudaSuccess &&
@@ -1060,9 +1136,7 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_keys96) cudaFree(c->d_keys96);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
     if (c->d_gv48) cudaFree(c->d_gv48);
-    if (c->d_gweight48) cudaFree(c->d_gweight48);
-    if (c->d_tabS48) cudaFree(c->d_tabS48);
-    if (c->d_tail48) cudaFree(c->d_tail48);
+
     delete c;
 }
 

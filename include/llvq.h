@@ -56,8 +56,8 @@ typedef enum {
 
 /* Sticky device flags returned by llvq_get_error. */
 #define LLVQ_FLAG_INDEX_RANGE 0x1u  /* some index was >= N_M (its block decoded to zero) */
-#define LLVQ_FLAG_WAIT_TIMEOUT 0x2u /* a bounded wait for the tensor cores gave up; the output of
-                                       that call is incomplete */
+#define LLVQ_FLAG_WAIT_TIMEOUT 0x2u /* a bounded wait (table copy, tensor-core products) gave up;
+                                       the output of that call is incomplete */
 #define LLVQ_FLAG_NOT_CODED 0x4u    /* llvq_encode met a vector that is not a coded lattice point */
 
 /* Opaque codec: owns the decode tables of one index budget on one device. */
@@ -185,6 +185,16 @@ const char *llvq_status_string(llvq_status status);
 /* The reason of the last failed call on this thread that gave one (table construction, device
  * memory), or an empty string.  Valid until the next call on this thread. */
 const char *llvq_last_error_message(void);
+
+/* Limits of the kernels' bounded waits, for tests of the timeout paths.  The paper has no
+ * counterpart.  A kernel waits at most table_polls polls for its table copy into shared memory
+ * and at most mma_polls polls for each round of its tensor-core products (tcgen05.mma completion);
+ * when a wait gives up the kernel raises LLVQ_FLAG_WAIT_TIMEOUT (read by llvq_get_error), skips
+ * the rest of its work (its outputs are then unspecified), and before it exits waits again, up to
+ * the default limit, for the copy or the products in flight, so that nothing is still writing the
+ * memory it releases.  0 makes the first wait give up at once; 0xFFFFFFFF restores the defaults
+ * (2^22 and 2^20 polls).  Applies to launches made after the call, process-wide. */
+void llvq_set_wait_polls(uint32_t table_polls, uint32_t mma_polls);
 
 #ifdef __cplusplus
 }
