@@ -33,12 +33,21 @@ METRIC = "fused 2-bit LLVQ GEMV effective GB/s and % of HBM roofline; decoded ve
 ROWS, K = 4096, 4096
 NB = -(-K // 24)
 CONFIG_ID = 2
-WORKLOAD = "llvq 2-bit fused GEMV, 4096x4096 layer (K padded to 4104), u8 gain table, batch 1"
 
 
-def algorithmic_bytes(rows=ROWS, nb=NB, batch=1) -> int:
+def workload(rows=None, cols=None, batch=1) -> str:
+    rows, cols = rows or ROWS, cols or K
+    return (f"llvq 2-bit fused GEMV, {rows}x{cols} layer (K padded to {-(-cols // 24) * 24}), u8 gain table, "
+            f"batch {batch}")
+
+
+WORKLOAD = workload()
+
+
+def algorithmic_bytes(rows=None, nb=None, batch=1) -> int:
     """Bytes one launch must move: packed words (8 B/block), per-row gain tables (512 B),
     activations (fp16) and outputs (fp32)."""
+    rows, nb = rows or ROWS, nb or NB
     return rows * nb * 8 + rows * 512 + batch * nb * 24 * 2 + batch * rows * 4
 
 
@@ -451,7 +460,7 @@ def build_line(steps, warmup, R, B, world, secs, secs_e2e, clk, sms, gpu_name):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": steps,
         "warmup": warmup, "ms_per_step": secs / steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD if B == 1 else WORKLOAD.replace("batch 1", f"batch {B}"),
+        "config": {"workload": workload(batch=B),
                    "rows": ROWS, "cols": K, "blocks_per_row": NB,
                    "batch": B, "index_bits": 48, "layer_copies_per_step": R,
                    "l2_policy": f"inputs larger than L2: {R} distinct layer copies "
@@ -511,7 +520,13 @@ def main():
                     help="decode: time llvq_decode alone (profiling aid); sweep: every layer shape, "
                          "budget and batch against cuBLAS fp16, plus the full 7B stack")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: batch (1 = the metric's workload)")
+    ap.add_argument("--rows", type=int, default=4096, help="gemv mode: layer rows (4096 = the metric's workload)")
+    ap.add_argument("--cols", type=int, default=4096, help="gemv mode: layer columns (4096 = the metric's workload)")
     args = ap.parse_args()
+    global ROWS, K, NB, WORKLOAD
+    ROWS, K = args.rows, args.cols
+    NB = -(-K // 24)
+    WORKLOAD = workload()
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
