@@ -2,12 +2,13 @@
 
 TEST INFRASTRUCTURE ONLY.  The oracle is a plain, slow, obviously-correct C implementation of
 the LLVQ index decode (shell -> class -> Golay refinement r, sign pattern s, lexicographic
-arrangement rank I'') and of the fp64 GEMV/GEMM on packed words.  Only the tests, the
+arrangement rank I''), of the fp64 GEMV/GEMM on packed words and of the nearest-point search
+over the shell union (angular and Euclidean criteria, with a brute-force search beside it).  Only the tests, the
 package's smoke check and the bench's CPU-baseline leg import this module; the product path
 never does.  Indices wider than 64 bits travel as (lo, hi) uint64 pairs.
 
 Method source: "Leech Lattice Vector Quantization for Efficient LLM Compression",
-papernotes.org notes, 方法详解 / 关键设计 1-2 and 4; gist.science summary, Methodik 1 and 3.
+papernotes.org notes, 方法详解 / 关键设计 1-2 and 4; gist.science summary, Methodik 1-3.
 """
 from __future__ import annotations
 
@@ -70,6 +71,14 @@ def lib():
         L.ora_gemm_mt.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_void_p, C.c_int32,
                                   C.c_int64, C.c_int32, u16p, u16p, C.c_int32, f64p, C.c_int32]
         L.ora_gemm_mt.restype = C.c_int64
+        f32p = C.POINTER(C.c_float)
+        L.ora_search.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_double, f64p, i32p, f64p]
+        L.ora_search_batch.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_double, C.c_int64, f32p,
+                                       i8p, f64p, C.c_int32]
+        L.ora_search_brute.argtypes = [C.c_int32, C.c_int32, C.c_double, C.c_int64, f32p, i8p, f64p,
+                                       C.c_int32]
+        L.ora_search_brute.restype = C.c_int64
+        L.ora_class_best.argtypes = [C.c_void_p, C.c_int32, C.c_int64, C.c_uint32, f64p, i32p, f64p]
         L.ora_half_to_double.argtypes = [C.c_uint16]
         L.ora_half_to_double.restype = C.c_double
         _lib = L
@@ -221,6 +230,26 @@ class Codec:
             return out, shell, int(bad)
         return out
 
+    def search(self, X, m_max: int, mode: int, scale: float = 1.0, threads: int = 1):
+        """Best point of shells 2..m_max for each row of X (fp32 [n, 24]) under the angular
+        (mode 0) or Euclidean (mode 1, reconstruction scale * v) criterion.
+        Returns (points int8 [n, 24], <x, v> fp64 [n])."""
+        X, n, V, d = _search_args(X)
+        if lib().ora_search_batch(self._h, m_max, mode, scale, n, X.ctypes.data_as(C.POINTER(C.c_float)),
+                                  _p(V, i8p), _p(d, f64p), threads):
+            raise ValueError("bad search arguments")
+        return V, d
+
+    def class_best(self, m: int, j: int, word: int, y):
+        """Best point of class j of shell m with codeword word (1-mod-4 set of an odd class,
+        2-mod-4 set of an even one) for target y; returns (point, <y, v>)."""
+        yy = np.ascontiguousarray(y, np.float64)
+        v = np.zeros(24, np.int32)
+        d = C.c_double()
+        if lib().ora_class_best(self._h, m, j, word, _p(yy, f64p), _p(v, i32p), C.byref(d)):
+            raise ValueError("no such class, or the word does not fit it")
+        return v, d.value
+
     def gemm(self, words: np.ndarray, nb: int, gain_mode: int, gains: np.ndarray, x: np.ndarray,
              batch: int, row_pitch_words: int | None = None, threads: int = 1) -> np.ndarray:
         """fp64 y[batch, rows] from packed words [rows, pitch] (uint64, or uint64 pairs for
@@ -243,6 +272,35 @@ class Codec:
         if bad < 0:
             raise ValueError("word size does not match the index budget")
         return y
+
+
+ANGULAR, EUCLIDEAN = 0, 1
+
+
+def _search_args(X):
+    X = np.ascontiguousarray(X, np.float32).reshape(-1, 24)
+    n = X.shape[0]
+    return X, n, np.zeros((n, 24), np.int8), np.zeros(n, np.float64)
+
+
+def search_brute(X, m_max: int, mode: int, scale: float = 1.0, threads: int = 1):
+    """Best point of shells 2..m_max for each row of X by enumerating every point from the
+    congruences (no classes).  Returns (points int8 [n, 24], <x, v> [n], points visited)."""
+    X, n, V, d = _search_args(X)
+    visited = lib().ora_search_brute(m_max, mode, scale, n, X.ctypes.data_as(C.POINTER(C.c_float)),
+                                     _p(V, i8p), _p(d, f64p), threads)
+    if visited < 0:
+        raise ValueError("bad search arguments")
+    return V, d, int(visited)
+
+
+def search_objective(mode: int, scale: float, dot, norm2):
+    """The quantity each search mode maximizes, from <x, v> and |v|^2 (scaled coordinates)."""
+    dot = np.asarray(dot, np.float64)
+    norm2 = np.asarray(norm2, np.float64)
+    if mode == ANGULAR:
+        return dot / np.sqrt(norm2)
+    return 2.0 * scale * dot - scale * scale * norm2
 
 
 def half_to_double(h: int) -> float:

@@ -19,6 +19,8 @@
  *   [notes-K4]  papernotes.org, 方法详解 / 关键设计 4: fused dequantize-and-multiply.
  *   [gist-M1]   gist.science, Methodik 1: Leech lattice built from G24, integer vectors in
  *               even and odd cosets, shells of equal squared norm.
+ *   [gist-M2]   gist.science, Methodik 2: search over the union of shells, Euclidean distance
+ *               (spherical shaping) or cosine similarity (shape-gain); extends Adoul & Barth.
  *   [gist-M3]   gist.science, Methodik 3: index hierarchy shell -> class -> local symmetries.
  * Textbook facts the pages point to but do not print (Conway & Sloane, "Sphere Packings,
  * Lattices and Groups", ch. 4 sec. 11): the sqrt(8)-scaled Leech lattice is the set of
@@ -1081,4 +1083,305 @@ int ora_check_shells(ora_codec *c, int32_t m_lo, int32_t m_hi, int32_t nthreads,
     free(bm); free(jobs); free(th);
     for (int k = 1; k < 7; k++) if (result[k]) return 1;
     return 0;
+}
+
+/* ===================================================================================== */
+/* Nearest-point search over the shell union Lambda24(M) = Shell(2) u ... u Shell(M)     */
+/* ([notes-K1] 关键设计 1 "多壳层球面与角度搜索": the union of shells, the unit-vector      */
+/* inner product for the shape of a shape-gain split; [gist-M2] Methodik 2: two modes,     */
+/* Euclidean distance for spherical shaping, cosine similarity for shape-gain, both over   */
+/* the union; the search extends Adoul & Barth's single-shell search).                     */
+/*                                                                                         */
+/* Readings (the pages name the two criteria but print no algorithm):                     */
+/*   angular   (mode 0): maximize <y, v> / |v| over v in the union.                        */
+/*   Euclidean (mode 1): the reconstruction is c v for a given scale c > 0; minimize       */
+/*                       |y - c v|^2, i.e. maximize 2 c <y, v> - c^2 |v|^2.                */
+/* Every point of a class has the same norm, so each criterion is the best <y, v> inside   */
+/* each class, compared across classes.  Inside a class and for one Golay codeword (the    */
+/* 2-mod-4 set S of an even point, the 1-mod-4 set T of an odd one) the best point follows */
+/* from the rearrangement inequality (larger |y_i| take larger magnitudes):               */
+/*   even: S takes the 2-mod-4 magnitudes and the other positions the 0-mod-4 ones, each   */
+/*         in descending order of |y_i|, signs those of y; when the coordinate sum is not  */
+/*         0 mod 8 the sign on S with the smallest |y_i| turns (one turn costs least).    */
+/*   odd:  the signs follow from T and the magnitudes (x_i = 1 mod 4 exactly on T), so a   */
+/*         position wants a 1-mod-4 magnitude when (i in T) equals (y_i >= 0) and a       */
+/*         3-mod-4 one otherwise.  Each set takes its own magnitudes in descending order;  */
+/*         when a set has more positions than magnitudes of its kind, its smallest-|y|     */
+/*         positions take the other kind's smallest magnitudes with the wrong sign, the   */
+/*         largest of those |y_i| taking the smallest magnitude.                          */
+/* The brute-force search below enumerates the shells from the congruences alone and pins  */
+/* these rules on shells 2..4.  Ties keep the first best in the order shell, class,       */
+/* codeword (by mask).                                                                     */
+/* ===================================================================================== */
+
+/* positions by |y_i| descending, equal values by position */
+static void order_desc(const double y[ORA_DIM], int ord[ORA_DIM]) {
+    for (int i = 0; i < ORA_DIM; i++) ord[i] = i;
+    for (int i = 1; i < ORA_DIM; i++)                     /* insertion sort, stable */
+        for (int j = i; j > 0 && fabs(y[ord[j]]) > fabs(y[ord[j - 1]]); j--) {
+            int t = ord[j]; ord[j] = ord[j - 1]; ord[j - 1] = t;
+        }
+}
+
+/* class magnitudes of residue res (mod 4), descending; returns how many */
+static int class_mags(const ocls *o, int res, int out[ORA_DIM]) {
+    int n = 0;
+    for (int g = o->nvals - 1; g >= 0; g--)
+        if (o->vals[g] % 4 == res)
+            for (int t = 0; t < o->cnts[g]; t++) out[n++] = o->vals[g];
+    return n;
+}
+
+/* the point of odd class o whose 1-mod-4 set is T with the largest <y, v> */
+static void best_odd(const ocls *o, uint32_t T, const double y[ORA_DIM], const int ord[ORA_DIM],
+                     int v[ORA_DIM]) {
+    int L1[ORA_DIM], L3[ORA_DIM], P1[ORA_DIM], P3[ORA_DIM], a[ORA_DIM];
+    int n1 = class_mags(o, 1, L1), n3 = class_mags(o, 3, L3), p1 = 0, p3 = 0;
+    for (int t = 0; t < ORA_DIM; t++) {
+        int i = ord[t];
+        int inT = (int)(T >> i & 1u), pos = y[i] >= 0.0;
+        if (inT == pos) P1[p1++] = i; else P3[p3++] = i;
+    }
+    if (p1 >= n1) {                     /* P1 has s = p1 - n1 positions too many */
+        int s = p1 - n1;
+        for (int j = 0; j < n1; j++) a[P1[j]] = L1[j];
+        for (int j = 0; j < p3; j++) a[P3[j]] = L3[j];
+        for (int j = 0; j < s; j++) a[P1[n1 + j]] = L3[n3 - 1 - j];
+    } else {                            /* P3 has s = p3 - n3 positions too many */
+        int s = p3 - n3;
+        for (int j = 0; j < n3; j++) a[P3[j]] = L3[j];
+        for (int j = 0; j < p1; j++) a[P1[j]] = L1[j];
+        for (int j = 0; j < s; j++) a[P3[n3 + j]] = L1[n1 - 1 - j];
+    }
+    for (int i = 0; i < ORA_DIM; i++)
+        v[i] = ((a[i] % 4 == 1) == (int)(T >> i & 1u)) ? a[i] : -a[i];
+}
+
+/* the point of even class o whose 2-mod-4 set is S with the largest <y, v> */
+static void best_even(const ocls *o, uint32_t S, const double y[ORA_DIM], const int ord[ORA_DIM],
+                      int v[ORA_DIM]) {
+    int L2[ORA_DIM], L0[ORA_DIM];
+    class_mags(o, 2, L2);
+    class_mags(o, 0, L0);
+    int j2 = 0, j0 = 0, sum = 0, last_on_S = -1;
+    for (int t = 0; t < ORA_DIM; t++) {
+        int i = ord[t];
+        int a = (S >> i & 1u) ? L2[j2++] : L0[j0++];
+        if (S >> i & 1u) last_on_S = i;
+        v[i] = y[i] >= 0.0 ? a : -a;
+        sum += v[i];
+    }
+    if (mod_pos(sum, 8) != 0 && last_on_S >= 0) v[last_on_S] = -v[last_on_S];
+}
+
+static double dot24(const double y[ORA_DIM], const int v[ORA_DIM]) {
+    double s = 0.0;
+    for (int i = 0; i < ORA_DIM; i++) s += y[i] * (double)v[i];
+    return s;
+}
+
+static double search_objective(int mode, double scale, double dot, int norm2) {
+    return mode == 0 ? dot / sqrt((double)norm2) : 2.0 * scale * dot - scale * scale * (double)norm2;
+}
+
+int ora_search(ora_codec *c, int32_t m_max, int32_t mode, double scale, const double y[ORA_DIM],
+               int32_t v_out[ORA_DIM], double *dot_out) {
+    if (m_max < 2 || m_max > c->M || (mode != 0 && mode != 1) || (mode == 1 && !(scale > 0.0)))
+        return -1;
+    int ord[ORA_DIM], v[ORA_DIM];
+    order_desc(y, ord);
+    double best = -INFINITY, best_dot = 0.0;
+    int have = 0;
+    for (int m = 2; m <= m_max; m++) {
+        if (build_shell(c, m)) return -1;
+        for (int64_t j = 0; j < c->ncls[m]; j++) {
+            const ocls *o = &c->cls[m][j];
+            int first = o->odd ? 0 : c->wbase[o->k], end = o->odd ? 4096 : c->wbase[o->k + 1];
+            for (int w = first; w < end; w++) {
+                if (o->odd) best_odd(o, c->golay_mask[w], y, ord, v);
+                else best_even(o, c->golay_weight[w], y, ord, v);
+                double d = dot24(y, v);
+                double f = search_objective(mode, scale, d, 16 * m);
+                if (!have || f > best) {
+                    have = 1; best = f; best_dot = d;
+                    for (int i = 0; i < ORA_DIM; i++) v_out[i] = v[i];
+                }
+            }
+        }
+        drop_shell(c, m);
+    }
+    if (dot_out) *dot_out = best_dot;
+    return 0;
+}
+
+typedef struct {
+    ora_codec *c;
+    int m_max, mode, tid, nthreads, bad;
+    double scale;
+    int64_t n;
+    const float *X;
+    int8_t *V;
+    double *dot;
+} search_job;
+
+static void *search_thread(void *arg) {
+    search_job *j = arg;
+    double y[ORA_DIM], d;
+    int32_t v[ORA_DIM];
+    for (int64_t r = j->tid; r < j->n; r += j->nthreads) {
+        for (int i = 0; i < ORA_DIM; i++) y[i] = (double)j->X[r * ORA_DIM + i];
+        if (ora_search(j->c, j->m_max, j->mode, j->scale, y, v, &d)) { j->bad = 1; return NULL; }
+        for (int i = 0; i < ORA_DIM; i++) j->V[r * ORA_DIM + i] = (int8_t)v[i];
+        if (j->dot) j->dot[r] = d;
+    }
+    return NULL;
+}
+
+int ora_search_batch(ora_codec *c, int32_t m_max, int32_t mode, double scale, int64_t n,
+                     const float *X, int8_t *V, double *dot, int32_t nthreads) {
+    if (!c->store_all || m_max < 2 || m_max > c->M || n < 0) return -1;
+    if (nthreads < 1) nthreads = 1;
+    search_job *jobs = calloc((size_t)nthreads, sizeof(search_job));
+    pthread_t *th = calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!jobs || !th) { free(jobs); free(th); return -2; }
+    for (int t = 0; t < nthreads; t++) {
+        search_job jb = {c, m_max, mode, t, nthreads, 0, scale, n, X, V, dot};
+        jobs[t] = jb;
+        pthread_create(&th[t], NULL, search_thread, &jobs[t]);
+    }
+    int bad = 0;
+    for (int t = 0; t < nthreads; t++) { pthread_join(th[t], NULL); bad |= jobs[t].bad; }
+    free(jobs); free(th);
+    return bad ? -1 : 0;
+}
+
+/* ---- brute force: every point of shells 2..m_max from the congruences ----------------- */
+typedef struct {
+    int m_max, mode, target_sum8;
+    double scale;
+    int64_t n;
+    const double *Y;            /* [n][24] */
+    int res[ORA_DIM];           /* residue mod 4 each coordinate must have */
+    int minrest[ORA_DIM + 1];   /* least squared norm coordinates i.. can take */
+    int x[ORA_DIM];
+    double *part;               /* [25][n]: <y, x> over the first i coordinates */
+    double *best, *bestdot;     /* [n] */
+    int32_t *bestv;             /* [n][24] */
+    int64_t visited;
+} brute_ctx;
+
+static void brute_rec(brute_ctx *e, int i, int rem, int sum) {
+    if (i == ORA_DIM) {
+        int norm2 = 16 * e->m_max - rem;
+        if (norm2 < 32 || mod_pos(sum, 8) != e->target_sum8) return;   /* shell >= 2, mod 8 */
+        e->visited++;
+        const double *d = e->part + (size_t)ORA_DIM * e->n;
+        for (int64_t t = 0; t < e->n; t++) {
+            double f = search_objective(e->mode, e->scale, d[t], norm2);
+            if (f > e->best[t]) {
+                e->best[t] = f;
+                e->bestdot[t] = d[t];
+                for (int k = 0; k < ORA_DIM; k++) e->bestv[t * ORA_DIM + k] = e->x[k];
+            }
+        }
+        return;
+    }
+    int vmax = (int)floor(sqrt((double)rem)) + 1;
+    for (int v = -vmax; v <= vmax; v++) {
+        if (mod_pos(v, 4) != e->res[i]) continue;
+        int r2 = rem - v * v;
+        if (r2 < e->minrest[i + 1]) continue;
+        e->x[i] = v;
+        const double *p = e->part + (size_t)i * e->n;
+        double *q = e->part + (size_t)(i + 1) * e->n;
+        for (int64_t t = 0; t < e->n; t++) q[t] = p[t] + e->Y[t * ORA_DIM + i] * (double)v;
+        brute_rec(e, i + 1, r2, sum + v);
+    }
+}
+
+typedef struct {
+    brute_ctx e;
+    int tid, nthreads;
+} brute_job;
+
+static void *brute_thread(void *arg) {
+    brute_job *j = arg;
+    brute_ctx *e = &j->e;
+    for (int job = j->tid; job < 2 * 4096; job += j->nthreads) {   /* (coset, codeword) */
+        int odd = job / 4096;
+        uint32_t cw = g_golay_mask[job % 4096];
+        e->target_sum8 = odd ? 4 : 0;
+        for (int i = 0; i < ORA_DIM; i++) {
+            int in = (int)(cw >> i & 1u);
+            e->res[i] = odd ? (in ? 1 : 3) : (in ? 2 : 0);
+        }
+        e->minrest[ORA_DIM] = 0;
+        for (int i = ORA_DIM - 1; i >= 0; i--)
+            e->minrest[i] = e->minrest[i + 1] + (e->res[i] == 0 ? 0 : (e->res[i] == 2 ? 4 : 1));
+        brute_rec(e, 0, 16 * e->m_max, 0);
+    }
+    return NULL;
+}
+
+int64_t ora_search_brute(int32_t m_max, int32_t mode, double scale, int64_t n, const float *X,
+                         int8_t *V, double *dot, int32_t nthreads) {
+    if (m_max < 2 || (mode != 0 && mode != 1) || (mode == 1 && !(scale > 0.0)) || n < 0) return -1;
+    ensure_golay();
+    if (nthreads < 1) nthreads = 1;
+    double *Y = malloc(sizeof(double) * (size_t)(n * ORA_DIM + 1));
+    brute_job *jobs = calloc((size_t)nthreads, sizeof(brute_job));
+    pthread_t *th = calloc((size_t)nthreads, sizeof(pthread_t));
+    if (!Y || !jobs || !th) { free(Y); free(jobs); free(th); return -2; }
+    for (int64_t k = 0; k < n * ORA_DIM; k++) Y[k] = (double)X[k];
+    int ok = 1;
+    for (int t = 0; t < nthreads; t++) {
+        brute_ctx *e = &jobs[t].e;
+        e->m_max = m_max; e->mode = mode; e->scale = scale; e->n = n; e->Y = Y;
+        e->part = calloc((size_t)(ORA_DIM + 1) * (size_t)(n + 1), sizeof(double));
+        e->best = malloc(sizeof(double) * (size_t)(n + 1));
+        e->bestdot = calloc((size_t)(n + 1), sizeof(double));
+        e->bestv = calloc((size_t)(n + 1) * ORA_DIM, sizeof(int32_t));
+        if (!e->part || !e->best || !e->bestdot || !e->bestv) ok = 0;
+        else for (int64_t k = 0; k < n; k++) e->best[k] = -INFINITY;
+        jobs[t].tid = t;
+        jobs[t].nthreads = nthreads;
+    }
+    int64_t visited = 0;
+    if (ok) {
+        for (int t = 0; t < nthreads; t++) pthread_create(&th[t], NULL, brute_thread, &jobs[t]);
+        for (int t = 0; t < nthreads; t++) { pthread_join(th[t], NULL); visited += jobs[t].e.visited; }
+        for (int64_t k = 0; k < n; k++) {          /* best over the threads */
+            int bt = 0;
+            for (int t = 1; t < nthreads; t++)
+                if (jobs[t].e.best[k] > jobs[bt].e.best[k]) bt = t;
+            for (int i = 0; i < ORA_DIM; i++) V[k * ORA_DIM + i] = (int8_t)jobs[bt].e.bestv[k * ORA_DIM + i];
+            if (dot) dot[k] = jobs[bt].e.bestdot[k];
+        }
+    }
+    for (int t = 0; t < nthreads; t++) {
+        free(jobs[t].e.part); free(jobs[t].e.best); free(jobs[t].e.bestdot); free(jobs[t].e.bestv);
+    }
+    free(Y); free(jobs); free(th);
+    return ok ? visited : -2;
+}
+
+/* The best point of one class and one codeword (the rearrangement rules above), exposed so
+ * that tests can check them against an exact assignment solver.  word: the 1-mod-4 set T
+ * (odd class, any codeword) or the 2-mod-4 set S (even class, a codeword of weight k).
+ * Returns 0, or -1 when the class does not exist or the word does not fit it. */
+int ora_class_best(ora_codec *c, int32_t m, int64_t j, uint32_t word, const double y[ORA_DIM],
+                   int32_t v_out[ORA_DIM], double *dot_out) {
+    if (m < 2 || m > c->M || build_shell(c, m) || j < 0 || j >= c->ncls[m]) return -1;
+    const ocls *o = &c->cls[m][j];
+    int ok = golay_contains(c->golay_mask, word & 0xFFFFFFu, NULL) && word <= 0xFFFFFFu &&
+             (o->odd || popcount24(word) == o->k);
+    if (ok) {
+        int ord[ORA_DIM], v[ORA_DIM];
+        order_desc(y, ord);
+        if (o->odd) best_odd(o, word, y, ord, v); else best_even(o, word, y, ord, v);
+        for (int i = 0; i < ORA_DIM; i++) v_out[i] = v[i];
+        if (dot_out) *dot_out = dot24(y, v);
+    }
+    drop_shell(c, m);
+    return ok ? 0 : -1;
 }

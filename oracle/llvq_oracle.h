@@ -112,6 +112,27 @@ int64_t ora_gemm_mt(const ora_codec *c, int32_t rows, int32_t nb, const void *wo
 /* Exhaustive self-check of shells m_lo..m_hi (48/72-bit codecs): direct enumeration,
  * encode, one hit per index, decode round trip.  See the definition for result[]. */
 int ora_check_shells(ora_codec *c, int32_t m_lo, int32_t m_hi, int32_t nthreads, int64_t result[7]);
+/* ---- nearest-point search over the shell union Shell(2) u ... u Shell(m_max) ------------
+ * mode 0 (angular, the shape of a shape-gain split): maximize <y, v> / |v|.
+ * mode 1 (Euclidean, spherical clipping): minimize |y - scale * v|^2 (scale > 0).
+ * v is in sqrt(8)-scaled integer coordinates; m_max <= the codec's largest shell.  The
+ * search takes the best point of every class and Golay codeword (rearrangement rules in the
+ * definition).  ora_search returns 0, or -1 on bad arguments; *dot_out = <y, v>. */
+int ora_search(ora_codec *c, int32_t m_max, int32_t mode, double scale, const double y[ORA_DIM],
+               int32_t v_out[ORA_DIM], double *dot_out);
+/* The same over rows of X (fp32 [n][24], read as exact doubles), rows split over host threads;
+ * V: int8 [n][24]; dot: [n] or NULL.  48/72-bit codecs only.  Returns 0, or -1. */
+int ora_search_batch(ora_codec *c, int32_t m_max, int32_t mode, double scale, int64_t n,
+                     const float *X, int8_t *V, double *dot, int32_t nthreads);
+/* The best point (largest <y, v>) of class j of shell m among the points whose 1-mod-4 set
+ * (odd class) or 2-mod-4 set (even class) is the codeword word.  Returns 0, or -1. */
+int ora_class_best(ora_codec *c, int32_t m, int64_t j, uint32_t word, const double y[ORA_DIM],
+                   int32_t v_out[ORA_DIM], double *dot_out);
+/* Brute force over every point of shells 2..m_max, enumerated from the congruences alone
+ * (no classes, no rearrangement).  Returns the number of points visited, or a negative
+ * value on bad arguments. */
+int64_t ora_search_brute(int32_t m_max, int32_t mode, double scale, int64_t n, const float *X,
+                         int8_t *V, double *dot, int32_t nthreads);
 /* fp16 bits -> double (exact). */
 double ora_half_to_double(uint16_t h);
 
