@@ -292,6 +292,130 @@ def cpu_baseline(steps_seconds=12.0, one_core_seconds=3.0):
     return out
 
 
+# ------------------------------------------------------------------ nearest-point search
+# The pages' Gaussian-source experiment at 2 bits per dimension: spherical clipping spends all
+# 48 bits of a block on the index (shells 2..13, Euclidean criterion, reconstruction c v); the
+# shape-gain split gives 1 or 2 bits to a scalar gain and the rest to the direction (angular
+# criterion over shells 2..12, 46.66 bits, or 2..11, 45.20 bits).
+SEARCH_N = 1 << 17
+SEARCH_TRAIN = 1 << 16
+SEARCH_CONFIGS = [
+    # name, criterion, max_shell, gain bits
+    ("spherical clipping", 1, 13, 0),
+    ("shape-gain, 1 gain bit", 0, 12, 1),
+    ("shape-gain, 2 gain bits", 0, 11, 2),
+]
+
+
+def _search(torch, codec, X, max_shell, mode, scale, levels=None):
+    n = X.shape[0]
+    P = torch.empty((n, 24), dtype=torch.int8, device=X.device)
+    D = torch.empty(n, dtype=torch.float64, device=X.device)
+    codes = None if levels is None else torch.empty(n, dtype=torch.uint8, device=X.device)
+    codec.search(X, P, max_shell, mode, scale, dots=D, levels=levels, codes=codes)
+    return P, D, codes
+
+
+def search_quality(torch, codec, dev):
+    """MSE per dimension, SQNR (bits) and share of the Shannon bound (2 bits) on SEARCH_N test
+    blocks; the scale c (clipping) and the gain levels (shape-gain, Lloyd-Max on the best gains
+    <x, v> / |v|) are fitted on SEARCH_TRAIN other blocks."""
+    from codebook_free_lattice_b200 import synth
+    import math
+    Xtr = torch.from_numpy(synth.gaussian_blocks(synth.rng(60, 4), SEARCH_TRAIN)).to(dev)
+    Xte = torch.from_numpy(synth.gaussian_blocks(synth.rng(61, 4), SEARCH_N)).to(dev)
+    out = []
+    for name, mode, ms, gbits in SEARCH_CONFIGS:
+        if mode == 1:
+            def mse(c, X):
+                P, _, _ = _search(torch, codec, X, ms, 1, c)
+                return float(((X.double() - c * P.double()) ** 2).mean())
+            lo, hi = 0.15, 0.60                                   # golden-section search for c
+            r = (math.sqrt(5) - 1) / 2
+            a, b = hi - r * (hi - lo), lo + r * (hi - lo)
+            fa, fb = mse(a, Xtr), mse(b, Xtr)
+            for _ in range(18):
+                if fa < fb:
+                    hi, b, fb = b, a, fa
+                    a = hi - r * (hi - lo)
+                    fa = mse(a, Xtr)
+                else:
+                    lo, a, fa = a, b, fb
+                    b = lo + r * (hi - lo)
+                    fb = mse(b, Xtr)
+            c = (lo + hi) / 2
+            m = mse(c, Xte)
+            extra = {"scale": c}
+            index_bits = 47.997
+        else:
+            P, D, _ = _search(torch, codec, Xtr, ms, 0, 1.0)
+            g = (D / P.double().pow(2).sum(1).sqrt()).cpu().numpy()
+            L = np.quantile(g, (np.arange(2 ** gbits) + 0.5) / 2 ** gbits)   # Lloyd-Max levels
+            for _ in range(100):
+                idx = np.argmin(np.abs(g[:, None] - L[None, :]), axis=1)
+                L = np.array([g[idx == k].mean() if (idx == k).any() else L[k] for k in range(L.size)])
+            lev = torch.tensor(L, dtype=torch.float64, device=dev)
+            P, D, codes = _search(torch, codec, Xte, ms, 0, 1.0, lev)
+            V = P.double()
+            Xh = lev[codes.long()][:, None] * V / V.pow(2).sum(1, keepdim=True).sqrt()
+            m = float(((Xte.double() - Xh) ** 2).mean())
+            g_exact = D / V.pow(2).sum(1).sqrt()
+            shape_only = float(((Xte.double() - g_exact[:, None] * V / V.pow(2).sum(1, keepdim=True).sqrt()) ** 2).mean())
+            extra = {"gain_levels": [round(float(x), 4) for x in L], "mse_exact_gain": shape_only}
+            index_bits = {11: 45.205, 12: 46.658}[ms]
+        sq = -0.5 * math.log2(m)
+        out.append({"config": name, "max_shell": ms, "bits_per_dim": (index_bits + gbits) / 24,
+                    "mse": m, "sqnr_bits": sq, "shannon_retention": sq / 2.0, **extra})
+    return {"source": f"N(0, I_24), {SEARCH_N} test blocks (fit on {SEARCH_TRAIN} others)", "results": out}
+
+
+def search_throughput(torch, codec, dev, steps, warmup, max_shell=13, mode=1, scale=0.3):
+    """llvq_search on SEARCH_N Gaussian blocks, CUDA events around each launch on the launching
+    stream; L2 flushed (a 3x L2 buffer written) before every launch, outside the timed span."""
+    from codebook_free_lattice_b200 import synth
+    X = torch.from_numpy(synth.gaussian_blocks(synth.rng(62, 4), SEARCH_N)).to(dev)
+    P = torch.empty((SEARCH_N, 24), dtype=torch.int8, device=dev)
+    D = torch.empty(SEARCH_N, dtype=torch.float64, device=dev)
+    flush = torch.empty(3 * torch.cuda.get_device_properties(dev).L2_cache_size // 4, dtype=torch.int32, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    total = 0.0
+    with torch.cuda.stream(stream):
+        for i in range(warmup + steps):
+            flush.fill_(i)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            codec.search(X, P, max_shell, mode, scale, dots=D, stream=stream)
+            e.record(stream)
+            e.synchronize()
+            if i >= warmup:
+                total += s.elapsed_time(e) / 1e3
+    if codec.get_error(stream) != 0:
+        raise RuntimeError("llvq_search raised a device flag")
+    t = total / steps
+    return {"n": SEARCH_N, "max_shell": max_shell, "mode": "euclidean" if mode else "angular",
+            "ms_per_launch": t * 1e3, "vectors_per_s": SEARCH_N / t}
+
+
+def search_cpu_baseline(seconds=12.0, max_shell=13, mode=1, scale=0.3):
+    """The oracle's search (plain C, fp64) on all host cores, on a bounded sample of the same
+    Gaussian blocks, timed until ~seconds of work."""
+    import oracle
+    from codebook_free_lattice_b200 import synth
+    oc = oracle.Codec(48)
+    cores = os.cpu_count() or 1
+    X = synth.gaussian_blocks(synth.rng(62, 4), 4 * cores)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oc.search(X, max_shell, mode, scale, threads=cores)
+        done += X.shape[0]
+        el = time.perf_counter() - t0
+        if el > seconds:
+            break
+    return {"value": done / el, "unit": "vectors/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of the Gaussian blocks ({X.shape[0]} per pass, all cores), {el:.1f} s",
+            "cpu_model": cpu_model()}
+
+
 # ------------------------------------------------------------------ secondary measurements
 SWEEP_CASES = [
     # (name, rows, K, index_bits, batch)
@@ -516,9 +640,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-n", type=int, default=28672 * 342,
                     help="indices for the llvq_decode throughput line (default: the 28672x8192 layer)")
-    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "encode", "sweep"],
+    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "encode", "sweep", "search"],
                     help="decode: time llvq_decode alone (profiling aid); sweep: every layer shape, "
-                         "budget and batch against cuBLAS fp16, plus the full 7B stack")
+                         "budget and batch against cuBLAS fp16, plus the full 7B stack; search: "
+                         "the nearest-point search on the Gaussian source (throughput and quality)")
+    ap.add_argument("--search-quality", type=int, default=1, help="search mode: run the quality experiment")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: batch (1 = the metric's workload)")
     ap.add_argument("--rows", type=int, default=4096, help="gemv mode: layer rows (4096 = the metric's workload)")
     ap.add_argument("--cols", type=int, default=4096, help="gemv mode: layer columns (4096 = the metric's workload)")
@@ -558,6 +684,21 @@ def main():
     if args.mode == "sweep":
         if rank == 0:
             sweep(torch, dev)
+        return 0
+    if args.mode == "search":
+        if rank == 0:
+            with ClockSampler(torch.cuda.current_device()) as clocks:
+                r = search_throughput(torch, codec, dev, args.steps, args.warmup)
+            line = {"mode": "search", "metric": "search_vectors_per_s", "value": r["vectors_per_s"],
+                    "unit": "vectors/s", "steps": args.steps, "warmup": args.warmup,
+                    "config": {"workload": f"nearest point of Leech shells 2..13 (Euclidean, c = 0.3) "
+                                           f"for {SEARCH_N} N(0, I_24) blocks", "l2": "flushed"},
+                    "dtype": "f64", "data": "synthetic", **r, "clocks": clocks.summary()}
+            if args.search_quality:
+                line["quality"] = search_quality(torch, codec, dev)
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = search_cpu_baseline()
+            print(json.dumps(line), flush=True)
         return 0
 
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size

@@ -23,6 +23,9 @@ LLVQ_GAIN_U8_TABLE = 1
 LLVQ_FLAG_INDEX_RANGE = 0x1
 LLVQ_FLAG_WAIT_TIMEOUT = 0x2
 LLVQ_FLAG_NOT_CODED = 0x4
+LLVQ_FLAG_SEARCH_INPUT = 0x8
+LLVQ_SEARCH_ANGULAR = 0
+LLVQ_SEARCH_EUCLIDEAN = 1
 
 
 class llvq_weight(C.Structure):
@@ -67,6 +70,8 @@ def lib() -> C.CDLL:
         L.llvq_get_error.argtypes = [C.c_void_p, C.c_void_p, C.POINTER(C.c_uint32)]
         L.llvq_decode_noalloc.argtypes = [C.c_int32, C.c_void_p, C.c_int32, C.c_int64, C.c_void_p, C.c_void_p]
         L.llvq_encode.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_int32, C.c_void_p]
+        L.llvq_search.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_double, C.c_void_p, C.c_int64,
+                                  C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]
         L.llvq_set_wait_polls.argtypes = [C.c_uint32, C.c_uint32]
         L.llvq_set_wait_polls.restype = None
         L.llvq_last_error_message.argtypes = []
@@ -74,7 +79,7 @@ def lib() -> C.CDLL:
         L.llvq_class_table96.argtypes = [C.c_int32, C.c_void_p, C.c_int64, C.POINTER(C.c_int64)]
         for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
                   "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc", "llvq_class_table96",
-                  "llvq_encode"):
+                  "llvq_encode", "llvq_search"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -83,7 +88,7 @@ def lib() -> C.CDLL:
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
             "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
             "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message", "llvq_encode",
-            "llvq_set_wait_polls")
+            "llvq_set_wait_polls", "llvq_search")
 
 
 def llvq_set_wait_polls(table_polls: int = 0xFFFFFFFF, mma_polls: int = 0xFFFFFFFF) -> None:
@@ -187,6 +192,17 @@ class Codec:
         n = vectors.shape[0] if n is None else n
         _check(lib().llvq_encode(self._h, C.c_void_p(vectors.data_ptr()), n, C.c_void_p(words.data_ptr()),
                                  self.word_bytes, _stream(stream)), "llvq_encode")
+
+    def search(self, X, points, max_shell: int, mode: int, scale: float = 1.0, dots=None,
+               levels=None, codes=None, n: int | None = None, stream=None):
+        """Nearest point of shells 2..max_shell for each row of X (device fp32 [n, 24]) into points
+        (device int8 [n, 24]); dots (device fp64 [n]) receives <x, v>; with levels (device fp64)
+        and codes (device uint8 [n]) the angular criterion also picks the nearest gain level."""
+        n = X.shape[0] if n is None else n
+        ptr = lambda t: None if t is None else C.c_void_p(t.data_ptr())
+        _check(lib().llvq_search(self._h, max_shell, mode, scale, ptr(X), n, ptr(points), ptr(dots),
+                                 ptr(levels), 0 if levels is None else levels.numel(), ptr(codes),
+                                 _stream(stream)), "llvq_search")
 
     def gemv(self, w: llvq_weight, x, y, stream=None):
         _check(lib().llvq_gemv(self._h, C.byref(w), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()),

@@ -16,6 +16,7 @@ namespace llvq {
 constexpr unsigned kFlagIndexRange = 0x1u;   // an index >= N_M was met (LLVQ_FLAG_INDEX_RANGE)
 constexpr unsigned kFlagWaitTimeout = 0x2u;  // a bounded wait gave up (LLVQ_FLAG_WAIT_TIMEOUT)
 constexpr unsigned kFlagNotCoded = 0x4u;     // an encoded vector is not a coded point (LLVQ_FLAG_NOT_CODED)
+constexpr unsigned kFlagSearchInput = 0x8u;  // a searched row held a NaN or an infinity (LLVQ_FLAG_SEARCH_INPUT)
 
 // Decode n packed words into int8 [n][24].
 template <class D>

@@ -26,10 +26,15 @@
 #include "encode48.cuh"
 #include "encode72.cuh"
 #include "encode96.cuh"
+#include "search48.cuh"
 #include "tables.h"
 #include "tables96.h"
 
 using namespace llvq;
+
+static_assert(kFlagIndexRange == LLVQ_FLAG_INDEX_RANGE && kFlagWaitTimeout == LLVQ_FLAG_WAIT_TIMEOUT &&
+                  kFlagNotCoded == LLVQ_FLAG_NOT_CODED && kFlagSearchInput == LLVQ_FLAG_SEARCH_INPUT,
+              "device flag bits match the C ABI");
 
 struct llvq_codec {
     int index_bits = 0;
@@ -47,6 +52,7 @@ struct llvq_codec {
     uint32_t *d_tabC48 = nullptr;  // complement arrangement tables (48-bit table path)
     void *d_gv48 = nullptr;        // SmemGv48 image (48-bit fused products, k_gemv48)
     void *d_enc48 = nullptr;       // EncSmem48 image (48-bit encoder)
+    void *d_search48 = nullptr;    // SearchImage48 (48-bit nearest-point search)
     void *d_enc72 = nullptr;       // EncSmem72 image (72-bit encoder)
     unsigned long long *d_keys72 = nullptr;  // 72-bit class keys (encoder)
     void *d_enc96 = nullptr;       // EncSmem96 image (96-bit encoder)
@@ -326,6 +332,83 @@ llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E
         const uint32_t w = r << 12 | (uint32_t)(G.tlow[r & 63u] ^ G.tlow[64u + (r >> 6)]);
         if (w != T.golay_by_mask[r]) { err = "Golay low bits are not linear in the top 12"; return LLVQ_ERR_UNSUPPORTED; }
     }
+    return LLVQ_OK;
+}
+
+// Search tables of the 48-bit budget (k_search48): per class its magnitude groups split by kind
+// (odd: 1 / 3 mod 4; even: on S (2 mod 4) / off S (0 mod 4), zeros dropped), each kind in
+// descending magnitude with steps da and column offsets (kind * 25 + count of that kind's
+// magnitudes >= a_g) * 256; classes odd first, then even by codeword weight, each block by group
+// count descending (equal counts in index order).  Then the codewords: by mask, by (weight, mask).
+llvq_status build_search48(const HostTables &T, SearchImage48 &I, std::string &err) {
+    std::memset(&I, 0, sizeof I);
+    SearchHead48 &H = I.head;
+    static const int kWeights[kSrEvenWeights] = {0, 8, 12, 16, 24};
+    struct Item { int id, ng; };
+    std::vector<Item> blocks[kSrBlocks];
+    for (size_t i = 0; i < T.classes.size(); i++) {
+        const HostClass &c = T.classes[i];
+        int b = 0, ng = 0;
+        if (!c.odd) {
+            b = -1;
+            for (int w = 0; w < kSrEvenWeights; w++) if (kWeights[w] == c.k) b = 1 + w;
+            if (b < 0) { err = "search: even class of an unexpected codeword weight"; return LLVQ_ERR_UNSUPPORTED; }
+        }
+        for (int v : c.vals) ng += v != 0;
+        if (ng < 1 || ng > kSrGroups) { err = "search: magnitude groups out of range"; return LLVQ_ERR_UNSUPPORTED; }
+        blocks[b].push_back({(int)i, ng});
+    }
+    int j = 0;
+    for (int b = 0; b < kSrBlocks; b++) {
+        std::stable_sort(blocks[b].begin(), blocks[b].end(), [](const Item &x, const Item &y) { return x.ng > y.ng; });
+        if (b == 0) H.n_odd = (int)blocks[0].size();
+        for (int G = kSrGroups; G >= 1; G--) {
+            H.ng_base[b][kSrGroups - G] = j;
+            for (const Item &it : blocks[b]) {
+                if (it.ng != G) continue;
+                const HostClass &c = T.classes[it.id];
+                if (j >= kSrClasses || c.m > 255) { err = "search: class table too large"; return LLVQ_ERR_UNSUPPORTED; }
+                SearchRec48 &K = H.rec[j];
+                std::vector<std::pair<int, int>> kind[2];       // (magnitude, count), descending
+                for (size_t g = 0; g < c.vals.size(); g++) {
+                    const int a = c.vals[g];
+                    if (a == 0) continue;
+                    kind[c.odd ? (a % 4 == 3) : (a % 4 == 0)].push_back({a, c.cnts[g]});
+                }
+                int g = 0;
+                for (int kd = 0; kd < 2; kd++) {
+                    std::sort(kind[kd].begin(), kind[kd].end(), [](auto x, auto y) { return x.first > y.first; });
+                    int cum = 0;
+                    for (size_t u = 0; u < kind[kd].size(); u++, g++) {
+                        cum += kind[kd][u].second;
+                        const int next = u + 1 < kind[kd].size() ? kind[kd][u + 1].first : 0;
+                        K.da[g] = (double)(kind[kd][u].first - next);
+                        K.off[g] = (uint16_t)((kd * kSrCols + cum) * kSrRowBytes);
+                        I.mag[j][g] = (uint8_t)kind[kd][u].first;
+                    }
+                }
+                K.ng = (uint8_t)g;
+                K.m = (uint8_t)c.m;
+                K.id = (uint16_t)it.id;
+                if (!c.odd) {
+                    K.turn = kind[0].empty() ? 0.0 : 2.0 * (double)kind[0].back().first;
+                    K.q = (uint8_t)(c.k > 0 ? (c.sum_abs / 4) & 1 : 0);
+                }
+                j++;
+            }
+        }
+        H.ng_base[b][kSrGroups] = j;
+    }
+    for (int w = 0; w < kSrEvenWeights; w++) H.word_base[w] = T.weight_base[kWeights[w]];
+    H.word_base[kSrEvenWeights] = 4096;
+    H.chunk_base[0] = 0;
+    for (int w = 0; w < kSrEvenWeights; w++) {
+        for (int t = H.word_base[w]; t < H.word_base[w + 1]; t++)
+            if (__builtin_popcount(T.golay_by_weight[t]) != kWeights[w]) { err = "search: codeword weights"; return LLVQ_ERR_UNSUPPORTED; }
+        H.chunk_base[w + 1] = H.chunk_base[w] + (H.word_base[w + 1] - H.word_base[w] + 31) / 32;
+    }
+    std::memcpy(I.words, T.golay_by_mask, 4096 * sizeof(uint32_t));
+    std::memcpy(I.words + 4096, T.golay_by_weight, 4096 * sizeof(uint32_t));
     return LLVQ_OK;
 }
 
@@ -923,6 +1006,7 @@ void set_kernel_attrs() {
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         set_gemv48_attrs(std::make_integer_sequence<int, 2>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
+        cudaFuncSetAttribute(k_search48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SearchSmem48));
         cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
         cudaFuncSetAttribute(k_encode96, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem96));
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
@@ -1057,6 +1141,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
     std::vector<unsigned char> even(sizeof(SmemEven48));
     std::vector<unsigned char> gv(sizeof(SmemGv48));
     std::vector<unsigned char> enc(sizeof(EncSmem48));
+    std::unique_ptr<SearchImage48> search_image(new SearchImage48);
     std::vector<unsigned char> enc72(sizeof(EncSmem72));
     std::vector<unsigned long long> keys72;
     llvq_status st;
@@ -1070,6 +1155,7 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
             st = build_gv48(T, *reinterpret_cast<const Smem48 *>(image.data()), *reinterpret_cast<const SmemEven48 *>(even.data()),
                             *reinterpret_cast<SmemGv48 *>(gv.data()), err);
         if (st == LLVQ_OK) st = build_enc48(T, *reinterpret_cast<EncSmem48 *>(enc.data()), err);
+        if (st == LLVQ_OK) st = build_search48(T, *search_image, err);
     } else {
         image.resize(sizeof(Smem72));
         st = build_image72(T, *reinterpret_cast<Smem72 *>(image.data()), recs, guide, err);
@@ -1096,8 +1182,8 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out) {
               cudaMemcpy(c->d_tabC48, tabC.data(), tabC.size() * sizeof(uint32_t), cudaMemcpyHostToDevice) == cudaSuccess &&
               cudaMalloc(&c->d_gv48, gv.size()) == cudaSuccess &&
               cudaMemcpy(c->d_gv48, gv.data(), gv.size(), cudaMemcpyHostToDevice) == cudaSuccess &&
-
-              true;
+              cudaMalloc(&c->d_search48, sizeof(SearchImage48)) == cudaSuccess &&
+              cudaMemcpy(c->d_search48, search_image.get(), sizeof(SearchImage48), cudaMemcpyHostToDevice) == cudaSuccess;
     }
     if (okc && index_bits == 72) {
         okc = cudaMalloc(&c->d_recs72, recs.size() * sizeof(Rec72)) == cudaSuccess &&
@@ -1136,6 +1222,7 @@ void llvq_codec_destroy(llvq_codec *c) {
     if (c->d_keys96) cudaFree(c->d_keys96);
     if (c->d_tabC48) cudaFree(c->d_tabC48);
     if (c->d_gv48) cudaFree(c->d_gv48);
+    if (c->d_search48) cudaFree(c->d_search48);
 
     delete c;
 }
@@ -1209,6 +1296,39 @@ llvq_status llvq_gemm_smallbatch(const llvq_codec *c, const llvq_weight *w, cons
 llvq_status llvq_gemv(const llvq_codec *c, const llvq_weight *w, const void *d_x, float *d_y,
                       void *stream) {
     return llvq_gemm_smallbatch(c, w, d_x, 1, d_y, stream);
+}
+
+llvq_status llvq_search(const llvq_codec *c, int32_t max_shell, int32_t mode, double scale, const float *d_X,
+                        int64_t n, int8_t *d_points, double *d_dots, const double *d_gain_levels,
+                        int32_t n_levels, uint8_t *d_gain_codes, void *stream) {
+    if (!c || n < 0) return LLVQ_ERR_ARG;
+    if (c->index_bits != 48) return LLVQ_ERR_UNSUPPORTED;
+    if (max_shell < 2 || max_shell > c->M) return LLVQ_ERR_ARG;
+    if (mode != LLVQ_SEARCH_ANGULAR && mode != LLVQ_SEARCH_EUCLIDEAN) return LLVQ_ERR_ARG;
+    if (mode == LLVQ_SEARCH_EUCLIDEAN && !(std::isfinite(scale) && scale > 0.0)) return LLVQ_ERR_ARG;
+    const bool gains = n_levels != 0 || d_gain_levels || d_gain_codes;
+    if (gains && (mode != LLVQ_SEARCH_ANGULAR || n_levels < 1 || n_levels > 256 || !d_gain_levels || !d_gain_codes ||
+                  !aligned(d_gain_levels, 8)))
+        return LLVQ_ERR_ARG;
+    if (n == 0) return LLVQ_OK;
+    if (!d_X || !d_points || !aligned(d_X, 4) || (d_dots && !aligned(d_dots, 8))) return LLVQ_ERR_ARG;
+    SearchArgs48 a;
+    a.image = (const SearchImage48 *)c->d_search48;
+    a.max_shell = max_shell;
+    a.mode = mode;
+    a.scale = scale;
+    a.X = d_X;
+    a.n = n;
+    a.points = d_points;
+    a.dots = d_dots;
+    a.levels = gains ? d_gain_levels : nullptr;
+    a.n_levels = gains ? n_levels : 0;
+    a.codes = gains ? d_gain_codes : nullptr;
+    a.flags = c->d_flags;
+    // one CTA per vector, two resident per SM
+    const long long grid = std::min<long long>(n, (long long)c->num_sms * 2);
+    k_search48<<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 
 llvq_status llvq_get_error(const llvq_codec *c, void *stream, uint32_t *flags) {

@@ -9,6 +9,8 @@ Recipe (seeds numpy.random.default_rng([20260313, config_id, stream])):
   stream 1  8-bit gain codes (uniform; equiprobable quantile bins) or direct gains
   stream 2  per-row scale sigma_r ~ U[0.5, 2) of the chi(24) gain tables
   stream 3  activations x ~ N(0, 1) rounded to fp16, zero tail from K to K_pad
+  stream 4  Gaussian-source blocks for the search: x ~ N(0, I_24) in fp32 (the pages' 2-bit
+            Gaussian-source experiment: zero-mean, unit-variance i.i.d. coordinates)
 Layer shapes follow Llama-2 linear layers; real weights are not available, so uniform indices
 stand in for quantised weight blocks.
 """
@@ -91,3 +93,8 @@ def activations(g: np.random.Generator, batch: int, K: int) -> np.ndarray:
     x = np.zeros((batch, k_pad(K)), np.float16)
     x[:, :K] = g.standard_normal((batch, K)).astype(np.float16)
     return x
+
+
+def gaussian_blocks(g: np.random.Generator, n: int) -> np.ndarray:
+    """n blocks of 24 i.i.d. zero-mean unit-variance Gaussian values, fp32 [n, 24]."""
+    return g.standard_normal((n, BLOCK), dtype=np.float64).astype(np.float32)

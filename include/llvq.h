@@ -59,6 +59,11 @@ typedef enum {
 #define LLVQ_FLAG_WAIT_TIMEOUT 0x2u /* a bounded wait (table copy, tensor-core products) gave up;
                                        the output of that call is incomplete */
 #define LLVQ_FLAG_NOT_CODED 0x4u    /* llvq_encode met a vector that is not a coded lattice point */
+#define LLVQ_FLAG_SEARCH_INPUT 0x8u /* llvq_search met a row holding a NaN or an infinity */
+
+/* Criteria of llvq_search. */
+#define LLVQ_SEARCH_ANGULAR 0       /* maximize <x, v> / |v| (the shape of a shape-gain split) */
+#define LLVQ_SEARCH_EUCLIDEAN 1     /* minimize |x - scale * v| (spherical clipping) */
 
 /* Opaque codec: owns the decode tables of one index budget on one device. */
 typedef struct llvq_codec llvq_codec;
@@ -174,6 +179,33 @@ typedef struct {
     uint32_t vals[4];
 } llvq_class96;
 llvq_status llvq_class_table96(int32_t m, llvq_class96 *out, int64_t capacity, int64_t *n_classes);
+
+/* Nearest-point search over the shell union Shell(2) u ... u Shell(max_shell) of the 48-bit
+ * budget: for each row x of d_X, the lattice point v (sqrt(8)-scaled coordinates, |v|^2 = 16 m on
+ * shell m) that maximizes <x, v> / |v| (LLVQ_SEARCH_ANGULAR: the direction of a shape-gain split)
+ * or minimizes |x - scale * v| (LLVQ_SEARCH_EUCLIDEAN: spherical clipping, reconstruction
+ * scale * v).  Source: papernotes.org notes, 方法详解 / 关键设计 1 (search over the union of shells,
+ * unit vectors compared by their inner product for the shape-gain split) and gist.science,
+ * Methodik 2 (Euclidean distance for spherical shaping, cosine similarity for shape-gain, both
+ * over the union; an extension of Adoul & Barth's single-shell search).  The search is exact: it
+ * takes the best point of every class and Golay codeword in closed form (rearrangement of the
+ * sorted |x_i|), in fp64.  Ties between equally good points go to the lower class (index order),
+ * then the lower codeword mask.
+ *   codec: 48-bit (others: LLVQ_ERR_UNSUPPORTED); 2 <= max_shell <= 13.  Shells 2..11 fit 46
+ *     index bits, 2..12 47 bits, 2..13 48 bits; every point found encodes with llvq_encode.
+ *   scale: Euclidean only, finite and > 0 (ignored by the angular criterion).
+ *   d_X: device fp32 [n][24], 4-byte aligned.  d_points: device int8 [n][24], overwritten.
+ *   d_dots: device fp64 [n] (<x, v>), 8-byte aligned, or NULL.
+ *   d_gain_levels / n_levels / d_gain_codes: angular only, optional (all NULL / 0, or all set with
+ *     1 <= n_levels <= 256): d_gain_codes[i] = the level nearest to <x, v> / |v| (the best gain for
+ *     the direction v / |v|), ties to the lower level; device fp64 levels, 8-byte aligned; device
+ *     uint8 codes.
+ * A row holding a NaN or an infinity gets the zero point, a NaN dot and code 0, and raises
+ * LLVQ_FLAG_SEARCH_INPUT.  One CTA per row (grid up to 2 per SM); no allocation. */
+llvq_status llvq_search(const llvq_codec *codec, int32_t max_shell, int32_t mode, double scale,
+                        const float *d_X, int64_t n, int8_t *d_points, double *d_dots,
+                        const double *d_gain_levels, int32_t n_levels, uint8_t *d_gain_codes,
+                        void *stream);
 
 /* Synchronise `stream`, return the sticky device flags raised since the last call in *flags
  * and clear them.  Returns LLVQ_ERR_DEVICE_FLAG when any flag was set, LLVQ_OK otherwise. */
