@@ -335,77 +335,56 @@ llvq_status build_gv48(const HostTables &T, const Smem48 &S, const SmemEven48 &E
     return LLVQ_OK;
 }
 
-// Search tables of the 48-bit budget (k_search48): per class its magnitude groups split by kind
-// (odd: 1 / 3 mod 4; even: on S (2 mod 4) / off S (0 mod 4), zeros dropped), each kind in
-// descending magnitude with steps da and column offsets (kind * 25 + count of that kind's
-// magnitudes >= a_g) * 256; classes odd first, then even by codeword weight, each block by group
-// count descending (equal counts in index order).  Then the codewords: by mask, by (weight, mask).
+// Search tables of the 48-bit budget (k_search48).  The kernel's classes are a compile-time table
+// (search48_classes.cuh); this checks it, class by class, against the codec's own list (shell,
+// coset, magnitude multiset, and the column entries, steps and sign parity derived here from
+// the HostClass), and writes what the point's reconstruction reads: per class its column entries
+// and magnitudes, and the codewords by mask, then by (weight, mask).
 llvq_status build_search48(const HostTables &T, SearchImage48 &I, std::string &err) {
     std::memset(&I, 0, sizeof I);
-    SearchHead48 &H = I.head;
     static const int kWeights[kSrEvenWeights] = {0, 8, 12, 16, 24};
-    struct Item { int id, ng; };
-    std::vector<Item> blocks[kSrBlocks];
-    for (size_t i = 0; i < T.classes.size(); i++) {
-        const HostClass &c = T.classes[i];
-        int b = 0, ng = 0;
-        if (!c.odd) {
-            b = -1;
-            for (int w = 0; w < kSrEvenWeights; w++) if (kWeights[w] == c.k) b = 1 + w;
-            if (b < 0) { err = "search: even class of an unexpected codeword weight"; return LLVQ_ERR_UNSUPPORTED; }
-        }
-        for (int v : c.vals) ng += v != 0;
-        if (ng < 1 || ng > kSrGroups) { err = "search: magnitude groups out of range"; return LLVQ_ERR_UNSUPPORTED; }
-        blocks[b].push_back({(int)i, ng});
-    }
-    int j = 0;
-    for (int b = 0; b < kSrBlocks; b++) {
-        std::stable_sort(blocks[b].begin(), blocks[b].end(), [](const Item &x, const Item &y) { return x.ng > y.ng; });
-        if (b == 0) H.n_odd = (int)blocks[0].size();
-        for (int G = kSrGroups; G >= 1; G--) {
-            H.ng_base[b][kSrGroups - G] = j;
-            for (const Item &it : blocks[b]) {
-                if (it.ng != G) continue;
-                const HostClass &c = T.classes[it.id];
-                if (j >= kSrClasses || c.m > 255) { err = "search: class table too large"; return LLVQ_ERR_UNSUPPORTED; }
-                SearchRec48 &K = H.rec[j];
-                std::vector<std::pair<int, int>> kind[2];       // (magnitude, count), descending
-                for (size_t g = 0; g < c.vals.size(); g++) {
-                    const int a = c.vals[g];
-                    if (a == 0) continue;
-                    kind[c.odd ? (a % 4 == 3) : (a % 4 == 0)].push_back({a, c.cnts[g]});
-                }
-                int g = 0;
-                for (int kd = 0; kd < 2; kd++) {
-                    std::sort(kind[kd].begin(), kind[kd].end(), [](auto x, auto y) { return x.first > y.first; });
-                    int cum = 0;
-                    for (size_t u = 0; u < kind[kd].size(); u++, g++) {
-                        cum += kind[kd][u].second;
-                        const int next = u + 1 < kind[kd].size() ? kind[kd][u + 1].first : 0;
-                        K.da[g] = (double)(kind[kd][u].first - next);
-                        K.off[g] = (uint16_t)((kd * kSrCols + cum) * kSrRowBytes);
-                        I.mag[j][g] = (uint8_t)kind[kd][u].first;
-                    }
-                }
-                K.ng = (uint8_t)g;
-                K.m = (uint8_t)c.m;
-                K.id = (uint16_t)it.id;
-                if (!c.odd) {
-                    K.turn = kind[0].empty() ? 0.0 : 2.0 * (double)kind[0].back().first;
-                    K.q = (uint8_t)(c.k > 0 ? (c.sum_abs / 4) & 1 : 0);
-                }
-                j++;
+    const search_cx::Table &X = search_cx::kTable;
+    if ((int)T.classes.size() != X.n || X.n > kSrClasses) { err = "search: class count differs from the compile-time table"; return LLVQ_ERR_UNSUPPORTED; }
+    for (int id = 0; id < X.n; id++) {
+        const HostClass &c = T.classes[id];
+        const search_cx::Cls &x = X.c[id];
+        // (magnitude, count) descending, zeros included, against the compile-time multiset
+        std::vector<std::pair<int, int>> all;
+        for (size_t g = 0; g < c.vals.size(); g++) all.push_back({c.vals[g], c.cnts[g]});
+        std::sort(all.begin(), all.end(), [](auto a, auto b) { return a.first > b.first; });
+        bool same = x.m == c.m && x.odd == (int)c.odd && x.nv == (int)all.size() && (c.odd || x.k == c.k);
+        for (size_t g = 0; same && g < all.size(); g++) same = x.val[g] == all[g].first && x.cnt[g] == all[g].second;
+        // groups of the two kinds, descending, with cumulative counts
+        SearchRec48 &K = I.rec[id];
+        int g = 0;
+        for (int kd = 0; kd < 2 && same; kd++) {
+            int cum = 0;
+            std::vector<std::pair<int, int>> kind;
+            for (auto &vc : all)
+                if (vc.first != 0 && (c.odd ? (vc.first % 4 == 3) : (vc.first % 4 == 0)) == (kd == 1)) kind.push_back(vc);
+            for (size_t u = 0; u < kind.size() && same; u++, g++) {
+                if (g >= kSrGroups) { same = false; break; }
+                cum += kind[u].second;
+                const int next = u + 1 < kind.size() ? kind[u + 1].first : 0;
+                K.e[g] = (uint8_t)(kd * kSrCols + cum);
+                K.mag[g] = (uint8_t)kind[u].first;
+                same = x.e[g] == K.e[g] && x.da[g] == kind[u].first - next;
             }
         }
-        H.ng_base[b][kSrGroups] = j;
+        K.ng = (uint8_t)g;
+        K.m = (uint8_t)c.m;
+        K.odd = (uint8_t)c.odd;
+        K.q = (uint8_t)(!c.odd && c.k > 0 ? (c.sum_abs / 4) & 1 : 0);
+        same = same && x.ng == g && x.q == K.q;
+        if (!same) { err = "search: compile-time class table differs from the codec's class " + std::to_string(id); return LLVQ_ERR_UNSUPPORTED; }
     }
-    for (int w = 0; w < kSrEvenWeights; w++) H.word_base[w] = T.weight_base[kWeights[w]];
-    H.word_base[kSrEvenWeights] = 4096;
-    H.chunk_base[0] = 0;
+    for (int w = 0; w < kSrEvenWeights; w++) I.word_base[w] = T.weight_base[kWeights[w]];
+    I.word_base[kSrEvenWeights] = 4096;
+    I.chunk_base[0] = 0;
     for (int w = 0; w < kSrEvenWeights; w++) {
-        for (int t = H.word_base[w]; t < H.word_base[w + 1]; t++)
+        for (int t = I.word_base[w]; t < I.word_base[w + 1]; t++)
             if (__builtin_popcount(T.golay_by_weight[t]) != kWeights[w]) { err = "search: codeword weights"; return LLVQ_ERR_UNSUPPORTED; }
-        H.chunk_base[w + 1] = H.chunk_base[w] + (H.word_base[w + 1] - H.word_base[w] + 31) / 32;
+        I.chunk_base[w + 1] = I.chunk_base[w] + (I.word_base[w + 1] - I.word_base[w] + 31) / 32;
     }
     std::memcpy(I.words, T.golay_by_mask, 4096 * sizeof(uint32_t));
     std::memcpy(I.words + 4096, T.golay_by_weight, 4096 * sizeof(uint32_t));
@@ -1006,7 +985,8 @@ void set_kernel_attrs() {
         set_bin48_attrs(std::make_integer_sequence<int, 7>{});
         set_gemv48_attrs(std::make_integer_sequence<int, 2>{});
         cudaFuncSetAttribute(k_encode48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem48));
-        cudaFuncSetAttribute(k_search48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SearchSmem48));
+        cudaFuncSetAttribute(k_search48<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SearchSmem48));
+        cudaFuncSetAttribute(k_search48<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(SearchSmem48));
         cudaFuncSetAttribute(k_encode72, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem72));
         cudaFuncSetAttribute(k_encode96, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sizeof(EncSmem96));
         cudaFuncSetAttribute(k_gemm_tc48, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc48_smem_bytes());
@@ -1325,9 +1305,12 @@ llvq_status llvq_search(const llvq_codec *c, int32_t max_shell, int32_t mode, do
     a.n_levels = gains ? n_levels : 0;
     a.codes = gains ? d_gain_codes : nullptr;
     a.flags = c->d_flags;
-    // one CTA per vector, two resident per SM
-    const long long grid = std::min<long long>(n, (long long)c->num_sms * 2);
-    k_search48<<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
+    // one CTA per vector, one resident per SM
+    const long long grid = std::min<long long>(n, (long long)c->num_sms);
+    if (mode == LLVQ_SEARCH_ANGULAR)
+        k_search48<0><<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
+    else
+        k_search48<1><<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
     return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 

@@ -37,71 +37,57 @@
 //
 // Work split: one CTA per input vector.  Warp 0 sorts the input into shared memory; then each
 // lane owns one codeword (chunks of 32 codewords: the 4096 for the odd classes, then the even
-// codewords of weight 0, 8, 12, 16, 24 for the even classes of that weight), builds its G1 / G3
-// (even: C_on / C_off) columns in shared memory in a sequential pass over the 24 ranks, and the
-// warp walks the classes of the chunk together: the class is uniform across the warp, so its
-// record (column offsets, steps da_g, criterion coefficients) is one broadcast read of shared
-// memory, and each lane reads only its own column (conflict-free: element c of lane l at
-// [c][l]).  Classes are grouped by their number of magnitude groups, so that each group count
-// runs a fully unrolled loop.  All arithmetic is fp64.  The CTA
+// codewords of weight 0, 8, 12, 16, 24 for the even classes of that weight) and builds the prefix
+// sums of its two sets in a sequential pass over the 24 ranks (a shared-memory column, element c
+// of lane l at [c][l], conflict-free), loads the 50 entries into registers and, for odd
+// codewords, continues each set past its end there.  The 383 classes of the union are a
+// compile-time table (search48_classes.cuh, checked against the codec's class list when a codec
+// is created), so every class is a straight-line chain of fp64 FMAs on registers with constant
+// steps.  The criterion is a template parameter: angular V / sqrt(16 m), Euclidean (divided by
+// 2 c > 0, which keeps the order) V - 8 c m, with m and 1 / sqrt(16 m) compile-time constants.  The CTA
 // keeps the best (criterion, class ordinal, codeword), ties going to the lower class ordinal and
 // then the lower codeword mask, and warp 0 writes the point.
 #pragma once
 #include <climits>
 #include <cstdint>
+#include <utility>
 
 #include "device_common.cuh"
 #include "kernels.cuh"
+#include "search48_classes.cuh"
 
 namespace llvq {
 
-constexpr int kSrGroups = 5;       // distinct nonzero magnitudes a 48-bit class can have
+constexpr int kSrGroups = search_cx::kGroups;
 constexpr int kSrClasses = 384;    // 383 classes of the 48-bit union
-constexpr int kSrWarps = 6;        // two CTAs per SM: 2 x (6 warps x 12.8 KB of columns + the class table)
+constexpr int kSrWarps = 12;       // one CTA per SM: 12 x 12.8 KB of columns, about 168 registers a thread
 constexpr int kSrThreads = kSrWarps * 32;
 constexpr int kSrEvenWeights = 5;  // even codeword weights 0, 8, 12, 16, 24
-constexpr int kSrBlocks = 1 + kSrEvenWeights;   // class blocks: odd, then even by weight
-constexpr int kSrCols = 25;        // entries of one set's column: counts 0..24
-constexpr int kSrRowBytes = 32 * 8;             // one column entry for the warp's 32 lanes
+constexpr int kSrCols = search_cx::kCols;
 constexpr int kSrOddChunks = 4096 / 32;
+constexpr int kSrWords = 8192;
 
-// One class as the kernel reads it (80 bytes, shared memory, the same class on every lane).
+// One class for the point's reconstruction (global memory, indexed by the class ordinal).
 struct SearchRec48 {
-    uint16_t off[kSrGroups];       // byte offset of the group's column entry: (kind * 25 + hi_g) * 256
-                                   // (odd: 1- then 3-mod-4 kind; even: on S then off S)
-    uint16_t id;                   // ordinal in index order (ties)
-    uint8_t q;                     // even: parity of the negative signs the class needs on S
-    uint8_t m;                     // shell
+    uint8_t e[kSrGroups];          // column entry: kind * 25 + count of the kind's magnitudes >= a_g
+    uint8_t mag[kSrGroups];        // a_g
     uint8_t ng;                    // groups
-    uint8_t pad_;
-    double da[kSrGroups];          // a_g - a_{g+1} within the group's kind
-    double turn;                   // even: 2 x the smallest 2-mod-4 magnitude (sign-turn cost per unit weight)
-    double alpha, beta;            // criterion = alpha V + beta, set per launch (-inf: class off)
+    uint8_t m;                     // shell
+    uint8_t odd;
+    uint8_t q;                     // even: parity of the negative signs the class needs on S
+    uint8_t pad_[2];
 };
-static_assert(sizeof(SearchRec48) == 80, "one class in 80 bytes");
+static_assert(sizeof(SearchRec48) == 16, "one class in 16 bytes");
 
-// The part every CTA copies into shared memory.  Blocks: b = 0 the odd classes, b = 1 + w the
-// even classes of codeword weight index w (0, 8, 12, 16, 24); within a block, classes by group
-// count descending, those with G groups in [ng_base[b][5 - G], ng_base[b][6 - G]).  Codeword
-// chunks: [0, kSrOddChunks) the odd codewords, kSrOddChunks + [chunk_base[w], chunk_base[w + 1])
-// the even codewords of weight index w, by-weight slots [word_base[w], word_base[w + 1]).
-struct SearchHead48 {
+// Device image: the class records by ordinal, the codeword chunk bounds and the codewords:
+// [0, 4096) ascending mask (the odd classes' T), [4096, 8192) ascending (weight, mask) (the even
+// classes' S).  Chunks: [0, kSrOddChunks) the odd codewords, kSrOddChunks + [chunk_base[w],
+// chunk_base[w + 1]) the even codewords of weight index w, by-weight slots [word_base[w],
+// word_base[w + 1]).
+struct SearchImage48 {
     SearchRec48 rec[kSrClasses];
-    int n_odd;
-    int ng_base[kSrBlocks][kSrGroups + 1];
     int word_base[kSrEvenWeights + 1];
     int chunk_base[kSrEvenWeights + 1];
-    int pad_[3];
-};
-static_assert(sizeof(SearchHead48) % 16 == 0, "copied in 16-byte units");
-
-// Device image: the head, then per class its group magnitudes (the point's reconstruction, read
-// from global memory), then the codewords: [0, 4096) ascending mask (the odd classes' T),
-// [4096, 8192) ascending (weight, mask) (the even classes' S).
-constexpr int kSrWords = 8192;
-struct SearchImage48 {
-    SearchHead48 head;
-    uint8_t mag[kSrClasses][8];
     uint32_t words[kSrWords];
 };
 
@@ -121,7 +107,6 @@ struct SearchArgs48 {
 };
 
 struct SearchSmem48 {
-    SearchHead48 head;
     double col[kSrWarps][2 * kSrCols][32];        // per warp: entry e of lane l at [e][l]
     double w[24];                                 // |y| by rank (descending)
     int ord[24];                                  // rank -> position
@@ -129,92 +114,142 @@ struct SearchSmem48 {
     uint32_t negmask;                             // bit i: y_i < 0
     int bad;                                      // the row holds a NaN or an infinity
     int pad_;
+    int word_base[kSrEvenWeights + 1];
+    int chunk_base[kSrEvenWeights + 1];
     double red_f[kSrWarps];
-    int red_j[kSrWarps], red_id[kSrWarps];
+    int red_id[kSrWarps];
     uint32_t red_w[kSrWarps];
 };
-// two CTAs per SM: 228 KB per SM, 1 KB reserved per CTA
-static_assert(2 * (sizeof(SearchSmem48) + 1024) <= 228 * 1024, "two CTAs per SM");
+static_assert(sizeof(SearchSmem48) + 1024 <= 228 * 1024, "one CTA per SM");
 
 __device__ __forceinline__ bool sr_better(double f, int id, uint32_t w, double bf, int bid, uint32_t bw) {
     return f > bf || (f == bf && (id < bid || (id == bid && w < bw)));
 }
 
-__device__ __forceinline__ void sr_reduce(double &bf, int &bj, int &bid, uint32_t &bw) {
+__device__ __forceinline__ void sr_reduce(double &bf, int &bid, uint32_t &bw) {
     for (int off = 16; off; off >>= 1) {
         const double of = __shfl_xor_sync(0xFFFFFFFFu, bf, off);
-        const int oj = __shfl_xor_sync(0xFFFFFFFFu, bj, off), oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
+        const int oid = __shfl_xor_sync(0xFFFFFFFFu, bid, off);
         const uint32_t ow = __shfl_xor_sync(0xFFFFFFFFu, bw, off);
-        if (sr_better(of, oid, ow, bf, bid, bw)) { bf = of; bj = oj; bid = oid; bw = ow; }
+        if (sr_better(of, oid, ow, bf, bid, bw)) { bf = of; bid = oid; bw = ow; }
     }
 }
 
 // the magnitude at descending rank r (0-based) among a class's magnitudes of one kind (0 past them)
-__device__ __forceinline__ int sr_mag(const SearchRec48 &K, const uint8_t *mag, int second_kind, int r) {
+__device__ __forceinline__ int sr_mag(const SearchRec48 &K, int second_kind, int r) {
     for (int g = 0; g < K.ng; g++) {
-        const int e = K.off[g] / kSrRowBytes, kind = e >= kSrCols;
-        if (kind == second_kind && r < e - kind * kSrCols) return mag[g];
+        const int kind = K.e[g] >= kSrCols;
+        if (kind == second_kind && r < K.e[g] - kind * kSrCols) return K.mag[g];
     }
     return 0;
 }
 
 struct SrBest {
     double f;
-    int j, id;
+    int id;
     uint32_t w;
 };
 
-// classes [jb, je) with G groups each, against this lane's column (colb: its entry 0)
-template <bool ODD, int G>
-__device__ __forceinline__ void sr_eval(const SearchRec48 *R, int jb, int je, const char *colb, uint32_t word,
-                                        bool valid, int turn, double wlast, SrBest &b) {
-#pragma unroll 2
-    for (int j = jb; j < je; j++) {
-        const SearchRec48 &K = R[j];
-        double V = 0.0;
+// 1 / sqrt(x) for the compile-time criterion constants (Newton's iteration from 0.1, which lies
+// below sqrt(3 / x) for every x = 16 m <= 208, so the iteration converges; 12 steps reach the
+// fp64 rounding level)
+constexpr double sr_rsqrt(double x) {
+    double y = 0.1;
+    for (int i = 0; i < 12; i++) y = y * (1.5 - 0.5 * x * y * y);
+    return y;
+}
+
+struct SrCrit {
+    double nc8;               // Euclidean: -8 c
+    int max_shell;
+};
+
+// criterion value of class J of the compile-time table against this lane's column entries
+// (-inf when its shell is outside the union)
+template <int MODE, int J>
+__device__ __forceinline__ double sr_class(const double (&c)[2 * kSrCols], const SrCrit &cr, int turn,
+                                           double wlast) {
+    constexpr search_cx::Cls K = search_cx::kTable.c[J];
+    double V = 0.0;
 #pragma unroll
-        for (int g = 0; g < G; g++) V = fma(K.da[g], *reinterpret_cast<const double *>(colb + K.off[g]), V);
-        if (!ODD && turn != K.q) V = fma(-K.turn, wlast, V);
-        const double f = fma(K.alpha, V, K.beta);
-        if (valid && sr_better(f, K.id, word, b.f, b.id, b.w)) { b.f = f; b.j = j; b.id = K.id; b.w = word; }
+    for (int g = 0; g < K.ng; g++) V = fma((double)K.da[g], c[K.e[g]], V);
+    if constexpr (!K.odd && K.k > 0) {
+        if (turn != K.q) V = fma(-(double)K.turn2, wlast, V);
     }
+    double f;
+    if constexpr (MODE == 0) {
+        constexpr double r = sr_rsqrt(16.0 * K.m);
+        f = V * r;
+    } else {
+        f = fma((double)K.m, cr.nc8, V);
+    }
+    return K.m <= cr.max_shell ? f : -INFINITY;
 }
 
-template <bool ODD>
-__device__ __forceinline__ void sr_eval_block(const SearchRec48 *R, const int *nb, const char *colb, uint32_t word,
-                                              bool valid, int turn, double wlast, SrBest &b) {
-    sr_eval<ODD, 5>(R, nb[0], nb[1], colb, word, valid, turn, wlast, b);
-    sr_eval<ODD, 4>(R, nb[1], nb[2], colb, word, valid, turn, wlast, b);
-    sr_eval<ODD, 3>(R, nb[2], nb[3], colb, word, valid, turn, wlast, b);
-    sr_eval<ODD, 2>(R, nb[3], nb[4], colb, word, valid, turn, wlast, b);
-    sr_eval<ODD, 1>(R, nb[4], nb[5], colb, word, valid, turn, wlast, b);
+// class lists: 0 the odd classes, 1 + w the even classes of codeword weight index w
+constexpr int sr_list_n(int list) {
+    return list == 0 ? search_cx::kTable.n_odd : search_cx::kTable.n_even[list - 1];
+}
+constexpr int sr_list_id(int list, int i) {
+    return list == 0 ? search_cx::kTable.odd_ids[i] : search_cx::kTable.even_ids[list - 1][i];
 }
 
-__global__ void __launch_bounds__(kSrThreads, 2) k_search48(const SearchArgs48 a) {
+// classes B, B + 1, ... of list LST (up to four, ascending ordinals): four independent chains, the
+// best of them (the lower ordinal on equal values), then one comparison with the running best
+template <int MODE, int LST, int B>
+__device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const SrCrit &cr, uint32_t word,
+                                        bool valid, int turn, double wlast, SrBest &b) {
+    constexpr int N = sr_list_n(LST);
+    constexpr int j0 = sr_list_id(LST, B);
+    double f = sr_class<MODE, j0>(c, cr, turn, wlast);
+    int id = j0;
+    if constexpr (B + 1 < N) {
+        constexpr int j1 = sr_list_id(LST, B + 1);
+        constexpr int j2 = sr_list_id(LST, B + 2 < N ? B + 2 : B + 1);
+        constexpr int j3 = sr_list_id(LST, B + 3 < N ? B + 3 : B + 1);
+        const double f1 = sr_class<MODE, j1>(c, cr, turn, wlast);
+        double f2 = -INFINITY, f3 = -INFINITY;
+        if constexpr (B + 2 < N) f2 = sr_class<MODE, j2>(c, cr, turn, wlast);
+        if constexpr (B + 3 < N) f3 = sr_class<MODE, j3>(c, cr, turn, wlast);
+        int id2 = j2;
+        if (f1 > f) { f = f1; id = j1; }
+        if (f3 > f2) { f2 = f3; id2 = j3; }
+        if (f2 > f) { f = f2; id = id2; }
+    }
+    if (valid && f >= b.f && sr_better(f, id, word, b.f, b.id, b.w)) { b.f = f; b.id = id; b.w = word; }
+}
+
+template <int MODE, int LST, int... Q>
+__device__ __forceinline__ void sr_list(std::integer_sequence<int, Q...>, const double (&c)[2 * kSrCols],
+                                        const SrCrit &cr, uint32_t word, bool valid, int turn, double wlast,
+                                        SrBest &b) {
+    (sr_quad<MODE, LST, 4 * Q>(c, cr, word, valid, turn, wlast, b), ...);
+}
+
+template <int MODE, int LST>
+__device__ __forceinline__ void sr_block(const double (&c)[2 * kSrCols], const SrCrit &cr, uint32_t word,
+                                         bool valid, int turn, double wlast, SrBest &b) {
+    sr_list<MODE, LST>(std::make_integer_sequence<int, (sr_list_n(LST) + 3) / 4>{}, c, cr, word, valid, turn,
+                       wlast, b);
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kSrThreads, 1) k_search48(const SearchArgs48 a) {
     extern __shared__ __align__(16) unsigned char sr_raw[];
     SearchSmem48 &S = *reinterpret_cast<SearchSmem48 *>(sr_raw);
     const unsigned FULL = 0xFFFFFFFFu;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    load_smem_image(&S.head, &a.image->head, sizeof(SearchHead48));
-    __syncthreads();
-    for (int j = tid; j < kSrClasses; j += kSrThreads) {
-        SearchRec48 &K = S.head.rec[j];
-        const int m = K.m;
-        const bool on = m >= 2 && m <= a.max_shell;
-        const double al = a.mode == 0 ? 1.0 / sqrt(16.0 * (double)(m ? m : 1)) : 2.0 * a.scale;
-        const double be = a.mode == 0 ? 0.0 : -a.scale * a.scale * 16.0 * (double)m;
-        K.alpha = on ? al : 0.0;
-        K.beta = on ? be : -INFINITY;
+    const SrCrit cr{-8.0 * a.scale, a.max_shell};
+    if (tid < kSrEvenWeights + 1) {
+        S.word_base[tid] = a.image->word_base[tid];
+        S.chunk_base[tid] = a.image->chunk_base[tid];
     }
     double(*col)[32] = S.col[warp];
     col[0][lane] = 0.0;                     // count 0 of either set: never rewritten
     col[kSrCols][lane] = 0.0;
-    const char *colb = reinterpret_cast<const char *>(&col[0][lane]);
-    const SearchRec48 *R = S.head.rec;
-    const int n_odd = S.head.n_odd;
-    const int n_chunks = kSrOddChunks + S.head.chunk_base[kSrEvenWeights];
     const bool act = lane < 24;
     __syncthreads();
+    const int n_chunks = kSrOddChunks + S.chunk_base[kSrEvenWeights];
 
     for (long long v = blockIdx.x; v < a.n; v += gridDim.x) {
         // ---- warp 0: the input sorted by |y_i| descending (equal values by position) ---------
@@ -247,7 +282,7 @@ __global__ void __launch_bounds__(kSrThreads, 2) k_search48(const SearchArgs48 a
         }
         const uint32_t posb = S.pos, negmask = S.negmask;
 
-        SrBest best{-INFINITY, -1, INT_MAX, 0u};
+        SrBest best{-INFINITY, INT_MAX, 0u};
         for (int ch = warp; ch < n_chunks; ch += kSrWarps) {
             // ---- this lane's codeword --------------------------------------------------------
             const bool odd = ch < kSrOddChunks;
@@ -258,9 +293,9 @@ __global__ void __launch_bounds__(kSrThreads, 2) k_search48(const SearchArgs48 a
                 word = __ldg(a.image->words + ch * 32 + lane);
             } else {
                 const int e = ch - kSrOddChunks;
-                while (e >= S.head.chunk_base[wi + 1]) wi++;
-                const int t = S.head.word_base[wi] + (e - S.head.chunk_base[wi]) * 32 + lane;
-                valid = t < S.head.word_base[wi + 1];
+                while (e >= S.chunk_base[wi + 1]) wi++;
+                const int t = S.word_base[wi] + (e - S.chunk_base[wi]) * 32 + lane;
+                valid = t < S.word_base[wi + 1];
                 word = valid ? __ldg(a.image->words + 4096 + t) : 0u;
             }
             // ---- prefix sums of the sorted weights in the two sets, one pass over the ranks ----
@@ -273,64 +308,73 @@ __global__ void __launch_bounds__(kSrThreads, 2) k_search48(const SearchArgs48 a
                 if (b) { s1 += wt; c1++; col[c1][lane] = s1; wlast = wt; }
                 else { s2 += wt; c2++; col[kSrCols + c2][lane] = s2; }
             }
-            if (odd) {                                      // continue each set past its end
+            double c[2 * kSrCols];
+#pragma unroll
+            for (int e = 0; e < 2 * kSrCols; e++) c[e] = (e % kSrCols) ? col[e][lane] : 0.0;
+            if (odd) {
+                // continue each set past its end: entries c > c1 of the first set read raw entries
+                // 24 - c < c2 of the second, and the other way round, so the order is free
                 const double d = s1 - s2;
-                for (int c = 1; c < kSrCols; c++) {
-                    if (c > c1) col[c][lane] = d + col[kSrCols + 24 - c][lane];
-                    if (c > c2) col[kSrCols + c][lane] = col[24 - c][lane] - d;
+#pragma unroll
+                for (int e = 1; e < kSrCols; e++) {
+                    if (e > c1) c[e] = d + c[kSrCols + 24 - e];
+                    if (e > c2) c[kSrCols + e] = c[24 - e] - d;
                 }
-                sr_eval_block<true>(R, S.head.ng_base[0], colb, word, true, 0, 0.0, best);
+                sr_block<MODE, 0>(c, cr, word, true, 0, 0.0, best);
             } else {
                 const int turn = __popc(word & negmask) & 1;
-                sr_eval_block<false>(R, S.head.ng_base[1 + wi], colb, word, valid, turn, wlast, best);
+                switch (wi) {
+                    case 0: sr_block<MODE, 1>(c, cr, word, valid, turn, wlast, best); break;
+                    case 1: sr_block<MODE, 2>(c, cr, word, valid, turn, wlast, best); break;
+                    case 2: sr_block<MODE, 3>(c, cr, word, valid, turn, wlast, best); break;
+                    case 3: sr_block<MODE, 4>(c, cr, word, valid, turn, wlast, best); break;
+                    default: sr_block<MODE, 5>(c, cr, word, valid, turn, wlast, best); break;
+                }
             }
         }
 
         // ---- the best over the CTA -----------------------------------------------------------
         double bf = best.f;
-        int bj = best.j, bid = best.id;
+        int bid = best.id;
         uint32_t bw = best.w;
-        sr_reduce(bf, bj, bid, bw);
-        if (lane == 0) { S.red_f[warp] = bf; S.red_j[warp] = bj; S.red_id[warp] = bid; S.red_w[warp] = bw; }
+        sr_reduce(bf, bid, bw);
+        if (lane == 0) { S.red_f[warp] = bf; S.red_id[warp] = bid; S.red_w[warp] = bw; }
         __syncthreads();
         if (warp == 0) {
             const int r = lane < kSrWarps ? lane : 0;
-            bf = S.red_f[r]; bj = S.red_j[r]; bid = S.red_id[r]; bw = S.red_w[r];
-            sr_reduce(bf, bj, bid, bw);
-            // ---- the point of class bj and codeword bw (lane = rank) ---------------------
-            const int j = bj < 0 ? 0 : bj;
-            const SearchRec48 &K = R[j];
-            const uint8_t *mag = a.image->mag[j];
+            bf = S.red_f[r]; bid = S.red_id[r]; bw = S.red_w[r];
+            sr_reduce(bf, bid, bw);
+            // ---- the point of class bid and codeword bw (lane = rank) --------------------
+            const bool found = bid >= 0 && bid < search_cx::kClasses;
+            const SearchRec48 K = a.image->rec[found ? bid : 0];
             const int ord = act ? S.ord[lane] : 0;
             const double wt = act ? S.w[lane] : 0.0;
             const bool pos = (posb >> lane) & 1u;
             const unsigned le = lane == 31 ? FULL : (2u << lane) - 1u;
             const bool inw = (bw >> ord) & 1u;
             int x;
-            if (j < n_odd) {
+            if (K.odd) {
                 const bool b = act && (inw == pos);
                 const unsigned m1 = __ballot_sync(FULL, b);
                 const int c1 = __popc(m1 & le), c3 = lane + 1 - c1;
                 int n1 = 0;
-                for (int g = 0; g < K.ng; g++) {
-                    const int e = K.off[g] / kSrRowBytes;
-                    if (e < kSrCols) n1 = max(n1, e);
-                }
+                for (int g = 0; g < K.ng; g++)
+                    if (K.e[g] < kSrCols) n1 = max(n1, (int)K.e[g]);
                 const int n3 = 24 - n1;
                 int mg;
-                if (b) mg = c1 <= n1 ? sr_mag(K, mag, 0, c1 - 1) : sr_mag(K, mag, 1, n3 - 1 - (c1 - n1 - 1));
-                else mg = c3 <= n3 ? sr_mag(K, mag, 1, c3 - 1) : sr_mag(K, mag, 0, n1 - 1 - (c3 - n3 - 1));
+                if (b) mg = c1 <= n1 ? sr_mag(K, 0, c1 - 1) : sr_mag(K, 1, n3 - 1 - (c1 - n1 - 1));
+                else mg = c3 <= n3 ? sr_mag(K, 1, c3 - 1) : sr_mag(K, 0, n1 - 1 - (c3 - n3 - 1));
                 x = (((mg & 3) == 1) == inw) ? mg : -mg;
             } else {
                 const bool b = act && inw;
                 const unsigned mS = __ballot_sync(FULL, b);
                 const int con = __popc(mS & le), coff = lane + 1 - con;
-                const int mg = b ? sr_mag(K, mag, 0, con - 1) : sr_mag(K, mag, 1, coff - 1);
+                const int mg = b ? sr_mag(K, 0, con - 1) : sr_mag(K, 1, coff - 1);
                 x = pos ? mg : -mg;
                 const int turn = __popc(bw & negmask) & 1;
                 if (mS && turn != K.q && lane == 31 - __clz(mS)) x = -x;
             }
-            if (!act || bj < 0) x = 0;
+            if (!act || !found) x = 0;
             double d = (pos ? wt : -wt) * (double)x;
             for (int off = 16; off; off >>= 1) d += __shfl_xor_sync(FULL, d, off);
             if (act) a.points[v * 24 + ord] = (int8_t)x;
@@ -339,9 +383,9 @@ __global__ void __launch_bounds__(kSrThreads, 2) k_search48(const SearchArgs48 a
                 const double g = d / sqrt(16.0 * (double)(K.m ? K.m : 1));
                 double be = INFINITY;
                 int bc = INT_MAX;
-                for (int c = lane; c < a.n_levels; c += 32) {
-                    const double e = fabs(g - a.levels[c]);
-                    if (e < be) { be = e; bc = c; }
+                for (int cc = lane; cc < a.n_levels; cc += 32) {
+                    const double e = fabs(g - a.levels[cc]);
+                    if (e < be) { be = e; bc = cc; }
                 }
                 for (int off = 16; off; off >>= 1) {
                     const double oe = __shfl_xor_sync(FULL, be, off);

@@ -201,7 +201,7 @@ llvq_status llvq_class_table96(int32_t m, llvq_class96 *out, int64_t capacity, i
  *     the direction v / |v|), ties to the lower level; device fp64 levels, 8-byte aligned; device
  *     uint8 codes.
  * A row holding a NaN or an infinity gets the zero point, a NaN dot and code 0, and raises
- * LLVQ_FLAG_SEARCH_INPUT.  One CTA per row (grid up to 2 per SM); no allocation. */
+ * LLVQ_FLAG_SEARCH_INPUT.  One CTA per row (one resident per SM); no allocation. */
 llvq_status llvq_search(const llvq_codec *codec, int32_t max_shell, int32_t mode, double scale,
                         const float *d_X, int64_t n, int8_t *d_points, double *d_dots,
                         const double *d_gain_levels, int32_t n_levels, uint8_t *d_gain_codes,
