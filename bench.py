@@ -97,6 +97,19 @@ def profile_record():
     return None
 
 
+def search_record():
+    """The committed ncu record of the search kernel ("search" in profiles/traffic.json), keyed by
+    the kernel sources like profile_record, or None when they changed since the capture."""
+    try:
+        with open(os.path.join(ROOT, "profiles", "traffic.json")) as f:
+            rec = json.load(f).get("search")
+        if rec and rec.get("kernel_sources_sha256") == kernel_sources_hash():
+            return rec
+    except Exception:
+        pass
+    return None
+
+
 def measured_traffic():
     rec = profile_record()
     return int(rec["traffic_bytes_per_launch"]) if rec else None
@@ -299,6 +312,12 @@ def cpu_baseline(steps_seconds=12.0, one_core_seconds=3.0):
 # criterion over shells 2..12, 46.66 bits, or 2..11, 45.20 bits).
 SEARCH_N = 1 << 17
 SEARCH_TRAIN = 1 << 16
+# Algorithmic fp64 FMAs per searched vector: over every (class, codeword) pair of shells 2..M
+# (4096 codewords for an odd class, those of weight k for an even one), one FMA per nonzero
+# magnitude group and one for the criterion (the even classes' data-dependent sign turn is left
+# out).  Counted from the class list of the 48-bit union: 921,486 pairs at M = 13.
+SEARCH_FMAS = {11: 2081740, 12: 2857480, 13: 3805180}
+FP64_FMA_PER_SM_CLK = 64      # ncu: sm__sass_thread_inst_executed_op_dfma_pred_on.sum.peak_sustained / SMs
 SEARCH_CONFIGS = [
     # name, criterion, max_shell, gain bits
     ("spherical clipping", 1, 13, 0),
@@ -392,8 +411,22 @@ def search_throughput(torch, codec, dev, steps, warmup, max_shell=13, mode=1, sc
     if codec.get_error(stream) != 0:
         raise RuntimeError("llvq_search raised a device flag")
     t = total / steps
-    return {"n": SEARCH_N, "max_shell": max_shell, "mode": "euclidean" if mode else "angular",
+    return {"n": SEARCH_N, "max_shell": max_shell, "criterion": "euclidean" if mode else "angular",
             "ms_per_launch": t * 1e3, "vectors_per_s": SEARCH_N / t}
+
+
+def search_roofline(r, sm_mhz, sms):
+    """fp64 roofline of the search kernel: algorithmic FMAs (SEARCH_FMAS) x 2 per second against
+    sms x 64 fp64 FMA lanes x 2 x the SM clock measured under load; DRAM traffic per launch from
+    the committed ncu record when it matches the sources."""
+    flops = 2.0 * SEARCH_FMAS[r["max_shell"]] * r["n"]
+    achieved = flops / (r["ms_per_launch"] / 1e3) / 1e12
+    peak = sms * FP64_FMA_PER_SM_CLK * 2 * sm_mhz * 1e6 / 1e12
+    rec = search_record()
+    return {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "traffic": rec["traffic_bytes_per_launch"] if rec and rec.get("n") == r["n"] else None,
+            "peak_source": f"{sms} SMs x {FP64_FMA_PER_SM_CLK} fp64 FMA/clk x 2 x {sm_mhz:.0f} MHz (clock under load)",
+            "algorithmic": f"{SEARCH_FMAS[r['max_shell']]} fp64 FMAs per vector (class-codeword pairs x (groups + 1))"}
 
 
 def search_cpu_baseline(seconds=12.0, max_shell=13, mode=1, scale=0.3):
@@ -689,11 +722,14 @@ def main():
         if rank == 0:
             with ClockSampler(torch.cuda.current_device()) as clocks:
                 r = search_throughput(torch, codec, dev, args.steps, args.warmup)
-            line = {"mode": "search", "metric": "search_vectors_per_s", "value": r["vectors_per_s"],
+            line = {"metric": "search_vectors_per_s", "value": r["vectors_per_s"],
                     "unit": "vectors/s", "steps": args.steps, "warmup": args.warmup,
                     "config": {"workload": f"nearest point of Leech shells 2..13 (Euclidean, c = 0.3) "
                                            f"for {SEARCH_N} N(0, I_24) blocks", "l2": "flushed"},
                     "dtype": "f64", "data": "synthetic", **r, "clocks": clocks.summary()}
+            props = torch.cuda.get_device_properties(dev)
+            line["roofline"] = search_roofline(r, line["clocks"].get("sm_mhz") or 1965.0,
+                                               props.multi_processor_count)
             if args.search_quality:
                 line["quality"] = search_quality(torch, codec, dev)
             if not args.no_cpu_baseline:
