@@ -79,6 +79,8 @@ def lib():
                                        C.c_int32]
         L.ora_search_brute.restype = C.c_int64
         L.ora_class_best.argtypes = [C.c_void_p, C.c_int32, C.c_int64, C.c_uint32, f64p, i32p, f64p]
+        L.ora_spherical_gptq.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, f64p, f64p, i8p, f64p]
+        L.ora_gptq_block_matrix.argtypes = [C.c_int32, f64p, C.c_int32, f64p]
         L.ora_half_to_double.argtypes = [C.c_uint16]
         L.ora_half_to_double.restype = C.c_double
         _lib = L
@@ -250,6 +252,19 @@ class Codec:
             raise ValueError("no such class, or the word does not fit it")
         return v, d.value
 
+    def spherical_gptq(self, W, U, max_shell: int):
+        """One Spherical GPTQ pass: returns (W after the pass, points int8 [rows, nb, 24], norms
+        [rows, nb]); W fp64 [rows, cols], U fp64 [cols, cols] upper triangular, H^-1 = U^T U."""
+        W = np.array(W, np.float64, order="C", copy=True)
+        U = np.ascontiguousarray(U, np.float64)
+        rows, cols = W.shape
+        nb = cols // 24
+        P = np.zeros((rows, nb, 24), np.int8)
+        Nr = np.zeros((rows, nb), np.float64)
+        if lib().ora_spherical_gptq(self._h, max_shell, rows, cols, _p(W, f64p), _p(U, f64p), _p(P, i8p), _p(Nr, f64p)):
+            raise ValueError("bad Spherical GPTQ arguments")
+        return W, P, Nr
+
     def gemm(self, words: np.ndarray, nb: int, gain_mode: int, gains: np.ndarray, x: np.ndarray,
              batch: int, row_pitch_words: int | None = None, threads: int = 1) -> np.ndarray:
         """fp64 y[batch, rows] from packed words [rows, pitch] (uint64, or uint64 pairs for
@@ -292,6 +307,16 @@ def search_brute(X, m_max: int, mode: int, scale: float = 1.0, threads: int = 1)
     if visited < 0:
         raise ValueError("bad search arguments")
     return V, d, int(visited)
+
+
+def gptq_block_matrix(U, b: int):
+    """G_B = U_BB^-1 U_B,rest of block b ([24, cols], zero before the later columns)."""
+    U = np.ascontiguousarray(U, np.float64)
+    cols = U.shape[0]
+    G = np.zeros((24, cols), np.float64)
+    if lib().ora_gptq_block_matrix(cols, _p(U, f64p), b, _p(G, f64p)):
+        raise ValueError("bad block")
+    return G
 
 
 def search_objective(mode: int, scale: float, dot, norm2):

@@ -16,6 +16,8 @@
  *               ranges; r = I_class mod A, I' = floor(I_class/A), s = I' mod 2^B,
  *               I'' = floor(I'/2^B); r = Golay refinement, s = sign pattern meeting the
  *               congruence check, I'' = lexicographic permutation rank.
+ *   [notes-K3]  papernotes.org, 方法详解 / 关键设计 3: Spherical GPTQ (norm-preserving
+ *               retraction w^ = (|w| / |w~|) w~, residual propagated through chol(H^-1)^T).
  *   [notes-K4]  papernotes.org, 方法详解 / 关键设计 4: fused dequantize-and-multiply.
  *   [gist-M1]   gist.science, Methodik 1: Leech lattice built from G24, integer vectors in
  *               even and odd cosets, shells of equal squared norm.
@@ -1384,4 +1386,79 @@ int ora_class_best(ora_codec *c, int32_t m, int64_t j, uint32_t word, const doub
     }
     drop_shell(c, m);
     return ok ? 0 : -1;
+}
+
+/* ===================================================================================== */
+/* Spherical GPTQ, one pass ([notes-K3] 关键设计 3 "保模长球面曲率反馈": the shape-gain        */
+/* candidate is rescaled to the original norm, w^ = (|w| / |w~|) w~, a retraction onto the   */
+/* product of spheres; the residual E = w - w^ is propagated to the unquantized weights      */
+/* through U = chol(H^-1)^T).  Readings:                                                     */
+/*   - blocks of 24 columns, in column order; each row's block is quantized jointly: its     */
+/*     direction is the angular search over shells 2..max_shell of the block rounded to fp32 */
+/*     (the search's input type), and w~ = g v / |v| for any gain g, so w^ = |w| v / |v|;     */
+/*   - the propagation is the joint (block) form of GPTQ's update: with H^-1 = U^T U (U upper */
+/*     triangular), the inverse Hessian of the columns not yet quantized is the trailing     */
+/*     block of U^T U, so quantizing block B with error E moves the later columns by          */
+/*     -E U_BB^-1 U_B,rest (one column at a time this is GPTQ's -e / U_ii * U_i,rest);        */
+/*   - fixed operation order, so that another implementation can reproduce it bit for bit:    */
+/*     |w|^2 = fma chain over i ascending; ratio = sqrt(|w|^2) / sqrt(16 m); w^_i = ratio v_i; */
+/*     G_B = U_BB^-1 U_B,rest by back substitution per column (g_i = (u_i - sum_{k>i}          */
+/*     U_ik g_k) / U_ii, the sum as an fma chain over k ascending from u_i); the update       */
+/*     W[r][c] -= (fma chain over k ascending of E_k G_B[k][c], from 0).                      */
+/* ===================================================================================== */
+
+int ora_gptq_block_matrix(int32_t cols, const double *U, int32_t b, double *G) {
+    /* G [24][cols]: G_B[k][c] for c >= 24 (b + 1), 0 elsewhere */
+    if (cols % 24 || b < 0 || b >= cols / 24) return -1;
+    const int base = 24 * b;
+    for (int k = 0; k < 24; k++)
+        for (int c = 0; c < cols; c++) G[(size_t)k * cols + c] = 0.0;
+    for (int c = base + 24; c < cols; c++) {
+        for (int i = 23; i >= 0; i--) {
+            double acc = U[(size_t)(base + i) * cols + c];
+            for (int k = i + 1; k < 24; k++)
+                acc = fma(-U[(size_t)(base + i) * cols + base + k], G[(size_t)k * cols + c], acc);
+            G[(size_t)i * cols + c] = acc / U[(size_t)(base + i) * cols + base + i];
+        }
+    }
+    return 0;
+}
+
+int ora_spherical_gptq(ora_codec *c, int32_t max_shell, int32_t rows, int32_t cols, double *W, const double *U,
+                       int8_t *points, double *norms) {
+    if (!c->store_all || max_shell < 2 || max_shell > c->M || rows < 0 || cols <= 0 || cols % 24) return -1;
+    const int nb = cols / 24;
+    double *G = malloc(sizeof(double) * (size_t)24 * cols);
+    double *E = malloc(sizeof(double) * 24 * (size_t)(rows > 0 ? rows : 1));
+    if (!G || !E) { free(G); free(E); return -2; }
+    int rc = 0;
+    for (int b = 0; b < nb && rc == 0; b++) {
+        ora_gptq_block_matrix(cols, U, b, G);
+        for (int r = 0; r < rows; r++) {
+            double *w = W + (size_t)r * cols + 24 * b;
+            double y[ORA_DIM], s = 0.0, d;
+            int32_t v[ORA_DIM];
+            for (int i = 0; i < ORA_DIM; i++) y[i] = (double)(float)w[i];
+            if (ora_search(c, max_shell, 0, 1.0, y, v, &d)) { rc = -1; break; }
+            int n2 = 0;
+            for (int i = 0; i < ORA_DIM; i++) { s = fma(w[i], w[i], s); n2 += v[i] * v[i]; }
+            const double ratio = sqrt(s) / sqrt((double)n2);
+            for (int i = 0; i < ORA_DIM; i++) {
+                const double what = ratio * (double)v[i];
+                E[(size_t)r * 24 + i] = w[i] - what;
+                w[i] = what;
+                points[((size_t)r * nb + b) * 24 + i] = (int8_t)v[i];
+            }
+            norms[(size_t)r * nb + b] = sqrt(s);
+        }
+        for (int r = 0; r < rows && rc == 0; r++)
+            for (int col = 24 * (b + 1); col < cols; col++) {
+                double acc = 0.0;
+                for (int k = 0; k < 24; k++) acc = fma(E[(size_t)r * 24 + k], G[(size_t)k * cols + col], acc);
+                W[(size_t)r * cols + col] -= acc;
+            }
+    }
+    free(G);
+    free(E);
+    return rc;
 }

@@ -15,6 +15,9 @@
  * takes the readings listed in the repository's design notes (generator polynomial, class
  * order, sign order, lexicographic arrangement order).
  *
+ * The last sections add the nearest-point search over the shell union and one pass of
+ * Spherical GPTQ (关键设计 1 and 3).
+ *
  * Indices are up to 96 bits wide; at this interface they travel as (lo, hi) uint64 pairs.
  */
 #ifndef LLVQ_ORACLE_H
@@ -133,6 +136,16 @@ int ora_class_best(ora_codec *c, int32_t m, int64_t j, uint32_t word, const doub
  * value on bad arguments. */
 int64_t ora_search_brute(int32_t m_max, int32_t mode, double scale, int64_t n, const float *X,
                          int8_t *V, double *dot, int32_t nthreads);
+/* ---- Spherical GPTQ, one pass (papernotes 关键设计 3) ----------------------------------
+ * W: fp64 [rows][cols], cols = 24 nb, updated in place (each block ends as its retraction
+ * |w| v / |v|).  U: fp64 [cols][cols], upper triangular with H^-1 = U^T U.  points: int8
+ * [rows][nb][24] (the angular search's v per block); norms: [rows][nb] (|w| when quantized).
+ * Operation order as stated in the definition.  Returns 0, or a negative value. */
+int ora_spherical_gptq(ora_codec *c, int32_t max_shell, int32_t rows, int32_t cols, double *W, const double *U,
+                       int8_t *points, double *norms);
+/* G_B = U_BB^-1 U_B,rest of block b by back substitution, as [24][cols] (zero before the later
+ * columns).  Returns 0, or -1 on bad arguments. */
+int ora_gptq_block_matrix(int32_t cols, const double *U, int32_t b, double *G);
 /* fp16 bits -> double (exact). */
 double ora_half_to_double(uint16_t h);
 
