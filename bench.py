@@ -449,6 +449,73 @@ def search_cpu_baseline(seconds=12.0, max_shell=13, mode=1, scale=0.3):
             "cpu_model": cpu_model()}
 
 
+# ------------------------------------------------------------------ Spherical GPTQ pass
+GPTQ_ROWS, GPTQ_COLS, GPTQ_SHELL = 4096, 4104, 12
+
+
+def gptq_inputs(torch, dev, rows, cols, seed=70):
+    """Gaussian weights and the Cholesky factor U (H^-1 = U^T U) of a synthetic calibration
+    Hessian H = X X^T / n + damping over correlated inputs; U is prepared with library routines
+    (torch.linalg) outside any timed region."""
+    from codebook_free_lattice_b200 import synth
+    g = synth.rng(seed, 4)
+    W = torch.from_numpy(g.standard_normal((rows, cols))).to(dev)
+    X = torch.from_numpy(g.standard_normal((cols, 2 * cols))).to(dev)
+    X = X * torch.linspace(0.3, 2.0, cols, dtype=torch.float64, device=dev)[:, None]
+    X[1:] += 0.5 * X[:-1].clone()
+    H = X @ X.T / X.shape[1]
+    H += 0.05 * H.diagonal().mean() * torch.eye(cols, dtype=torch.float64, device=dev)
+    U = torch.linalg.cholesky(torch.linalg.inv(H)).T.contiguous()
+    return W, U
+
+
+def gptq_throughput(torch, codec, dev, steps, warmup):
+    """One Spherical GPTQ pass over a 4096 x 4104 layer per step (fp64), CUDA events per pass; each
+    pass starts from a fresh copy of the weights (the copy is outside the timed span)."""
+    rows, cols = GPTQ_ROWS, GPTQ_COLS
+    W0, U = gptq_inputs(torch, dev, rows, cols)
+    W = torch.empty_like(W0)
+    nb = cols // 24
+    P = torch.empty((rows, nb, 24), dtype=torch.int8, device=dev)
+    N = torch.empty((rows, nb), dtype=torch.float64, device=dev)
+    ws = None
+    stream = torch.cuda.Stream(device=dev)
+    total = 0.0
+    with torch.cuda.stream(stream):
+        for i in range(warmup + steps):
+            W.copy_(W0)
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            ws = codec.spherical_gptq(W, U, P, N, GPTQ_SHELL, workspace=ws, stream=stream)
+            e.record(stream)
+            e.synchronize()
+            if i >= warmup:
+                total += s.elapsed_time(e) / 1e3
+    if codec.get_error(stream) != 0:
+        raise RuntimeError("llvq_spherical_gptq raised a device flag")
+    t = total / steps
+    upd = rows * 24 * sum(cols - 24 * (b + 1) for b in range(nb))        # propagation FMAs
+    gmat = sum((cols - 24 * (b + 1)) * 276 for b in range(nb))             # back substitution FMAs
+    fmas = rows * nb * SEARCH_FMAS[GPTQ_SHELL] + upd + gmat
+    return {"rows": rows, "cols": cols, "max_shell": GPTQ_SHELL, "ms_per_pass": t * 1e3,
+            "weights_per_s": rows * cols / t, "fp64_fmas_per_pass": fmas,
+            "search_share_of_fmas": rows * nb * SEARCH_FMAS[GPTQ_SHELL] / fmas}
+
+
+def gptq_cpu_baseline(rows=2, cols=960):
+    """The oracle's pass on a bounded sample (rows x cols of the same kind of layer, one core)."""
+    import oracle
+    import torch
+    W, U = gptq_inputs(torch, torch.device("cpu"), rows, cols)
+    oc = oracle.Codec(48)
+    t0 = time.perf_counter()
+    oc.spherical_gptq(W.numpy(), U.numpy(), GPTQ_SHELL)
+    el = time.perf_counter() - t0
+    return {"value": rows * cols / el, "unit": "weights/s", "cores": 1, "kind": "oracle",
+            "sample": f"one pass over a {rows} x {cols} layer ({rows * cols // 24} blocks), {el:.1f} s",
+            "cpu_model": cpu_model()}
+
+
 # ------------------------------------------------------------------ secondary measurements
 SWEEP_CASES = [
     # (name, rows, K, index_bits, batch)
@@ -673,10 +740,11 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--decode-n", type=int, default=28672 * 342,
                     help="indices for the llvq_decode throughput line (default: the 28672x8192 layer)")
-    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "encode", "sweep", "search"],
+    ap.add_argument("--mode", default="gemv", choices=["gemv", "decode", "encode", "sweep", "search", "gptq"],
                     help="decode: time llvq_decode alone (profiling aid); sweep: every layer shape, "
                          "budget and batch against cuBLAS fp16, plus the full 7B stack; search: "
-                         "the nearest-point search on the Gaussian source (throughput and quality)")
+                         "the nearest-point search on the Gaussian source (throughput and quality); gptq: "
+                         "one Spherical GPTQ pass over a 4096 x 4104 layer")
     ap.add_argument("--search-quality", type=int, default=1, help="search mode: run the quality experiment")
     ap.add_argument("--batch", type=int, default=1, help="gemv mode: batch (1 = the metric's workload)")
     ap.add_argument("--rows", type=int, default=4096, help="gemv mode: layer rows (4096 = the metric's workload)")
@@ -717,6 +785,27 @@ def main():
     if args.mode == "sweep":
         if rank == 0:
             sweep(torch, dev)
+        return 0
+    if args.mode == "gptq":
+        if rank == 0:
+            with ClockSampler(torch.cuda.current_device()) as clocks:
+                r = gptq_throughput(torch, codec, dev, args.steps, args.warmup)
+            clk = clocks.summary()
+            props = torch.cuda.get_device_properties(dev)
+            sm = clk.get("sm_mhz") or 1965.0
+            achieved = 2.0 * r["fp64_fmas_per_pass"] / (r["ms_per_pass"] / 1e3) / 1e12
+            peak = props.multi_processor_count * FP64_FMA_PER_SM_CLK * 2 * sm * 1e6 / 1e12
+            line = {"metric": "gptq_weights_per_s", "value": r["weights_per_s"], "unit": "weights/s",
+                    "steps": args.steps, "warmup": args.warmup,
+                    "config": {"workload": f"one Spherical GPTQ pass, {GPTQ_ROWS} x {GPTQ_COLS} Gaussian layer, "
+                                           f"synthetic SPD Hessian, angular search over shells 2..{GPTQ_SHELL}"},
+                    "dtype": "f64", "data": "synthetic", **r, "clocks": clk,
+                    "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                                 "frac": achieved / peak, "traffic": None,
+                                 "peak_source": f"{props.multi_processor_count} SMs x {FP64_FMA_PER_SM_CLK} fp64 FMA/clk x 2 x {sm:.0f} MHz"}}
+            if not args.no_cpu_baseline:
+                line["cpu_baseline"] = gptq_cpu_baseline()
+            print(json.dumps(line), flush=True)
         return 0
     if args.mode == "search":
         if rank == 0:

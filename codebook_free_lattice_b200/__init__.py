@@ -72,6 +72,10 @@ def lib() -> C.CDLL:
         L.llvq_encode.argtypes = [C.c_void_p, C.c_void_p, C.c_int64, C.c_void_p, C.c_int32, C.c_void_p]
         L.llvq_search.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_double, C.c_void_p, C.c_int64,
                                   C.c_void_p, C.c_void_p, C.c_void_p, C.c_int32, C.c_void_p, C.c_void_p]
+        L.llvq_spherical_gptq_workspace.argtypes = [C.c_int32, C.c_int32]
+        L.llvq_spherical_gptq_workspace.restype = C.c_size_t
+        L.llvq_spherical_gptq.argtypes = [C.c_void_p, C.c_int32, C.c_int32, C.c_int32, C.c_void_p, C.c_void_p,
+                                          C.c_void_p, C.c_void_p, C.c_void_p, C.c_size_t, C.c_void_p]
         L.llvq_set_wait_polls.argtypes = [C.c_uint32, C.c_uint32]
         L.llvq_set_wait_polls.restype = None
         L.llvq_last_error_message.argtypes = []
@@ -79,7 +83,7 @@ def lib() -> C.CDLL:
         L.llvq_class_table96.argtypes = [C.c_int32, C.c_void_p, C.c_int64, C.POINTER(C.c_int64)]
         for f in ("llvq_codec_create", "llvq_codec_info", "llvq_decode", "llvq_gemv",
                   "llvq_gemm_smallbatch", "llvq_get_error", "llvq_decode_noalloc", "llvq_class_table96",
-                  "llvq_encode", "llvq_search"):
+                  "llvq_encode", "llvq_search", "llvq_spherical_gptq"):
             getattr(L, f).restype = C.c_int
         _lib = L
     return _lib
@@ -88,7 +92,7 @@ def lib() -> C.CDLL:
 EXPORTED = ("llvq_codec_create", "llvq_codec_destroy", "llvq_codec_info", "llvq_decode",
             "llvq_gemv", "llvq_gemm_smallbatch", "llvq_get_error", "llvq_status_string",
             "llvq_decode_noalloc", "llvq_class_table96", "llvq_last_error_message", "llvq_encode",
-            "llvq_set_wait_polls", "llvq_search")
+            "llvq_set_wait_polls", "llvq_search", "llvq_spherical_gptq", "llvq_spherical_gptq_workspace")
 
 
 def llvq_set_wait_polls(table_polls: int = 0xFFFFFFFF, mma_polls: int = 0xFFFFFFFF) -> None:
@@ -203,6 +207,22 @@ class Codec:
         _check(lib().llvq_search(self._h, max_shell, mode, scale, ptr(X), n, ptr(points), ptr(dots),
                                  ptr(levels), 0 if levels is None else levels.numel(), ptr(codes),
                                  _stream(stream)), "llvq_search")
+
+    def spherical_gptq(self, W, U, points, norms, max_shell: int, workspace=None, stream=None):
+        """One Spherical GPTQ pass in place on W (device fp64 [rows, cols]) with U (device fp64
+        [cols, cols], upper, H^-1 = U^T U); points (device int8 [rows, cols/24, 24]) and norms
+        (device fp64 [rows, cols/24]) receive v and |w| per block.  workspace: a device uint8 tensor
+        of at least spherical_gptq_workspace(rows, cols) bytes (allocated here when None)."""
+        import torch
+        rows, cols = W.shape
+        need = lib().llvq_spherical_gptq_workspace(rows, cols)
+        if workspace is None:
+            workspace = torch.empty(max(int(need), 256), dtype=torch.uint8, device=W.device)
+        _check(lib().llvq_spherical_gptq(self._h, max_shell, rows, cols, C.c_void_p(W.data_ptr()),
+                                         C.c_void_p(U.data_ptr()), C.c_void_p(points.data_ptr()),
+                                         C.c_void_p(norms.data_ptr()), C.c_void_p(workspace.data_ptr()),
+                                         workspace.numel(), _stream(stream)), "llvq_spherical_gptq")
+        return workspace
 
     def gemv(self, w: llvq_weight, x, y, stream=None):
         _check(lib().llvq_gemv(self._h, C.byref(w), C.c_void_p(x.data_ptr()), C.c_void_p(y.data_ptr()),

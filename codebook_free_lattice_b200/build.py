@@ -10,7 +10,7 @@ LIB = os.path.join(HERE, "libllvq.so")
 SOURCES = [os.path.join(CSRC, f) for f in ("llvq.cu", "tables.cpp", "tables96.cpp")]
 HEADERS = [os.path.join(CSRC, f) for f in ("tables.h", "tables96.h", "device_common.cuh", "codec48.cuh", "codec72.cuh",
                                             "codec96.cuh", "encode48.cuh", "encode72.cuh", "encode96.cuh", "kernels.cuh", "kernels_bin48.cuh", "kernels_tc.cuh",
-                                            "kernels_tc48.cuh", "kernels_gemv48.cuh", "search48.cuh", "search48_classes.cuh")] + [os.path.join(ROOT, "include", "llvq.h")]
+                                            "kernels_tc48.cuh", "kernels_gemv48.cuh", "search48.cuh", "search48_classes.cuh", "gptq48.cuh")] + [os.path.join(ROOT, "include", "llvq.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
          "-Xcompiler", "-fPIC", "-Xcompiler", "-pthread", "-shared", "--expt-relaxed-constexpr", "-Xptxas", "-v"]

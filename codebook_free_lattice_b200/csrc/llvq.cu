@@ -27,6 +27,7 @@
 #include "encode72.cuh"
 #include "encode96.cuh"
 #include "search48.cuh"
+#include "gptq48.cuh"
 #include "tables.h"
 #include "tables96.h"
 
@@ -1311,6 +1312,60 @@ llvq_status llvq_search(const llvq_codec *c, int32_t max_shell, int32_t mode, do
         k_search48<0><<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
     else
         k_search48<1><<<(int)grid, kSrThreads, sizeof(SearchSmem48), (cudaStream_t)stream>>>(a);
+    return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
+}
+
+static size_t gptq_align(size_t x) { return (x + 255) & ~(size_t)255; }
+
+size_t llvq_spherical_gptq_workspace(int32_t rows, int32_t cols) {
+    if (rows < 0 || rows > 65535 || cols <= 0 || cols % 24) return 0;
+    const size_t nb = (size_t)cols / 24, r = (size_t)rows;
+    return gptq_align(nb * 24 * (size_t)cols * sizeof(double)) + gptq_align(r * 24 * sizeof(float)) +
+           gptq_align(r * 24) + gptq_align(r * 24 * sizeof(double));
+}
+
+llvq_status llvq_spherical_gptq(const llvq_codec *c, int32_t max_shell, int32_t rows, int32_t cols, double *d_W,
+                                const double *d_U, int8_t *d_points, double *d_norms, void *d_workspace,
+                                size_t workspace_bytes, void *stream) {
+    if (!c) return LLVQ_ERR_ARG;
+    if (c->index_bits != 48) return LLVQ_ERR_UNSUPPORTED;
+    if (max_shell < 2 || max_shell > c->M || rows < 0 || rows > 65535 || cols <= 0 || cols % 24) return LLVQ_ERR_ARG;
+    if (rows == 0) return LLVQ_OK;
+    if (!d_W || !d_U || !d_points || !d_norms || !d_workspace || !aligned(d_W, 8) || !aligned(d_U, 8) ||
+        !aligned(d_norms, 8) || !aligned(d_workspace, 256) || workspace_bytes < llvq_spherical_gptq_workspace(rows, cols))
+        return LLVQ_ERR_ARG;
+    const int nb = cols / 24;
+    unsigned char *ws = (unsigned char *)d_workspace;
+    double *G = (double *)ws;
+    ws += gptq_align((size_t)nb * 24 * cols * sizeof(double));
+    float *Xf = (float *)ws;
+    ws += gptq_align((size_t)rows * 24 * sizeof(float));
+    int8_t *P = (int8_t *)ws;
+    ws += gptq_align((size_t)rows * 24);
+    double *E = (double *)ws;
+    cudaStream_t s = (cudaStream_t)stream;
+    k_gptq_gmat<<<dim3((cols + kGqThreads - 1) / kGqThreads, nb), kGqThreads, 0, s>>>(d_U, G, cols);
+    SearchArgs48 a;
+    a.image = (const SearchImage48 *)c->d_search48;
+    a.max_shell = max_shell;
+    a.mode = LLVQ_SEARCH_ANGULAR;
+    a.scale = 1.0;
+    a.X = Xf;
+    a.n = rows;
+    a.points = P;
+    a.dots = nullptr;
+    a.levels = nullptr;
+    a.n_levels = 0;
+    a.codes = nullptr;
+    a.flags = c->d_flags;
+    const int sgrid = std::min(rows, c->num_sms);
+    for (int b = 0; b < nb; b++) {
+        k_gptq_gather<<<(rows * 24 + 255) / 256, 256, 0, s>>>(d_W, Xf, rows, cols, b);
+        k_search48<0><<<sgrid, kSrThreads, sizeof(SearchSmem48), s>>>(a);
+        k_gptq_retract<<<(rows + 127) / 128, 128, 0, s>>>(d_W, P, E, d_points, d_norms, rows, cols, b);
+        const int rest = cols - 24 * (b + 1);
+        if (rest > 0) k_gptq_update<<<dim3((rest + kGqThreads - 1) / kGqThreads, rows), kGqThreads, 0, s>>>(d_W, E, G, cols, b);
+    }
     return cudaGetLastError() == cudaSuccess ? LLVQ_OK : LLVQ_ERR_CUDA;
 }
 

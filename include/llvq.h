@@ -33,6 +33,7 @@
  */
 #ifndef LLVQ_H
 #define LLVQ_H
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -206,6 +207,32 @@ llvq_status llvq_search(const llvq_codec *codec, int32_t max_shell, int32_t mode
                         const float *d_X, int64_t n, int8_t *d_points, double *d_dots,
                         const double *d_gain_levels, int32_t n_levels, uint8_t *d_gain_codes,
                         void *stream);
+
+/* One pass of Spherical GPTQ over a weight matrix W [rows][cols] on the 48-bit union
+ * (papernotes.org notes, 方法详解 / 关键设计 3 "保模长球面曲率反馈": the shape-gain candidate w~ is
+ * rescaled to the original norm, w^ = (|w| / |w~|) w~, a retraction onto the product of spheres,
+ * and the residual E = w - w^ is propagated to the weights not yet quantized through
+ * U = chol(H^-1)^T).  For each 24-column block B in column order: every row's block w gets its
+ * direction v from the angular search over shells 2..max_shell (the block rounded to fp32), is
+ * replaced by w^ = |w| v / |v| (so the gain drops out), and the later columns move by -E G_B with
+ * G_B = U_BB^-1 U_B,rest (GPTQ's update in block form).  fp64 throughout, in a fixed operation
+ * order (stated in csrc/gptq48.cuh) that makes the result reproducible bit for bit.
+ *   codec: 48-bit (others: LLVQ_ERR_UNSUPPORTED); 2 <= max_shell <= 13.
+ *   d_W: device fp64 [rows][cols], row-major, 8-byte aligned, overwritten: each block ends as
+ *     its retraction; 0 <= rows <= 65535; cols > 0 a multiple of 24.  Finite values only (a
+ *     non-finite row raises LLVQ_FLAG_SEARCH_INPUT and its results are unspecified).
+ *   d_U: device fp64 [cols][cols], upper triangular with H^-1 = U^T U (the caller factors its
+ *     calibration Hessian, e.g. with a library Cholesky); only the upper triangle is read.
+ *   d_points: device int8 [rows][cols / 24][24]: v per block.  d_norms: device fp64
+ *     [rows][cols / 24], 8-byte aligned: |w| per block when it was quantized (the gain a gain
+ *     quantizer would code).
+ *   d_workspace: device, 256-byte aligned, at least llvq_spherical_gptq_workspace(rows, cols)
+ *     bytes (cols^2 x 8 for the block matrices, plus 36 bytes per row), owned by the caller.
+ * Launches 1 + 4 (cols / 24) kernels on `stream`; no allocation. */
+size_t llvq_spherical_gptq_workspace(int32_t rows, int32_t cols);
+llvq_status llvq_spherical_gptq(const llvq_codec *codec, int32_t max_shell, int32_t rows, int32_t cols,
+                                double *d_W, const double *d_U, int8_t *d_points, double *d_norms,
+                                void *d_workspace, size_t workspace_bytes, void *stream);
 
 /* Synchronise `stream`, return the sticky device flags raised since the last call in *flags
  * and clear them.  Returns LLVQ_ERR_DEVICE_FLAG when any flag was set, LLVQ_OK otherwise. */

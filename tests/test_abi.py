@@ -62,12 +62,19 @@ def test_host_argument_checks_without_device(lib):
     assert lib.llvq_gemm_smallbatch(None, None, None, 1, None, None) == L.LLVQ_ERR_ARG
     assert lib.llvq_decode_noalloc(72, None, 16, 1, None, None) == L.LLVQ_ERR_UNSUPPORTED
     assert "48-bit" in L.lib().llvq_last_error_message().decode()
+    assert lib.llvq_search(None, 13, 0, 1.0, None, 1, None, None, None, 0, None, None) == L.LLVQ_ERR_ARG
+    assert lib.llvq_spherical_gptq(None, 13, 1, 24, None, None, None, None, None, 0, None) == L.LLVQ_ERR_ARG
+    # workspace: the block matrices (cols^2 doubles) plus per-row scratch, each part 256-aligned
+    assert lib.llvq_spherical_gptq_workspace(4096, 4104) == 4104 * 4104 * 8 + 4096 * 24 * (4 + 1 + 8)
+    assert lib.llvq_spherical_gptq_workspace(3, 48) == 48 * 48 * 8 + 512 + 256 + 768   # 288, 72, 576 B rounded up
+    for bad in ((-1, 48), (8, 40), (8, 0), (70000, 48)):
+        assert lib.llvq_spherical_gptq_workspace(*bad) == 0
 
 
 def test_flag_values_match_the_header():
     import codebook_free_lattice_b200 as L
     src = open(os.path.join(ROOT, "include", "llvq.h")).read()
-    for name in ("LLVQ_FLAG_INDEX_RANGE", "LLVQ_FLAG_WAIT_TIMEOUT", "LLVQ_FLAG_NOT_CODED"):
+    for name in ("LLVQ_FLAG_INDEX_RANGE", "LLVQ_FLAG_WAIT_TIMEOUT", "LLVQ_FLAG_NOT_CODED", "LLVQ_FLAG_SEARCH_INPUT"):
         val = int(re.search(r"#define\s+" + name + r"\s+(0x[0-9a-fA-F]+)u", src).group(1), 16)
         assert getattr(L, name) == val
 
