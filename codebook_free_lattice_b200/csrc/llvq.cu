@@ -1306,6 +1306,7 @@ llvq_status llvq_search(const llvq_codec *c, int32_t max_shell, int32_t mode, do
     a.n_levels = gains ? n_levels : 0;
     a.codes = gains ? d_gain_codes : nullptr;
     a.flags = c->d_flags;
+    search_list_prefixes(max_shell, a.nal);
     // one CTA per vector, one resident per SM
     const long long grid = std::min<long long>(n, (long long)c->num_sms);
     if (mode == LLVQ_SEARCH_ANGULAR)
@@ -1358,6 +1359,7 @@ llvq_status llvq_spherical_gptq(const llvq_codec *c, int32_t max_shell, int32_t 
     a.n_levels = 0;
     a.codes = nullptr;
     a.flags = c->d_flags;
+    search_list_prefixes(max_shell, a.nal);
     const int sgrid = std::min(rows, c->num_sms);
     for (int b = 0; b < nb; b++) {
         k_gptq_gather<<<(rows * 24 + 255) / 256, 256, 0, s>>>(d_W, Xf, rows, cols, b);

@@ -104,7 +104,9 @@ struct SearchArgs48 {
     int n_levels;
     uint8_t *codes;           // [n] nearest level to <y, v> / |v|, or null
     unsigned *flags;
+    int nal[kSrEvenWeights + 1];   // per class list (odd, even by weight): classes in shells 2..max_shell
 };
+
 
 struct SearchSmem48 {
     double col[kSrWarps][2 * kSrCols][32];        // per warp: entry e of lane l at [e][l]
@@ -116,6 +118,7 @@ struct SearchSmem48 {
     int pad_;
     int word_base[kSrEvenWeights + 1];
     int chunk_base[kSrEvenWeights + 1];
+    int nal[kSrEvenWeights + 1];                  // per class list: how many of its classes lie in shells 2..max_shell
     double red_f[kSrWarps];
     int red_id[kSrWarps];
     uint32_t red_w[kSrWarps];
@@ -161,11 +164,9 @@ constexpr double sr_rsqrt(double x) {
 
 struct SrCrit {
     double nc8;               // Euclidean: -8 c
-    int max_shell;
 };
 
 // criterion value of class J of the compile-time table against this lane's column entries
-// (-inf when its shell is outside the union)
 template <int MODE, int J>
 __device__ __forceinline__ double sr_class(const double (&c)[2 * kSrCols], const SrCrit &cr, int turn,
                                            double wlast) {
@@ -183,7 +184,7 @@ __device__ __forceinline__ double sr_class(const double (&c)[2 * kSrCols], const
     } else {
         f = fma((double)K.m, cr.nc8, V);
     }
-    return K.m <= cr.max_shell ? f : -INFINITY;
+    return f;
 }
 
 // class lists: 0 the odd classes, 1 + w the even classes of codeword weight index w
@@ -194,11 +195,23 @@ constexpr int sr_list_id(int list, int i) {
     return list == 0 ? search_cx::kTable.odd_ids[i] : search_cx::kTable.even_ids[list - 1][i];
 }
 
+// the prefix of each class list (lists are in shell order) that lies in shells 2..max_shell (host)
+inline void search_list_prefixes(int max_shell, int (&nal)[kSrEvenWeights + 1]) {
+    for (int l = 0; l <= kSrEvenWeights; l++) {
+        int n = 0;
+        while (n < sr_list_n(l) && search_cx::kTable.c[sr_list_id(l, n)].m <= max_shell) n++;
+        nal[l] = n;
+    }
+}
+
 // classes B, B + 1, ... of list LST (up to four, ascending ordinals): four independent chains, the
-// best of them (the lower ordinal on equal values), then one comparison with the running best
+// best of them (the lower ordinal on equal values), then one comparison with the running best.
+// A list is in shell order, so the shells of the union are its first nal classes: a quad past them
+// is skipped, and the one that straddles the end masks its classes beyond it.
 template <int MODE, int LST, int B>
-__device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const SrCrit &cr, uint32_t word,
+__device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const SrCrit &cr, int nal, uint32_t word,
                                         bool valid, int turn, double wlast, SrBest &b) {
+    if (B >= nal) return;
     constexpr int N = sr_list_n(LST);
     constexpr int j0 = sr_list_id(LST, B);
     double f = sr_class<MODE, j0>(c, cr, turn, wlast);
@@ -207,10 +220,15 @@ __device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const Sr
         constexpr int j1 = sr_list_id(LST, B + 1);
         constexpr int j2 = sr_list_id(LST, B + 2 < N ? B + 2 : B + 1);
         constexpr int j3 = sr_list_id(LST, B + 3 < N ? B + 3 : B + 1);
-        const double f1 = sr_class<MODE, j1>(c, cr, turn, wlast);
+        double f1 = sr_class<MODE, j1>(c, cr, turn, wlast);
         double f2 = -INFINITY, f3 = -INFINITY;
         if constexpr (B + 2 < N) f2 = sr_class<MODE, j2>(c, cr, turn, wlast);
         if constexpr (B + 3 < N) f3 = sr_class<MODE, j3>(c, cr, turn, wlast);
+        if (B + 3 >= nal) {                          // the list's end falls in this quad
+            f3 = -INFINITY;
+            if (B + 2 >= nal) f2 = -INFINITY;
+            if (B + 1 >= nal) f1 = -INFINITY;
+        }
         int id2 = j2;
         if (f1 > f) { f = f1; id = j1; }
         if (f3 > f2) { f2 = f3; id2 = j3; }
@@ -221,16 +239,16 @@ __device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const Sr
 
 template <int MODE, int LST, int... Q>
 __device__ __forceinline__ void sr_list(std::integer_sequence<int, Q...>, const double (&c)[2 * kSrCols],
-                                        const SrCrit &cr, uint32_t word, bool valid, int turn, double wlast,
-                                        SrBest &b) {
-    (sr_quad<MODE, LST, 4 * Q>(c, cr, word, valid, turn, wlast, b), ...);
+                                        const SrCrit &cr, int nal, uint32_t word, bool valid, int turn,
+                                        double wlast, SrBest &b) {
+    (sr_quad<MODE, LST, 4 * Q>(c, cr, nal, word, valid, turn, wlast, b), ...);
 }
 
 template <int MODE, int LST>
-__device__ __forceinline__ void sr_block(const double (&c)[2 * kSrCols], const SrCrit &cr, uint32_t word,
-                                         bool valid, int turn, double wlast, SrBest &b) {
-    sr_list<MODE, LST>(std::make_integer_sequence<int, (sr_list_n(LST) + 3) / 4>{}, c, cr, word, valid, turn,
-                       wlast, b);
+__device__ __forceinline__ void sr_block(const double (&c)[2 * kSrCols], const SrCrit &cr, const int *nal,
+                                         uint32_t word, bool valid, int turn, double wlast, SrBest &b) {
+    sr_list<MODE, LST>(std::make_integer_sequence<int, (sr_list_n(LST) + 3) / 4>{}, c, cr, nal[LST], word, valid,
+                       turn, wlast, b);
 }
 
 template <int MODE>
@@ -239,10 +257,14 @@ __global__ void __launch_bounds__(kSrThreads, 1) k_search48(const SearchArgs48 a
     SearchSmem48 &S = *reinterpret_cast<SearchSmem48 *>(sr_raw);
     const unsigned FULL = 0xFFFFFFFFu;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SrCrit cr{-8.0 * a.scale, a.max_shell};
+    const SrCrit cr{-8.0 * a.scale};
     if (tid < kSrEvenWeights + 1) {
         S.word_base[tid] = a.image->word_base[tid];
         S.chunk_base[tid] = a.image->chunk_base[tid];
+    }
+    if (tid == 0) {
+#pragma unroll
+        for (int l = 0; l <= kSrEvenWeights; l++) S.nal[l] = a.nal[l];   // constant indices: no local copy
     }
     double(*col)[32] = S.col[warp];
     col[0][lane] = 0.0;                     // count 0 of either set: never rewritten
@@ -320,15 +342,15 @@ __global__ void __launch_bounds__(kSrThreads, 1) k_search48(const SearchArgs48 a
                     if (e > c1) c[e] = d + c[kSrCols + 24 - e];
                     if (e > c2) c[kSrCols + e] = c[24 - e] - d;
                 }
-                sr_block<MODE, 0>(c, cr, word, true, 0, 0.0, best);
+                sr_block<MODE, 0>(c, cr, S.nal, word, true, 0, 0.0, best);
             } else {
                 const int turn = __popc(word & negmask) & 1;
                 switch (wi) {
-                    case 0: sr_block<MODE, 1>(c, cr, word, valid, turn, wlast, best); break;
-                    case 1: sr_block<MODE, 2>(c, cr, word, valid, turn, wlast, best); break;
-                    case 2: sr_block<MODE, 3>(c, cr, word, valid, turn, wlast, best); break;
-                    case 3: sr_block<MODE, 4>(c, cr, word, valid, turn, wlast, best); break;
-                    default: sr_block<MODE, 5>(c, cr, word, valid, turn, wlast, best); break;
+                    case 0: sr_block<MODE, 1>(c, cr, S.nal, word, valid, turn, wlast, best); break;
+                    case 1: sr_block<MODE, 2>(c, cr, S.nal, word, valid, turn, wlast, best); break;
+                    case 2: sr_block<MODE, 3>(c, cr, S.nal, word, valid, turn, wlast, best); break;
+                    case 3: sr_block<MODE, 4>(c, cr, S.nal, word, valid, turn, wlast, best); break;
+                    default: sr_block<MODE, 5>(c, cr, S.nal, word, valid, turn, wlast, best); break;
                 }
             }
         }
