@@ -206,12 +206,15 @@ inline void search_list_prefixes(int max_shell, int (&nal)[kSrEvenWeights + 1]) 
 
 // classes B, B + 1, ... of list LST (up to four, ascending ordinals): four independent chains, the
 // best of them (the lower ordinal on equal values), then one comparison with the running best.
-// A list is in shell order, so the shells of the union are its first nal classes: a quad past them
-// is skipped, and the one that straddles the end masks its classes beyond it.
-template <int MODE, int LST, int B>
+// A list is in shell order, so the shells of the union are its first nal classes.  CHECK (a union
+// short of shell 13): a quad past them is skipped, and the one that straddles the end masks its
+// classes beyond it; without CHECK the quads run straight through.
+template <int MODE, bool CHECK, int LST, int B>
 __device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const SrCrit &cr, int nal, uint32_t word,
                                         bool valid, int turn, double wlast, SrBest &b) {
-    if (B >= nal) return;
+    if constexpr (CHECK) {
+        if (B >= nal) return;
+    }
     constexpr int N = sr_list_n(LST);
     constexpr int j0 = sr_list_id(LST, B);
     double f = sr_class<MODE, j0>(c, cr, turn, wlast);
@@ -224,10 +227,12 @@ __device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const Sr
         double f2 = -INFINITY, f3 = -INFINITY;
         if constexpr (B + 2 < N) f2 = sr_class<MODE, j2>(c, cr, turn, wlast);
         if constexpr (B + 3 < N) f3 = sr_class<MODE, j3>(c, cr, turn, wlast);
-        if (B + 3 >= nal) {                          // the list's end falls in this quad
-            f3 = -INFINITY;
-            if (B + 2 >= nal) f2 = -INFINITY;
-            if (B + 1 >= nal) f1 = -INFINITY;
+        if constexpr (CHECK) {
+            if (B + 3 >= nal) {                      // the list's end falls in this quad
+                f3 = -INFINITY;
+                if (B + 2 >= nal) f2 = -INFINITY;
+                if (B + 1 >= nal) f1 = -INFINITY;
+            }
         }
         int id2 = j2;
         if (f1 > f) { f = f1; id = j1; }
@@ -237,18 +242,19 @@ __device__ __forceinline__ void sr_quad(const double (&c)[2 * kSrCols], const Sr
     if (valid && f >= b.f && sr_better(f, id, word, b.f, b.id, b.w)) { b.f = f; b.id = id; b.w = word; }
 }
 
-template <int MODE, int LST, int... Q>
+template <int MODE, bool CHECK, int LST, int... Q>
 __device__ __forceinline__ void sr_list(std::integer_sequence<int, Q...>, const double (&c)[2 * kSrCols],
                                         const SrCrit &cr, int nal, uint32_t word, bool valid, int turn,
                                         double wlast, SrBest &b) {
-    (sr_quad<MODE, LST, 4 * Q>(c, cr, nal, word, valid, turn, wlast, b), ...);
+    (sr_quad<MODE, CHECK, LST, 4 * Q>(c, cr, nal, word, valid, turn, wlast, b), ...);
 }
 
 template <int MODE, int LST>
 __device__ __forceinline__ void sr_block(const double (&c)[2 * kSrCols], const SrCrit &cr, const int *nal,
-                                         uint32_t word, bool valid, int turn, double wlast, SrBest &b) {
-    sr_list<MODE, LST>(std::make_integer_sequence<int, (sr_list_n(LST) + 3) / 4>{}, c, cr, nal[LST], word, valid,
-                       turn, wlast, b);
+                                         bool full, uint32_t word, bool valid, int turn, double wlast, SrBest &b) {
+    constexpr auto q = std::make_integer_sequence<int, (sr_list_n(LST) + 3) / 4>{};
+    if (full) sr_list<MODE, false, LST>(q, c, cr, nal[LST], word, valid, turn, wlast, b);
+    else sr_list<MODE, true, LST>(q, c, cr, nal[LST], word, valid, turn, wlast, b);
 }
 
 template <int MODE>
@@ -272,6 +278,7 @@ __global__ void __launch_bounds__(kSrThreads, 1) k_search48(const SearchArgs48 a
     const bool act = lane < 24;
     __syncthreads();
     const int n_chunks = kSrOddChunks + S.chunk_base[kSrEvenWeights];
+    const bool full = a.max_shell >= search_cx::kShells;      // every class in the union
 
     for (long long v = blockIdx.x; v < a.n; v += gridDim.x) {
         // ---- warp 0: the input sorted by |y_i| descending (equal values by position) ---------
@@ -342,15 +349,15 @@ __global__ void __launch_bounds__(kSrThreads, 1) k_search48(const SearchArgs48 a
                     if (e > c1) c[e] = d + c[kSrCols + 24 - e];
                     if (e > c2) c[kSrCols + e] = c[24 - e] - d;
                 }
-                sr_block<MODE, 0>(c, cr, S.nal, word, true, 0, 0.0, best);
+                sr_block<MODE, 0>(c, cr, S.nal, full, word, true, 0, 0.0, best);
             } else {
                 const int turn = __popc(word & negmask) & 1;
                 switch (wi) {
-                    case 0: sr_block<MODE, 1>(c, cr, S.nal, word, valid, turn, wlast, best); break;
-                    case 1: sr_block<MODE, 2>(c, cr, S.nal, word, valid, turn, wlast, best); break;
-                    case 2: sr_block<MODE, 3>(c, cr, S.nal, word, valid, turn, wlast, best); break;
-                    case 3: sr_block<MODE, 4>(c, cr, S.nal, word, valid, turn, wlast, best); break;
-                    default: sr_block<MODE, 5>(c, cr, S.nal, word, valid, turn, wlast, best); break;
+                    case 0: sr_block<MODE, 1>(c, cr, S.nal, full, word, valid, turn, wlast, best); break;
+                    case 1: sr_block<MODE, 2>(c, cr, S.nal, full, word, valid, turn, wlast, best); break;
+                    case 2: sr_block<MODE, 3>(c, cr, S.nal, full, word, valid, turn, wlast, best); break;
+                    case 3: sr_block<MODE, 4>(c, cr, S.nal, full, word, valid, turn, wlast, best); break;
+                    default: sr_block<MODE, 5>(c, cr, S.nal, full, word, valid, turn, wlast, best); break;
                 }
             }
         }
