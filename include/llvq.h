@@ -90,7 +90,8 @@ typedef struct {
 } llvq_weight;
 
 /* Build the tables for an index budget (48 -> shells 2..13, 72 -> shells 2..53, 96 -> shells
- * 2..214) on the current device and upload them.  *out is owned by the caller and released with
+ * 2..214) on the current device and upload them (the union of shells m = 2..M and the
+ * shell / class offsets of papernotes.org notes, 关键设计 1 and 2).  *out is owned by the caller and released with
  * llvq_codec_destroy.  Thread-safe to use from several streams afterwards (the codec is
  * read-only except for its sticky flag word).
  * 48 and 72 bits: tables of 76 KB / 11 MB, built in well under a second.  96 bits: 304,649,365
@@ -102,12 +103,14 @@ llvq_status llvq_codec_create(int32_t index_bits, llvq_codec **out);
 void llvq_codec_destroy(llvq_codec *codec);
 
 /* Host query: largest shell M, number of coded points N_M (as lo/hi 64-bit halves) and the
- * number of classes. Any output pointer may be NULL. */
+ * number of classes (papernotes.org notes, 关键设计 1: the union's cumulative size N_M).  Any output
+ * pointer may be NULL. */
 llvq_status llvq_codec_info(const llvq_codec *codec, int32_t *max_shell, uint64_t *n_points_lo,
                             uint64_t *n_points_hi, int64_t *n_classes);
 
 /* Decode n packed words (their index bits; gain bits are ignored) into int8 d_out [n][24]
- * (the lattice coordinates).  d_words: device, n words of word_bytes (8 or 16, matching the
+ * (the lattice coordinates), by the hierarchical bijection of papernotes.org notes, 关键设计 2
+ * (shell, class, then r = I_class mod A, s, I'' by div/mod).  d_words: device, n words of word_bytes (8 or 16, matching the
  * codec), aligned to word_bytes.  d_out: device, 24*n bytes, 8-byte aligned.  n >= 0. */
 llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t word_bytes, int64_t n,
                         int8_t *d_out, void *stream);
@@ -122,13 +125,15 @@ llvq_status llvq_decode(const llvq_codec *codec, const void *d_words, int32_t wo
 llvq_status llvq_encode(const llvq_codec *codec, const int8_t *d_vectors, int64_t n, void *d_words,
                         int32_t word_bytes, void *stream);
 
-/* Fused decode-and-multiply, batch 1: d_y[r] = sum_j scale(r, j) * <v(r, j), x[24 j .. 24 j + 23]>
+/* Fused decode-and-multiply, batch 1 (papernotes.org notes, 关键设计 4: the GPU fused dequantization
+ * kernel; gist.science, Methodik 4): d_y[r] = sum_j scale(r, j) * <v(r, j), x[24 j .. 24 j + 23]>
  * with fp32 accumulation.  d_x: device fp16 [blocks_per_row * 24] (zero beyond cols), 16-byte
  * aligned.  d_y: device fp32 [rows], 4-byte aligned, overwritten. */
 llvq_status llvq_gemv(const llvq_codec *codec, const llvq_weight *w, const void *d_x, float *d_y,
                       void *stream);
 
-/* Fused decode-and-multiply for 1 <= batch <= 16: d_Y[b][r] for activations d_X [batch][nb*24]
+/* Fused decode-and-multiply for 1 <= batch <= 16 (papernotes.org notes, 关键设计 4; the batch-1
+ * call above with a small batch of activations): d_Y[b][r] for activations d_X [batch][nb*24]
  * (fp16, row stride nb*24, zero beyond cols, 16-byte aligned).  Each block is decoded once for the
  * whole batch.  d_Y: device fp32 [batch][rows], overwritten.  48-bit batches of 8 or more run on
  * the tensor cores: decoded 128-row tiles (exact fp16 integers) times a block-diagonal activation
