@@ -73,3 +73,36 @@ def test_committed_record_is_read_when_sources_match(monkeypatch, tmp_path):
     assert bench.measured_traffic() == 123
     line = _line()
     assert line["issue_roofline"]["achieved"] == pytest.approx(456 * 32 / 23.4e-6)
+
+
+def test_search_roofline_line(monkeypatch):
+    """The search line's fp64 roofline: algorithmic FMAs (class-codeword pairs x (groups + 1)) x 2
+    per launch over the launch time, against SMs x 64 FMA lanes x 2 x the clock; the DRAM traffic
+    only from a record of the same launch size."""
+    r = {"n": bench.SEARCH_N, "max_shell": 13, "ms_per_launch": 102.0}
+    monkeypatch.setattr(bench, "search_record", lambda: {"n": bench.SEARCH_N, "traffic_bytes_per_launch": 13_379_840})
+    ro = bench.search_roofline(r, 1965.0, 148)
+    json.dumps(ro)
+    assert ro["bound"] == "alu" and ro["unit"] == "TFLOP/s"
+    assert ro["achieved"] == pytest.approx(2 * 3_805_180 * bench.SEARCH_N / 0.102 / 1e12)
+    assert ro["peak"] == pytest.approx(148 * 64 * 2 * 1965e6 / 1e12)
+    assert ro["frac"] == pytest.approx(ro["achieved"] / ro["peak"]) and 0.2 < ro["frac"] < 0.3
+    assert ro["traffic"] == 13_379_840
+    monkeypatch.setattr(bench, "search_record", lambda: {"n": 1024, "traffic_bytes_per_launch": 1})
+    assert bench.search_roofline(r, 1965.0, 148)["traffic"] is None
+    monkeypatch.setattr(bench, "search_record", lambda: None)
+    assert bench.search_roofline(r, 1965.0, 148)["traffic"] is None
+
+
+def test_search_fma_counts_match_the_class_list():
+    """SEARCH_FMAS (the roofline's algorithmic work) recounted from the oracle's class list: for each
+    class of shells 2..M, its codewords (4096 odd; those of weight k even) x (nonzero groups + 1)."""
+    import oracle
+    words = {0: 1, 8: 759, 12: 2576, 16: 759, 24: 1}
+    o = oracle.Codec(48)
+    for M, fmas in bench.SEARCH_FMAS.items():
+        n = 0
+        for c in o.classes():
+            if c.m <= M:
+                n += (4096 if c.odd else words[c.k]) * (sum(1 for v in c.vals if v) + 1)
+        assert n == fmas, M

@@ -72,3 +72,11 @@ def test_direct_gains_follow_the_norms():
     assert g.shape == norms.shape and (g >= 0).all()
     # |z| sqrt(24) / norm with z ~ N(0, 1): mean sqrt(2/pi) sqrt(24) / norm
     assert abs(g.mean() - np.sqrt(2 / np.pi) * np.sqrt(24) / norms[0, 0]) < 0.05
+
+
+def test_gaussian_blocks_seeded_unit_variance():
+    a = synth.gaussian_blocks(synth.rng(61, 4), 50_000)
+    b = synth.gaussian_blocks(synth.rng(61, 4), 50_000)
+    assert a.dtype == np.float32 and a.shape == (50_000, 24) and np.array_equal(a, b)
+    assert not np.array_equal(a[:100], synth.gaussian_blocks(synth.rng(60, 4), 100))
+    assert abs(a.mean()) < 0.01 and abs(a.var() - 1.0) < 0.01            # N(0, 1), 1.2M samples
