@@ -43,7 +43,10 @@
 // codewords, continues each set past its end there.  The 383 classes of the union are a
 // compile-time table (search48_classes.cuh, checked against the codec's class list when a codec
 // is created), so every class is a straight-line chain of fp64 FMAs on registers with constant
-// steps.  The criterion is a template parameter: angular V / sqrt(16 m), Euclidean (divided by
+// steps, four classes at a time (four independent chains, then one comparison with the running
+// best).  A class list is in shell order, so a union short of shell 13 is a prefix of each list:
+// those launches skip the quads past it, and the full union runs without any check.  The
+// criterion is a template parameter: angular V / sqrt(16 m), Euclidean (divided by
 // 2 c > 0, which keeps the order) V - 8 c m, with m and 1 / sqrt(16 m) compile-time constants.  The CTA
 // keeps the best (criterion, class ordinal, codeword), ties going to the lower class ordinal and
 // then the lower codeword mask, and warp 0 writes the point.
