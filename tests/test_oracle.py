@@ -141,14 +141,22 @@ def test_class_counts(c48, c72):
 
 
 def _class_formula_by_brute_force(c48, m):
-    pts = np.sort(np.abs(oracle.shell_enumerate(m)).astype(np.int8), axis=1)[:, ::-1]
-    uniq, counts = np.unique(pts, axis=0, return_counts=True)
-    keys = {(int(a[0]) % 2, tuple(a.tolist())): int(n) for a, n in zip(uniq, counts)}
+    # a magnitude multiset is its count vector (how many coordinates have |x| = v, v = 0..15),
+    # packed base 25 into one integer; the coset is the parity of the magnitudes
+    mags = np.abs(oracle.shell_enumerate(m)).astype(np.int64)
+    key = np.zeros(mags.shape[0], np.int64)
+    for v in range(int(mags.max()), -1, -1):
+        key = key * 25 + (mags == v).sum(axis=1)
+    uniq, counts = np.unique(key, return_counts=True)
+    found = dict(zip(uniq.tolist(), counts.tolist()))
     for j in range(c48.shell_nclasses(m)):
         cl = c48.shell_class(m, j)
-        a = tuple(v for v, n in sorted(zip(cl.vals, cl.cnts), reverse=True) for _ in range(n))
-        assert keys.pop((int(cl.odd), a)) == cl.size
-    assert not keys
+        k = 0
+        for v in range(int(mags.max()), -1, -1):
+            k = k * 25 + dict(zip(cl.vals, cl.cnts)).get(v, 0)
+        assert found.pop(k) == cl.size
+        assert all(v % 2 == int(cl.odd) for v in cl.vals)
+    assert not found
 
 
 def test_class_formula_by_brute_force(c48):
