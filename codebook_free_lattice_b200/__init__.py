@@ -1,8 +1,9 @@
 """LLVQ (Leech lattice vector quantization) decode and fused decode-and-multiply on B200.
 
 A thin ctypes binding over libllvq.so (the C ABI in include/llvq.h).  Every step of the
-decode and of the products runs in the library's CUDA kernels; this module only marshals
-arguments (device pointers of torch tensors, the current CUDA stream).  There is no CPU
+decode, the products, the encoder, the nearest-point search and the Spherical GPTQ pass runs in
+the library's CUDA kernels; this module only marshals arguments (device pointers of torch
+tensors, the current CUDA stream; a workspace tensor for the GPTQ pass when none is given).  There is no CPU
 fallback: importing the binding fails if libllvq.so is missing or cannot be loaded.
 """
 from __future__ import annotations
