@@ -83,3 +83,40 @@ def test_compile_time_table_equals_the_oracle_classes(tmp_path):
         assert (q, turn2) == (q_ref, t_ref), i
         if not c.odd:
             assert k == c.k
+
+
+PREFIX_PROGRAM = r'''
+#include "search48.cuh"
+#include <cstdio>
+int main() {
+    for (int ms = 2; ms <= 13; ms++) {
+        int nal[6];
+        llvq::search_list_prefixes(ms, nal);
+        std::printf("%d", ms);
+        for (int l = 0; l < 6; l++) std::printf(" %d", nal[l]);
+        std::printf("\n");
+    }
+}
+'''
+
+
+def test_union_is_a_prefix_of_each_class_list(tmp_path):
+    """A search over shells 2..M skips, in each class list (odd; even by codeword weight), the
+    classes past a prefix; the prefix lengths the host computes must be the numbers of classes of
+    shells <= M in that list (so each list must be in shell order)."""
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("no nvcc")
+    src = tmp_path / "prefix.cu"
+    src.write_text(PREFIX_PROGRAM)
+    exe = tmp_path / "prefix"
+    subprocess.run([nvcc, "-std=c++17", "--expt-relaxed-constexpr", "-gencode", "arch=compute_100a,code=sm_100a",
+                    "-I", CSRC, "-o", str(exe), str(src)], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.splitlines()
+    classes = list(oracle.Codec(48).classes())
+    lists = [[c for c in classes if c.odd]] + [[c for c in classes if not c.odd and c.k == w] for w in (0, 8, 12, 16, 24)]
+    for line in out:
+        ms, *nal = map(int, line.split())
+        assert nal == [sum(1 for c in L if c.m <= ms) for L in lists], ms
+    for L in lists:
+        assert [c.m for c in L] == sorted(c.m for c in L)
