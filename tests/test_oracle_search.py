@@ -250,3 +250,38 @@ def test_class_rules_against_assignment_solver(codec):
                     assert abs(d - ref) <= 1e-12 * max(1.0, abs(ref)), (m, j, int(w), d, ref)
                     ntested += 1
     assert ntested > 1500
+
+
+def test_degenerate_targets_against_brute_force(codec):
+    """Targets with exact zeros, repeated magnitudes, integer and half-integer entries and a wide
+    range of scales (many equally good points): the search's criterion value equals brute force's
+    over shell 2 and over shells 2..3 for both criteria, and its answer is a point of the union.
+    Only the value is unique here, so the points themselves are not compared."""
+    rng = np.random.default_rng(61)
+    rows = []
+    for t in range(40):
+        kind = t % 5
+        if kind == 0:
+            x = rng.integers(-3, 4, 24).astype(np.float64)              # integers, many zeros and ties
+        elif kind == 1:
+            x = np.round(rng.standard_normal(24) * 2) / 2                # half-integers
+        elif kind == 2:
+            x = np.repeat(rng.standard_normal(3), 8)                     # three magnitudes, 8 times each
+            x *= rng.choice([-1, 1], 24)
+        elif kind == 3:
+            x = rng.standard_normal(24)
+            x[rng.choice(24, 20, replace=False)] = 0.0                   # sparse
+        else:
+            x = rng.standard_normal(24) * 10.0 ** rng.uniform(-3, 3)     # tiny to large scale
+        rows.append(x)
+    X = np.array(rows, np.float32)
+    for m_max in (2, 3):
+        for mode, scale in ((ANG, 1.0), (EUC, 0.35)):
+            V, d = codec.search(X, m_max, mode, scale, threads=8)
+            Vb, db, _ = oracle.search_brute(X, m_max, mode, scale, threads=8)
+            n = norms(V)
+            assert ((n >= 32) & (n <= 16 * m_max)).all()
+            for v in V:
+                assert oracle.in_leech(v.astype(np.int32))
+            f, fb = objective(mode, scale, X, V), objective(mode, scale, X, Vb)
+            np.testing.assert_allclose(f, fb, rtol=1e-12, atol=1e-12)

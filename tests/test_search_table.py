@@ -9,6 +9,8 @@ that the search's closed form needs derived here from the oracle's multisets:
   a - (next smaller magnitude of the kind, 0 after the last); even parity = (sum / 4) mod 2 when
   k > 0; turn cost = 2 x the smallest 2-mod-4 magnitude.
 (The codec repeats this comparison against its own host tables when it is created.)
+A second check compiles the host helper that gives, per class list, the prefix lying in shells
+2..M (the search skips the rest), and compares it with the oracle's class counts.
 """
 import os
 import shutil
