@@ -10,7 +10,9 @@ Pinned against things that do not share the oracle's Cholesky arithmetic:
   * one block alone is the retraction |w| v / |v| of the angular search, with the same norm;
   * two blocks equal a hand-run: search, retraction, the update through the H-form G, search;
   * the proxy loss tr(D H D^T) of the pass is below that of the same blockwise retraction
-    without feedback, on every seeded instance (a sign or index error in the feedback raises it).
+    without feedback, on every seeded instance (a sign or index error in the feedback raises it);
+  * a diagonal Hessian couples no columns: the block matrices vanish and the pass is the
+    blockwise retraction of the original weights.
 """
 import numpy as np
 import pytest
@@ -111,3 +113,22 @@ def test_feedback_lowers_the_proxy_loss(codec, seed):
     Wr = retraction_only(codec, W, 6)
     loss = lambda D: float(np.trace(D @ H @ D.T))
     assert loss(Wq - W) < loss(Wr - W)
+
+
+def test_diagonal_hessian_has_no_feedback(codec):
+    """A diagonal Hessian couples no columns: every G_B is zero and the pass is exactly the
+    blockwise retraction."""
+    rng = np.random.default_rng(9)
+    cols = 72
+    H = np.diag(rng.uniform(0.5, 3.0, cols))
+    U = chol_factor(H)
+    for b in range(cols // 24):
+        assert (oracle.gptq_block_matrix(U, b) == 0).all()
+    W = rng.standard_normal((10, cols))
+    Wq, P, N = codec.spherical_gptq(W, U, 8)
+    # the later columns reach the search unchanged: the same points as on the original blocks
+    for b in range(cols // 24):
+        V, _ = codec.search(W[:, 24 * b: 24 * b + 24].astype(np.float32), 8, ANG, 1.0)
+        assert (P[:, b] == V).all()
+    np.testing.assert_allclose(N, np.linalg.norm(W.reshape(10, -1, 24), axis=2), rtol=1e-15)
+    np.testing.assert_allclose(Wq, retraction_only(codec, W, 8), rtol=1e-15, atol=0)
